@@ -1,0 +1,164 @@
+"""fp64 CPU oracle for exact scaled dot-product attention -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never loads it and the
+two share no code.
+
+The arithmetic lives in ``attn_oracle.c`` (plain C, fp64, OpenMP over
+(batch, head)); this module compiles it with gcc on first use, widens the
+stored bf16/fp16 bits to fp64 exactly and marshals pointers.  ``brute.py`` holds
+an independent pure-Python statement used to pin the C code on tiny inputs.
+
+Definition (ai6s.net "ops-transformer FlashAttention" article, section
+"标准注意力的致命伤不在算力，在搬运"): O = softmax(scale·Q·Kᵀ + mask)·V, with the
+additive 0/-inf mask of the causal rule (adaptation point 2) and of the real
+KV length (adaptation point 3), LSE = natural log of the row's sum of
+exponentials.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_DP = ctypes.POINTER(ctypes.c_double)
+_IP = ctypes.POINTER(ctypes.c_int)
+
+
+def build(force: bool = False) -> str:
+    """Compile ``liboracle.so`` next to its source (gcc, -O2, no fast-math)."""
+    stale = (not os.path.exists(_LIB_PATH)) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+               "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            lib.oracle_attn_fwd.restype = ctypes.c_int
+            lib.oracle_attn_fwd.argtypes = [
+                _DP, _DP, _DP, _DP, _DP, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
+                _IP, _IP, ctypes.c_int]
+            lib.oracle_attn_kvcache.restype = ctypes.c_int
+            lib.oracle_attn_kvcache.argtypes = [
+                _DP, _DP, _DP, _IP, _IP, _DP, _DP, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int]
+            lib.oracle_lse_combine.restype = ctypes.c_int
+            lib.oracle_lse_combine.argtypes = [_DP, _DP, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, _DP, _DP]
+            lib.oracle_max_threads.restype = ctypes.c_int
+            lib.oracle_set_threads.argtypes = [ctypes.c_int]
+            _lib = lib
+    return _lib
+
+
+def _f64(t) -> np.ndarray:
+    """Widen stored bits to fp64 exactly (bf16/fp16/fp32 all embed in fp64)."""
+    if isinstance(t, torch.Tensor):
+        t = t.detach().to("cpu", torch.float64).contiguous().numpy()
+    return np.ascontiguousarray(t, dtype=np.float64)
+
+
+def _i32(t) -> np.ndarray:
+    if isinstance(t, torch.Tensor):
+        t = t.detach().to("cpu").numpy()
+    return np.ascontiguousarray(t, dtype=np.int32)
+
+
+def _dp(a: np.ndarray):
+    return a.ctypes.data_as(_DP)
+
+
+def _ip(a):
+    return None if a is None else a.ctypes.data_as(_IP)
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def set_threads(n: int) -> None:
+    _load().oracle_set_threads(int(n))
+
+
+def attn_fwd(q, k, v, scale: float, causal: bool, seqlens_k=None, rows=None):
+    """O, LSE of dense attention.
+
+    q [B, Nq, Hq, d], k/v [B, Nk, Hkv, d] (any float dtype; widened exactly).
+    seqlens_k: optional [B] key lengths (keys at or past it are masked).
+    rows: optional list of query-row indices; only those rows are computed
+    (the other entries of the returned arrays are NaN).
+    Returns (o [B, Nq, Hq, d] float64, lse [B, Hq, Nq] float64) numpy arrays.
+    """
+    qd, kd, vd = _f64(q), _f64(k), _f64(v)
+    B, Nq, Hq, d = qd.shape
+    _, Nk, Hkv, _ = kd.shape
+    o = np.full((B, Nq, Hq, d), np.nan)
+    lse = np.full((B, Hq, Nq), np.nan)
+    sl = None if seqlens_k is None else _i32(seqlens_k)
+    rw = None if rows is None else _i32(rows)
+    rc = _load().oracle_attn_fwd(_dp(qd), _dp(kd), _dp(vd), _dp(o), _dp(lse), B, Hq, Hkv, Nq,
+                                 Nk, d, float(scale), int(bool(causal)), _ip(sl), _ip(rw),
+                                 0 if rw is None else len(rw))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_fwd rejected its arguments (rc={rc})")
+    return o, lse
+
+
+def attn_kvcache(q, k_cache, v_cache, cu_seqlens_k, seqlens_k, scale: float, causal: bool):
+    """O, LSE of new query tokens against a packed variable-length KV cache.
+
+    q [B, Nq, Hq, d]; k_cache/v_cache [slots, Hkv, d]; cu_seqlens_k [B+1] slot
+    offsets; seqlens_k [B] filled lengths.  Returns float64 numpy arrays
+    (o [B, Nq, Hq, d], lse [B, Hq, Nq]).
+    """
+    qd, kd, vd = _f64(q), _f64(k_cache), _f64(v_cache)
+    B, Nq, Hq, d = qd.shape
+    Hkv = kd.shape[1]
+    cu, sl = _i32(cu_seqlens_k), _i32(seqlens_k)
+    o = np.full((B, Nq, Hq, d), np.nan)
+    lse = np.full((B, Hq, Nq), np.nan)
+    rc = _load().oracle_attn_kvcache(_dp(qd), _dp(kd), _dp(vd), _ip(cu), _ip(sl), _dp(o),
+                                     _dp(lse), B, Hq, Hkv, Nq, d, float(scale),
+                                     int(bool(causal)))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_kvcache rejected its arguments (rc={rc})")
+    return o, lse
+
+
+def lse_combine(o_parts, lse_parts):
+    """Merge partial results over disjoint key sets.
+
+    o_parts [P, R, d], lse_parts [P, R] -> (o [R, d], lse [R]).
+    """
+    op, lp = _f64(o_parts), _f64(lse_parts)
+    P, R, d = op.shape
+    o = np.empty((R, d))
+    lse = np.empty((R,))
+    rc = _load().oracle_lse_combine(_dp(op), _dp(lp), P, R, d, _dp(o), _dp(lse))
+    if rc != 0:
+        raise ValueError("oracle_lse_combine rejected its arguments")
+    return o, lse
+
+
+__all__ = ["build", "attn_fwd", "attn_kvcache", "lse_combine", "max_threads", "set_threads"]

@@ -1,0 +1,317 @@
+/*
+ * attn_oracle.c -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, obviously correct CPU statement of exact scaled dot-product
+ * attention in fp64.  Only the test suite, the smoke entry and the bench's
+ * CPU-baseline leg may load this library; the CUDA product path never does,
+ * and this file shares no source with it.
+ *
+ * What it computes (one batch b, one query head h, kv head g = h / (Hq/Hkv)):
+ *
+ *   S[i][j] = scale * sum_t q[i][t] * k[j][t]            (the score matrix)
+ *   S[i][j] = -inf  where key j is masked for query i      (additive 0/-inf mask)
+ *   P[i][j] = exp(S[i][j] - m_i) / l_i,  m_i = max_j S[i][j],
+ *             l_i = sum_j exp(S[i][j] - m_i)              (row softmax)
+ *   O[i][:] = sum_j P[i][j] * v[j][:]
+ *   LSE[i]  = m_i + log(l_i)                              (natural log)
+ *
+ * Sources, as printed on the pages:
+ *  - ai6s.net "ops-transformer FlashAttention" article, section "标准注意力的
+ *    致命伤不在算力，在搬运" (the flaw of standard attention is data movement):
+ *    the four steps Q·Kᵀ -> scale -> softmax -> ·V and the N×N matrix S, which
+ *    this oracle materialises on purpose.
+ *  - same article, section "FlashAttention 拆的不是算法，是数据流": the method
+ *    is exact, i.e. its result is this plain definition.
+ *  - same article, section "ops-transformer 里的 FlashAttention 做了什么额外
+ *    的事", points 2 and 3: the causal mask and the variable-length KV cache
+ *    whose real length bounds the keys.
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *  - the mask is additive 0/-inf, so a masked key gets exactly zero weight and
+ *    is never multiplied (a NaN stored in a masked slot cannot leak);
+ *  - causal alignment is bottom-right: query i of Nq attends key j iff
+ *    j <= i + (Lk - Nq), which is the usual top-left rule when Nq == Lk and
+ *    makes the newest query tokens the last rows of a growing KV cache;
+ *  - a row with no visible key gives O = 0 and LSE = -inf;
+ *  - grouped-query heads map contiguously: g = h / (Hq / Hkv).
+ *
+ * Arithmetic: every input is fp64 (the caller widens the bf16/fp16 bits
+ * exactly).  Row sums and output sums use Neumaier compensated summation so
+ * that a softmax row sums to 1 within 1e-12 even over 32K keys.  Build with
+ * -O2 -ffp-contract=off and without -ffast-math.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ---- compensated summation (Neumaier's variant of Kahan) ---------------- */
+typedef struct {
+    double sum;
+    double comp;
+} csum_t;
+
+static void csum_add(csum_t* a, double x) {
+    double t = a->sum + x;
+    if (fabs(a->sum) >= fabs(x))
+        a->comp += (a->sum - t) + x;
+    else
+        a->comp += (x - t) + a->sum;
+    a->sum = t;
+}
+
+static double csum_value(const csum_t* a) { return a->sum + a->comp; }
+
+/* ---- one query head against one key/value head --------------------------
+ * q_rows[r]   : pointer to the d values of the r-th requested query row
+ * row_index[r]: that row's index i in [0, Nq), used by the causal rule
+ * k, v        : key/value row j at k + j*kv_stride (j in [0, Lk))
+ * S           : scratch of nrows*Lk doubles, the materialised score rows
+ * o_rows[r]   : output row (d doubles), lse_out[r]: its log-sum-exp
+ */
+static void attend_head(int nrows, const double* const* q_rows, const int* row_index,
+                        const double* k, const double* v, long kv_stride, int Nq, int Lk,
+                        int d, double scale, int causal, double* const* o_rows,
+                        double* const* lse_out, double* S) {
+    for (int r = 0; r < nrows; ++r) {
+        const double* qi = q_rows[r];
+        const int i = row_index[r];
+        double* Srow = S + (size_t)r * (size_t)(Lk > 0 ? Lk : 1);
+        /* step 1 + 2: scores, then the additive 0 / -inf mask */
+        for (int j = 0; j < Lk; ++j) {
+            int visible = causal ? (j <= i + (Lk - Nq)) : 1;
+            if (!visible) {
+                Srow[j] = -INFINITY;
+                continue;
+            }
+            const double* kj = k + (size_t)j * (size_t)kv_stride;
+            double dot = 0.0;
+            for (int t = 0; t < d; ++t) dot += qi[t] * kj[t];
+            Srow[j] = scale * dot;
+        }
+        /* step 3: row softmax */
+        double m = -INFINITY;
+        for (int j = 0; j < Lk; ++j)
+            if (Srow[j] > m) m = Srow[j];
+        double* oi = o_rows[r];
+        if (m == -INFINITY) { /* no visible key */
+            for (int t = 0; t < d; ++t) oi[t] = 0.0;
+            *lse_out[r] = -INFINITY;
+            continue;
+        }
+        csum_t l = {0.0, 0.0};
+        for (int j = 0; j < Lk; ++j) {
+            if (Srow[j] == -INFINITY) {
+                Srow[j] = 0.0; /* exp(-inf) */
+                continue;
+            }
+            Srow[j] = exp(Srow[j] - m);
+            csum_add(&l, Srow[j]);
+        }
+        const double lsum = csum_value(&l);
+        for (int j = 0; j < Lk; ++j) Srow[j] = Srow[j] / lsum; /* P row */
+        /* step 4: O = P·V, masked keys skipped (their weight is exactly 0) */
+        for (int t = 0; t < d; ++t) {
+            csum_t acc = {0.0, 0.0};
+            for (int j = 0; j < Lk; ++j) {
+                if (Srow[j] == 0.0) continue;
+                csum_add(&acc, Srow[j] * v[(size_t)j * (size_t)kv_stride + t]);
+            }
+            oi[t] = csum_value(&acc);
+        }
+        *lse_out[r] = m + log(lsum);
+    }
+}
+
+static int pick_threads(size_t scratch_bytes_per_thread) {
+#ifdef _OPENMP
+    int n = omp_get_max_threads();
+    const size_t budget = (size_t)8 << 30; /* keep the materialised S under 8 GiB */
+    if (scratch_bytes_per_thread > 0) {
+        size_t cap = budget / scratch_bytes_per_thread;
+        if (cap < 1) cap = 1;
+        if ((size_t)n > cap) n = (int)cap;
+    }
+    return n;
+#else
+    (void)scratch_bytes_per_thread;
+    return 1;
+#endif
+}
+
+/* Threads the oracle will use (OpenMP), for reporting. */
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/*
+ * Dense (optionally key-padded) attention.
+ *   q   [B, Nq, Hq, d]   k, v [B, Nk, Hkv, d]   (row-major, fp64)
+ *   o   [B, Nq, Hq, d]   lse  [B, Hq, Nq]
+ *   seqlens_k: NULL, or [B] real key lengths (<= Nk); keys at or beyond the
+ *              length are masked (the variable-length reading of the KV-cache
+ *              point on the ai6s.net page).
+ *   rows, nrows: NULL/0 computes every query row; otherwise only the listed
+ *              row indices, for every (b, h); other outputs are left alone.
+ * Returns 0, or -1 on bad arguments.
+ */
+int oracle_attn_fwd(const double* q, const double* k, const double* v, double* o, double* lse,
+                    int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale, int causal,
+                    const int* seqlens_k, const int* rows, int nrows) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || d <= 0 || Hq % Hkv != 0) return -1;
+    if (seqlens_k)
+        for (int b = 0; b < B; ++b)
+            if (seqlens_k[b] < 0 || seqlens_k[b] > Nk) return -1;
+    const int nr = rows ? nrows : Nq;
+    if (rows)
+        for (int r = 0; r < nrows; ++r)
+            if (rows[r] < 0 || rows[r] >= Nq) return -1;
+    const int G = Hq / Hkv;
+    const size_t s_bytes = (size_t)(nr > 0 ? nr : 1) * (size_t)(Nk > 0 ? Nk : 1) * sizeof(double);
+    const int nthreads = pick_threads(s_bytes);
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long bh = 0; bh < (long)B * Hq; ++bh) {
+        const int b = (int)(bh / Hq), h = (int)(bh % Hq), g = h / G;
+        const int Lk = seqlens_k ? seqlens_k[b] : Nk;
+        double* S = (double*)malloc(s_bytes);
+        const double** qp = (const double**)malloc(sizeof(double*) * (size_t)(nr > 0 ? nr : 1));
+        double** op = (double**)malloc(sizeof(double*) * (size_t)(nr > 0 ? nr : 1));
+        double** lp = (double**)malloc(sizeof(double*) * (size_t)(nr > 0 ? nr : 1));
+        int* ri = (int*)malloc(sizeof(int) * (size_t)(nr > 0 ? nr : 1));
+        if (!S || !qp || !op || !lp || !ri) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+            for (int r = 0; r < nr; ++r) {
+                const int i = rows ? rows[r] : r;
+                ri[r] = i;
+                qp[r] = q + (((size_t)b * Nq + i) * Hq + h) * (size_t)d;
+                op[r] = o + (((size_t)b * Nq + i) * Hq + h) * (size_t)d;
+                lp[r] = lse + ((size_t)b * Hq + h) * (size_t)Nq + i;
+            }
+            const double* kb = k + ((size_t)b * Nk * Hkv + g) * (size_t)d;
+            const double* vb = v + ((size_t)b * Nk * Hkv + g) * (size_t)d;
+            attend_head(nr, qp, ri, kb, vb, (long)Hkv * d, Nq, Lk, d, scale, causal, op, lp, S);
+        }
+        free(S);
+        free(qp);
+        free(op);
+        free(lp);
+        free(ri);
+    }
+    return err ? -2 : 0;
+}
+
+/*
+ * Attention of new query tokens against a packed, variable-length KV cache.
+ *   q        [B, Nq, Hq, d]          (Nq new tokens per sequence)
+ *   k_cache, v_cache [slots, Hkv, d] sequence b owns slots
+ *            cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1, of which the first
+ *            seqlens_k[b] are filled (the cache is pre-allocated and grows by
+ *            one row per token: ai6s.net article, adaptation point 3)
+ *   o        [B, Nq, Hq, d]          lse [B, Hq, Nq]
+ * Causal means bottom-right: token i of Nq sees keys j <= i + Lk - Nq.
+ */
+int oracle_attn_kvcache(const double* q, const double* k_cache, const double* v_cache,
+                        const int* cu_seqlens_k, const int* seqlens_k, double* o, double* lse,
+                        int B, int Hq, int Hkv, int Nq, int d, double scale, int causal) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || d <= 0 || Hq % Hkv != 0) return -1;
+    int maxlen = 0;
+    for (int b = 0; b < B; ++b) {
+        const int cap = cu_seqlens_k[b + 1] - cu_seqlens_k[b];
+        if (cu_seqlens_k[b] < 0 || cap < 0 || seqlens_k[b] < 0 || seqlens_k[b] > cap) return -1;
+        if (seqlens_k[b] > maxlen) maxlen = seqlens_k[b];
+    }
+    const int G = Hq / Hkv;
+    const size_t s_bytes = (size_t)Nq * (size_t)(maxlen > 0 ? maxlen : 1) * sizeof(double);
+    const int nthreads = pick_threads(s_bytes);
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long bh = 0; bh < (long)B * Hq; ++bh) {
+        const int b = (int)(bh / Hq), h = (int)(bh % Hq), g = h / G;
+        const int Lk = seqlens_k[b];
+        double* S = (double*)malloc(s_bytes);
+        const double** qp = (const double**)malloc(sizeof(double*) * (size_t)Nq);
+        double** op = (double**)malloc(sizeof(double*) * (size_t)Nq);
+        double** lp = (double**)malloc(sizeof(double*) * (size_t)Nq);
+        int* ri = (int*)malloc(sizeof(int) * (size_t)Nq);
+        if (!S || !qp || !op || !lp || !ri) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+            for (int i = 0; i < Nq; ++i) {
+                ri[i] = i;
+                qp[i] = q + (((size_t)b * Nq + i) * Hq + h) * (size_t)d;
+                op[i] = o + (((size_t)b * Nq + i) * Hq + h) * (size_t)d;
+                lp[i] = lse + ((size_t)b * Hq + h) * (size_t)Nq + i;
+            }
+            const double* kb = k_cache + ((size_t)cu_seqlens_k[b] * Hkv + g) * (size_t)d;
+            const double* vb = v_cache + ((size_t)cu_seqlens_k[b] * Hkv + g) * (size_t)d;
+            attend_head(Nq, qp, ri, kb, vb, (long)Hkv * d, Nq, Lk, d, scale, causal, op, lp, S);
+        }
+        free(S);
+        free(qp);
+        free(op);
+        free(lp);
+        free(ri);
+    }
+    return err ? -2 : 0;
+}
+
+/*
+ * Merge of attention results computed over disjoint key sets (the online
+ * softmax correction of the ai6s.net article, section "FlashAttention 拆的不是
+ * 算法，是数据流", applied to whole partial results instead of tiles):
+ *   LSE = log sum_p exp(LSE_p)
+ *   O   = sum_p exp(LSE_p - LSE) * O_p
+ * o_parts [nparts][nrows][d], lse_parts [nparts][nrows]; a part whose LSE is
+ * -inf saw no key and has weight 0.  Rows with no key anywhere: O = 0,
+ * LSE = -inf.
+ */
+int oracle_lse_combine(const double* o_parts, const double* lse_parts, int nparts, int nrows,
+                       int d, double* o, double* lse) {
+    if (nparts <= 0 || nrows < 0 || d <= 0) return -1;
+    for (int r = 0; r < nrows; ++r) {
+        double m = -INFINITY;
+        for (int p = 0; p < nparts; ++p)
+            if (lse_parts[(size_t)p * nrows + r] > m) m = lse_parts[(size_t)p * nrows + r];
+        if (m == -INFINITY) {
+            for (int t = 0; t < d; ++t) o[(size_t)r * d + t] = 0.0;
+            lse[r] = -INFINITY;
+            continue;
+        }
+        csum_t s = {0.0, 0.0};
+        for (int p = 0; p < nparts; ++p) {
+            const double lp = lse_parts[(size_t)p * nrows + r];
+            if (lp != -INFINITY) csum_add(&s, exp(lp - m));
+        }
+        const double total = m + log(csum_value(&s));
+        for (int t = 0; t < d; ++t) {
+            csum_t acc = {0.0, 0.0};
+            for (int p = 0; p < nparts; ++p) {
+                const double lp = lse_parts[(size_t)p * nrows + r];
+                if (lp == -INFINITY) continue;
+                csum_add(&acc, exp(lp - total) * o_parts[((size_t)p * nrows + r) * d + t]);
+            }
+            o[(size_t)r * d + t] = csum_value(&acc);
+        }
+        lse[r] = total;
+    }
+    return 0;
+}
