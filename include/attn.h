@@ -1,0 +1,162 @@
+/*
+ * attn.h -- C ABI of libattn.so: exact scaled dot-product attention on B200
+ * (sm_100a), computed tile by tile with an online softmax so that the N x N
+ * score matrix never reaches device memory.
+ *
+ *   O = softmax(scale * Q K^T + mask) V          LSE = log(sum_j exp(...))
+ *
+ * The operation is the one stated on the ai6s.net article about the CANN
+ * ops-transformer FlashAttention operator: section "标准注意力的致命伤不在算力，
+ * 在搬运" gives the four steps (Q·Kᵀ, scale, softmax, ·V); section
+ * "FlashAttention 拆的不是算法，是数据流" the tiling and the running max / sum
+ * that keep it exact; section "ops-transformer 里的 FlashAttention 做了什么额外
+ * 的事" the fused causal mask (point 2) and the variable-length KV cache whose
+ * tiles stop at each sequence's real length (point 3).  The effectstory.com
+ * article "FlashAttention：IO 感知的精確注意力演算法如何加速 Transformer 訓練
+ * 與推論" (section "什麼是 FlashAttention？核心概念與 IO 感知機制") states the
+ * single-pass schedule: Q, K and V are read once and O is written once.
+ *
+ * Conventions shared by every entry point
+ *  - Pointers are DEVICE memory owned by the caller.  The library never
+ *    allocates, never synchronises and keeps no pointer after returning.
+ *    Work is queued on `stream` (a cudaStream_t; NULL = legacy default).
+ *  - Layouts are row-major with the head dimension d contiguous:
+ *      q, o     [B, Nq, Hq, d]         k, v [B, Nk, Hkv, d]
+ *      lse      [B, Hq, Nq] float32, natural logarithm
+ *    Query head h reads key/value head h / (Hq / Hkv) (grouped-query heads).
+ *  - Element type: bf16 or fp16 (`dtype`), fp32 accumulation.
+ *  - Masks are additive 0 / -inf.  Causal is bottom-right aligned: query i
+ *    sees key j iff j <= i + (Lk - Nq), where Lk is the number of real keys;
+ *    for Nq == Lk this is the usual lower-triangular mask.  A query row with
+ *    no visible key gets O = 0 and LSE = -inf.
+ *  - Requirements: d in {64, 128}; B, Hq, Hkv, Nq > 0; Nk >= 0;
+ *    Hq % Hkv == 0; every pointer 16-byte aligned; a device of compute
+ *    capability 10.0 (B200).  Violations return an error code before any
+ *    work is queued.  Faults during execution surface at the caller's next
+ *    synchronisation.  Every wait inside a kernel is bounded; a wait that
+ *    runs out records an error word, read with attn_get_device_error().
+ *  - Thread safety: calls are independent (tensor maps are built per call
+ *    and passed by value to the kernel).
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { ATTN_BF16 = 0, ATTN_FP16 = 1 } attn_dtype;
+
+enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = -1, /* bad size, pointer, alignment or length */
+    ATTN_ERR_UNSUPPORTED = -2, /* not a B200 / sm_100 device, unknown dtype or d */
+    ATTN_ERR_CUDA = -3,        /* a CUDA call or the kernel launch failed */
+    ATTN_ERR_WORKSPACE = -4,   /* decode workspace missing or too small */
+    ATTN_ERR_TIMEOUT = -5      /* a bounded in-kernel wait ran out (device error word) */
+};
+
+/*
+ * Forward attention (prefill / training forward), dense keys.
+ *   q [B, Nq, Hq, d], k/v [B, Nk, Hkv, d], o [B, Nq, Hq, d] (same dtype),
+ *   lse [B, Hq, Nq] float32.  scale is usually 1/sqrt(d).  causal: 0 or 1.
+ * The tcgen05 kernel stages Q, K and V tiles of 128 rows in shared memory by
+ * TMA, keeps S and the O accumulator in tensor memory and writes only O and
+ * LSE (ai6s.net article, section "FlashAttention 拆的不是算法，是数据流").
+ */
+ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype, void* stream);
+
+/*
+ * Forward attention with per-sequence key lengths: as attn_fwd, plus
+ * seqlens_k (device, int32 [B], each in [0, Nk]).  Keys j >= seqlens_k[b]
+ * are masked (the variable-length KV point 3 of the ai6s.net article); the
+ * K/V rows behind the length may hold anything, NaN included.  Every query
+ * row is computed.  NULL seqlens_k behaves as attn_fwd.
+ */
+ATTN_API int attn_fwd_kpad(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                  int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype,
+                  const int* seqlens_k, void* stream);
+
+/*
+ * Bytes of device workspace that attn_fwd_varlen_kvcache needs for these
+ * sizes.  split_keys: keys per split-K work unit, a multiple of 64, or 0 to
+ * let the library choose (the same rule the decode call applies).  Returns 0
+ * for invalid sizes.
+ */
+ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int d, int max_seqlen_k,
+                                   int split_keys);
+
+/*
+ * Attention of Nq new query tokens per sequence (1 <= Nq <= 16) against a
+ * packed, variable-length KV cache (decode).
+ *   q            [B, Nq, Hq, d]
+ *   k_cache, v_cache [slots, Hkv, d]; sequence b owns slots
+ *                cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1 (device int32 [B+1],
+ *                non-decreasing, cu_seqlens_k[0] >= 0)
+ *   seqlens_k    device int32 [B]: filled length of each sequence,
+ *                0 <= seqlens_k[b] <= cu_seqlens_k[b+1] - cu_seqlens_k[b]
+ *                (the cache is pre-allocated and grows by one row per
+ *                token; only the filled rows are read: ai6s.net article,
+ *                adaptation point 3).  Unfilled slots may hold anything.
+ *   max_seqlen_k host int, >= every seqlens_k[b] (sizes the grid)
+ *   cache_slots  host int, rows of k_cache / v_cache; no copy reads past it
+ *   o [B, Nq, Hq, d], lse [B, Hq, Nq] float32
+ *   causal       bottom-right within the chunk: token i sees keys
+ *                j <= i + seqlens_k[b] - Nq
+ *   workspace    device buffer of at least attn_decode_workspace_bytes(...)
+ *                bytes (256-byte aligned), owned by the caller; holds the
+ *                split-K partial results and their counters.  Calls that
+ *                share one workspace must not overlap on the GPU.
+ *   split_keys   keys per split (multiple of 64) or 0 for automatic.
+ * Each (sequence, kv head, split) work unit streams its keys once with
+ * 128-bit loads, scores the Hq/Hkv query heads that share the kv head, and
+ * keeps a running max and sum; the last unit of a (sequence, kv head) merges
+ * the partial results in a fixed order: LSE = log sum_i exp(LSE_i),
+ * O = sum_i exp(LSE_i - LSE) O_i.
+ */
+ATTN_API int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_cache,
+                            const int* cu_seqlens_k, const int* seqlens_k, int max_seqlen_k,
+                            int cache_slots, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int d,
+                            float scale, int causal, int dtype, void* workspace,
+                            size_t workspace_bytes, int split_keys, void* stream);
+
+/* Human-readable text of a status code (static storage). */
+ATTN_API const char* attn_status_string(int status);
+
+/*
+ * Read and clear the device error word of the current device after
+ * synchronising `stream`.  *code receives 0 when every bounded wait since the
+ * last call completed, otherwise a non-zero code naming the wait that ran out
+ * (kernel id * 16 + wait site).  Returns ATTN_OK, or ATTN_ERR_CUDA.
+ */
+ATTN_API int attn_get_device_error(int* code, void* stream);
+
+/*
+ * Self-test of the bounded waits: launches the forward kernel on a tiny
+ * problem with its loader told to skip the first arrival, with wait limit
+ * `limit_ms`.  No copy is issued, so nothing is in flight when the waits give
+ * up; the kernel frees its tensor memory and returns.  The status of the
+ * launch is returned; the timeout shows up in attn_get_device_error().
+ * q/k/v/o/lse as for attn_fwd with B = Hq = Hkv = 1, Nq = Nk = 128, d = 64.
+ */
+ATTN_API int attn_selftest_watchdog(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int limit_ms, void* stream);
+
+/* Library version string. */
+ATTN_API const char* attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

@@ -1,0 +1,185 @@
+"""ctypes binding of libattn.so (argument marshalling only).
+
+Every step of the attention path runs in the CUDA library; this module only
+allocates outputs with PyTorch, passes ``data_ptr()`` values and the current
+stream, and turns status codes into exceptions.  There is no CPU fallback: if
+the library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "attn.h")
+
+ATTN_BF16, ATTN_FP16 = 0, 1
+STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "CUDA error",
+          -4: "workspace", -5: "timeout"}
+ERR_FWD_BASE, ERR_DECODE_BASE = 16, 32
+
+_lock = threading.Lock()
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({status})")
+        self.status = status
+
+
+def load_library():
+    """Load libattn.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with `python -m io_aware_exact_29_b200.build`")
+            lib = ctypes.CDLL(LIB_PATH)
+            vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+            lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
+            lib.attn_fwd.restype = i
+            lib.attn_fwd_kpad.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp, vp]
+            lib.attn_fwd_kpad.restype = i
+            lib.attn_decode_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
+            lib.attn_decode_workspace_bytes.restype = sz
+            lib.attn_fwd_varlen_kvcache.argtypes = [vp, vp, vp, vp, vp, i, i, vp, vp, i, i, i, i,
+                                                    i, f, i, i, vp, sz, i, vp]
+            lib.attn_fwd_varlen_kvcache.restype = i
+            lib.attn_status_string.argtypes = [i]
+            lib.attn_status_string.restype = ctypes.c_char_p
+            lib.attn_get_device_error.argtypes = [ctypes.POINTER(i), vp]
+            lib.attn_get_device_error.restype = i
+            lib.attn_selftest_watchdog.argtypes = [vp, vp, vp, vp, vp, i, vp]
+            lib.attn_selftest_watchdog.restype = i
+            lib.attn_version.restype = ctypes.c_char_p
+            _lib = lib
+    return _lib
+
+
+def header_functions():
+    """Names of the functions that include/attn.h declares."""
+    with open(HEADER_PATH) as fh:
+        text = fh.read()
+    return sorted(set(re.findall(r"^ATTN_API\s+[A-Za-z_][\w \*]*?\b(attn_\w+)\s*\(", text, re.M)))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return ATTN_BF16
+    if t.dtype == torch.float16:
+        return ATTN_FP16
+    raise TypeError(f"unsupported dtype {t.dtype}: bf16 or fp16")
+
+
+def _stream_ptr(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise AttnError(fn, status)
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def attn_fwd(q, k, v, scale=None, causal=False, seqlens_k=None, out=None, lse=None,
+             stream=None):
+    """Exact attention forward.
+
+    q [B, Nq, Hq, d], k/v [B, Nk, Hkv, d] (bf16/fp16, CUDA, contiguous);
+    seqlens_k: optional int32 [B] key lengths.  Returns (o, lse) with
+    o [B, Nq, Hq, d] and lse [B, Hq, Nq] float32.
+    """
+    lib = load_library()
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    if scale is None:
+        scale = float(d) ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    st = _stream_ptr(stream)
+    if seqlens_k is None:
+        rc = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                          lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
+                          _dtype_code(q), st)
+        _check("attn_fwd", rc)
+    else:
+        _dev(seqlens_k, "seqlens_k")
+        if seqlens_k.dtype != torch.int32:
+            raise TypeError("seqlens_k must be int32")
+        rc = lib.attn_fwd_kpad(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
+                               int(bool(causal)), _dtype_code(q), seqlens_k.data_ptr(), st)
+        _check("attn_fwd_kpad", rc)
+    return out, lse
+
+
+def decode_workspace_bytes(B, Hq, Hkv, Nq, d, max_seqlen_k, split_keys=0) -> int:
+    return int(load_library().attn_decode_workspace_bytes(B, Hq, Hkv, Nq, d, max_seqlen_k,
+                                                           split_keys))
+
+
+def attn_fwd_varlen_kvcache(q, k_cache, v_cache, cu_seqlens_k, seqlens_k, max_seqlen_k,
+                            scale=None, causal=False, split_keys=0, workspace=None, out=None,
+                            lse=None, stream=None):
+    """Decode attention against a packed variable-length KV cache.
+
+    q [B, Nq, Hq, d]; k_cache/v_cache [slots, Hkv, d]; cu_seqlens_k int32
+    [B+1]; seqlens_k int32 [B]; max_seqlen_k (host int) >= every length.
+    Returns (o [B, Nq, Hq, d], lse [B, Hq, Nq] float32).
+    """
+    lib = load_library()
+    B, Nq, Hq, d = q.shape
+    slots, Hkv, _ = k_cache.shape
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"),
+                 (cu_seqlens_k, "cu_seqlens_k"), (seqlens_k, "seqlens_k")):
+        _dev(t, n)
+    if scale is None:
+        scale = float(d) ** -0.5
+    need = decode_workspace_bytes(B, Hq, Hkv, Nq, d, max_seqlen_k, split_keys)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    rc = lib.attn_fwd_varlen_kvcache(
+        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cu_seqlens_k.data_ptr(),
+        seqlens_k.data_ptr(), int(max_seqlen_k), int(slots), out.data_ptr(), lse.data_ptr(), B,
+        Hq, Hkv, Nq, d, float(scale), int(bool(causal)), _dtype_code(q), workspace.data_ptr(),
+        workspace.numel(), int(split_keys), _stream_ptr(stream))
+    _check("attn_fwd_varlen_kvcache", rc)
+    return out, lse
+
+
+def get_device_error(stream=None) -> int:
+    code = ctypes.c_int(0)
+    _check("attn_get_device_error",
+           load_library().attn_get_device_error(ctypes.byref(code), _stream_ptr(stream)))
+    return code.value
+
+
+def selftest_watchdog(q, k, v, out, lse, limit_ms=200, stream=None):
+    rc = load_library().attn_selftest_watchdog(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                               out.data_ptr(), lse.data_ptr(), int(limit_ms),
+                                               _stream_ptr(stream))
+    _check("attn_selftest_watchdog", rc)
+
+
+def version() -> str:
+    return load_library().attn_version().decode()

@@ -1,0 +1,299 @@
+// attn_api.cu -- the C ABI declared in include/attn.h: argument validation,
+// tile/split selection, TMA tensor-map encoding and kernel launches.  No
+// allocation, no synchronisation (except attn_get_device_error, which is
+// documented to synchronise).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "attn_internal.h"
+
+namespace attn {
+
+// One device error word per device that loads the library; kernels record
+// the first bounded wait that ran out here.
+static __device__ unsigned g_device_error = 0u;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultLimitNs = 2000000000ull;  // 2 s per wait
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+int g_dev_state[kMaxDevices] = {0};  // 0 unknown, 1 supported, -1 unsupported
+unsigned* g_err_addr[kMaxDevices] = {nullptr};
+
+EncodeTiledFn encode_fn() {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    return g_encode;
+}
+
+// Current device: 1 if it is a compute-capability 10.0 part, -1 if not, 0 on error.
+int check_device(int* dev_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    *dev_out = dev;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_dev_state[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return 0;
+        g_dev_state[dev] = (major == 10 && minor == 0) ? 1 : -1;
+        if (g_dev_state[dev] == 1) {
+            void* addr = nullptr;
+            if (cudaGetSymbolAddress(&addr, g_device_error) != cudaSuccess) {
+                g_dev_state[dev] = 0;
+                return 0;
+            }
+            g_err_addr[dev] = static_cast<unsigned*>(addr);
+        }
+    }
+    return g_dev_state[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Tiled map over a row-major tensor whose dims are given innermost first;
+// strides in bytes for dims 1..rank-1; 128-byte swizzle; zero fill outside.
+bool encode_map(CUtensorMap* m, int dtype, const void* base, int rank, const uint64_t* dims,
+                const uint64_t* strides, const uint32_t* box) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[5], gstride[4];
+    cuuint32_t bdim[5], estride[5];
+    for (int i = 0; i < rank; ++i) {
+        gdim[i] = dims[i];
+        bdim[i] = box[i];
+        estride[i] = 1;
+    }
+    for (int i = 0; i < rank - 1; ++i) gstride[i] = strides[i];
+    const CUtensorMapDataType dt =
+        dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void*>(base), gdim, gstride, bdim, estride,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// [B, N, H, d] tensor, box of 64 columns x 1 head x 128 rows x 1 batch.
+bool map_bnhd(CUtensorMap* m, int dtype, const void* base, int B, int N, int H, int d) {
+    const uint64_t dims[4] = {(uint64_t)d, (uint64_t)H, (uint64_t)N, (uint64_t)B};
+    const uint64_t strides[3] = {(uint64_t)d * 2, (uint64_t)H * d * 2, (uint64_t)N * H * d * 2};
+    const uint32_t box[4] = {64, 1, 128, 1};
+    return encode_map(m, dtype, base, 4, dims, strides, box);
+}
+
+int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+               int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype,
+               const int* seqlens_k, void* stream, int inject, unsigned long long limit_ns) {
+    if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk < 0 || Hq % Hkv != 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (B > 65535 || Hq > 65535) return ATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    if (!q || !o || !lse || !aligned16(q) || !aligned16(o) || !aligned16(lse))
+        return ATTN_ERR_INVALID_ARG;
+    if (Nk > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return ATTN_ERR_INVALID_ARG;
+    if (seqlens_k && (reinterpret_cast<uintptr_t>(seqlens_k) & 3u)) return ATTN_ERR_INVALID_ARG;
+    int dev = 0;
+    const int st = check_device(&dev);
+    if (st == 0) return ATTN_ERR_CUDA;
+    if (st < 0) return ATTN_ERR_UNSUPPORTED;
+
+    FwdMaps maps;
+    // With no keys at all the K/V maps are never read; point them at Q.
+    const void* kb = Nk > 0 ? k : q;
+    const void* vb = Nk > 0 ? v : q;
+    const int nk_map = Nk > 0 ? Nk : Nq;
+    const int hkv_map = Nk > 0 ? Hkv : Hq;
+    if (!map_bnhd(&maps.q, dtype, q, B, Nq, Hq, d) ||
+        !map_bnhd(&maps.k, dtype, kb, B, nk_map, hkv_map, d) ||
+        !map_bnhd(&maps.v, dtype, vb, B, nk_map, hkv_map, d) ||
+        !map_bnhd(&maps.o, dtype, o, B, Nq, Hq, d))
+        return ATTN_ERR_INVALID_ARG;
+
+    FwdParams p{};
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.G = Hq / Hkv;
+    p.n_qtiles = (Nq + 127) / 128;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.seqlens_k = Nk > 0 ? seqlens_k : nullptr;
+    p.lse = lse;
+    p.limit_ns = limit_ns;
+    p.inject = inject;
+    p.err = g_err_addr[dev];
+    // seqlens_k with Nk == 0 means every length is 0: same as no keys.
+    cudaError_t e = launch_fwd(maps, p, d, dtype == ATTN_BF16, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+unsigned* device_error_word() {
+    int dev = 0;
+    if (check_device(&dev) != 1) return nullptr;
+    return g_err_addr[dev];
+}
+
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype, void* stream) {
+    return fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, nullptr,
+                      stream, 0, kDefaultLimitNs);
+}
+
+int attn_fwd_kpad(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                  int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype,
+                  const int* seqlens_k, void* stream) {
+    return fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, seqlens_k,
+                      stream, 0, kDefaultLimitNs);
+}
+
+int attn_selftest_watchdog(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int limit_ms, void* stream) {
+    if (limit_ms <= 0 || limit_ms > 10000) return ATTN_ERR_INVALID_ARG;
+    return fwd_common(q, k, v, o, lse, 1, 1, 1, 128, 128, 64, 0.125f, 0, ATTN_BF16, nullptr,
+                      stream, 1, (unsigned long long)limit_ms * 1000000ull);
+}
+
+size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int d, int max_seqlen_k,
+                                   int split_keys) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq <= 0 || Nq > 16) return 0;
+    if ((d != 64 && d != 128) || max_seqlen_k < 0) return 0;
+    if (split_keys < 0 || (split_keys % 64) != 0) return 0;
+    return decode_layout(B, Hq, Hkv, Nq, d, max_seqlen_k, split_keys).total;
+}
+
+int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_cache,
+                            const int* cu_seqlens_k, const int* seqlens_k, int max_seqlen_k,
+                            int cache_slots, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                            int d, float scale, int causal, int dtype, void* workspace,
+                            size_t workspace_bytes, int split_keys, void* stream) {
+    if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq <= 0 || Nq > 16)
+        return ATTN_ERR_INVALID_ARG;
+    if (B > 65535 || Hkv > 65535 || max_seqlen_k < 0 || cache_slots <= 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (split_keys < 0 || (split_keys % 64) != 0) return ATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    if (!q || !k_cache || !v_cache || !cu_seqlens_k || !seqlens_k || !o || !lse)
+        return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+        !aligned16(lse) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) ||
+        (reinterpret_cast<uintptr_t>(seqlens_k) & 3u))
+        return ATTN_ERR_INVALID_ARG;
+    int dev = 0;
+    const int st = check_device(&dev);
+    if (st == 0) return ATTN_ERR_CUDA;
+    if (st < 0) return ATTN_ERR_UNSUPPORTED;
+
+    const DecodeLayout lay = decode_layout(B, Hq, Hkv, Nq, d, max_seqlen_k, split_keys);
+    if (lay.max_splits * lay.n_mgroups > 2147483647 / 2) return ATTN_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < lay.total ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return ATTN_ERR_WORKSPACE;
+
+    CUtensorMap kmap, vmap;
+    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)Hkv, (uint64_t)cache_slots};
+    const uint64_t strides[2] = {(uint64_t)d * 2, (uint64_t)Hkv * d * 2};
+    const uint32_t box[3] = {64, 1, 64};
+    if (!encode_map(&kmap, dtype, k_cache, 3, dims, strides, box) ||
+        !encode_map(&vmap, dtype, v_cache, 3, dims, strides, box))
+        return ATTN_ERR_INVALID_ARG;
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    DecodeParams p{};
+    p.q = q;
+    p.o = o;
+    p.lse = lse;
+    p.cu_seqlens_k = cu_seqlens_k;
+    p.seqlens_k = seqlens_k;
+    p.part_o = reinterpret_cast<float*>(ws + lay.part_o_off);
+    p.part_lse = reinterpret_cast<float*>(ws + lay.part_lse_off);
+    p.counters = reinterpret_cast<unsigned*>(ws + lay.counters_off);
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nq = Nq;
+    p.G = Hq / Hkv;
+    p.rows = Nq * p.G;
+    p.n_mgroups = lay.n_mgroups;
+    p.split_keys = lay.split_keys;
+    p.max_splits = lay.max_splits;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.limit_ns = kDefaultLimitNs;
+    p.err = g_err_addr[dev];
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(p.counters, 0, (size_t)B * Hkv * lay.n_mgroups * sizeof(unsigned), s) !=
+        cudaSuccess)
+        return ATTN_ERR_CUDA;
+    cudaError_t e = launch_decode(kmap, vmap, p, d, dtype == ATTN_BF16, s);
+    return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+const char* attn_status_string(int status) {
+    switch (status) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_INVALID_ARG: return "invalid argument";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported device, dtype or head dimension";
+        case ATTN_ERR_CUDA: return "CUDA error";
+        case ATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case ATTN_ERR_TIMEOUT: return "a bounded in-kernel wait ran out";
+        default: return "unknown status";
+    }
+}
+
+int attn_get_device_error(int* code, void* stream) {
+    if (!code) return ATTN_ERR_INVALID_ARG;
+    int dev = 0;
+    const int st = check_device(&dev);
+    if (st == 0) return ATTN_ERR_CUDA;
+    if (st < 0) return ATTN_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
+    unsigned v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    *code = (int)v;
+    return ATTN_OK;
+}
+
+const char* attn_version(void) { return "attn-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

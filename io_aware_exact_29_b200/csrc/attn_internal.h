@@ -1,0 +1,72 @@
+// attn_internal.h -- parameter blocks shared by the C-ABI layer and the
+// kernel translation units (host and device).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace attn {
+
+// Device error word codes: kernel id * 16 + wait site.
+enum : unsigned {
+    kErrFwdBase = 1 * 16,
+    kErrDecodeBase = 2 * 16,
+};
+
+struct FwdParams {
+    int B, Hq, Hkv, Nq, Nk;
+    int G;            // Hq / Hkv
+    int n_qtiles;     // ceil(Nq / 128)
+    int causal;
+    float scale_log2; // scale * log2(e)
+    const int* seqlens_k;  // [B] or nullptr
+    float* lse;            // [B, Hq, Nq]
+    unsigned long long limit_ns;
+    int inject;       // self-test: the loader skips everything
+    unsigned* err;    // device error word
+};
+
+struct FwdMaps {
+    CUtensorMap q, k, v, o;
+};
+
+// Launch the forward kernel for head dim d (64/128) and element type.
+cudaError_t launch_fwd(const FwdMaps& maps, const FwdParams& p, int d, bool bf16,
+                       cudaStream_t stream);
+
+struct DecodeParams {
+    const void* q;         // [B, Nq, Hq, d]
+    void* o;               // [B, Nq, Hq, d]
+    float* lse;            // [B, Hq, Nq]
+    const int* cu_seqlens_k;
+    const int* seqlens_k;
+    float* part_o;         // [B, Hkv, n_mgroups, max_splits, 16, d] fp32
+    float* part_lse;       // [B, Hkv, n_mgroups, max_splits, 16]
+    unsigned* counters;    // [B, Hkv, n_mgroups]
+    int B, Hq, Hkv, Nq, G;
+    int rows;              // Nq * G query rows per (sequence, kv head)
+    int n_mgroups;         // ceil(rows / 16)
+    int split_keys;        // multiple of 64
+    int max_splits;
+    int causal;
+    float scale_log2;
+    unsigned long long limit_ns;
+    unsigned* err;
+};
+
+struct DecodeLayout {
+    int split_keys, max_splits, n_mgroups;
+    size_t part_o_off, part_lse_off, counters_off, total;
+};
+
+DecodeLayout decode_layout(int B, int Hq, int Hkv, int Nq, int d, int max_seqlen_k,
+                           int split_keys);
+
+cudaError_t launch_decode(const CUtensorMap& kmap, const CUtensorMap& vmap,
+                          const DecodeParams& p, int d, bool bf16, cudaStream_t stream);
+
+// Address of the device error word on the current device.
+unsigned* device_error_word();
+
+}  // namespace attn

@@ -1,0 +1,105 @@
+"""The C-ABI library loads without a GPU and exports what include/attn.h
+declares; host-side validation rejects bad arguments before any CUDA call."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+from io_aware_exact_29_b200 import attn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_header_declares_the_boundary():
+    names = attn.header_functions()
+    for n in ("attn_fwd", "attn_fwd_kpad", "attn_fwd_varlen_kvcache",
+              "attn_decode_workspace_bytes", "attn_status_string", "attn_get_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = attn.load_library()
+    for n in attn.header_functions():
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", attn.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(attn.header_functions()) <= exported
+
+
+def test_library_is_built_for_sm100a():
+    # the build passes exactly one gencode, for sm_100a
+    from io_aware_exact_29_b200 import build
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def test_status_strings():
+    lib = attn.load_library()
+    assert lib.attn_status_string(0) == b"ok"
+    assert b"invalid" in lib.attn_status_string(-1)
+    assert lib.attn_status_string(-5)
+    assert attn.version().startswith("attn-b200")
+
+
+P = 1 << 20  # a fake, 16-byte aligned address: validation fails before it is used
+
+
+@pytest.mark.parametrize("args,expect", [
+    # (q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype)
+    ((0, P, P, P, P, 1, 1, 1, 1, 1, 64, 0.125, 0, 0), -1),   # null q
+    ((P + 2, P, P, P, P, 1, 1, 1, 1, 1, 64, 0.125, 0, 0), -1),  # misaligned q
+    ((P, P, P, P, P, 1, 3, 2, 1, 1, 64, 0.125, 0, 0), -1),   # Hq % Hkv != 0
+    ((P, P, P, P, P, 0, 1, 1, 1, 1, 64, 0.125, 0, 0), -1),   # B = 0
+    ((P, P, P, P, P, 1, 1, 1, 0, 1, 64, 0.125, 0, 0), -1),   # Nq = 0
+    ((P, P, P, P, P, 1, 1, 1, 1, -1, 64, 0.125, 0, 0), -1),  # Nk < 0
+    ((P, P, P, P, P, 1, 1, 1, 1, 1, 96, 0.125, 0, 0), -2),   # d = 96
+    ((P, P, P, P, P, 1, 1, 1, 1, 1, 64, 0.125, 0, 7), -2),   # dtype
+    ((P, P, P, P, P, 1, 1, 1, 1, 1, 64, -1.0, 0, 0), -1),    # scale <= 0
+    ((P, P, P, P, P, 1, 1, 1, 1, 1, 64, float("nan"), 0, 0), -1),
+])
+def test_fwd_rejects_bad_arguments(args, expect):
+    lib = attn.load_library()
+    assert lib.attn_fwd(*args, None) == expect
+
+
+def test_decode_rejects_bad_arguments():
+    lib = attn.load_library()
+    base = dict(q=P, k=P, v=P, cu=P, sl=P, maxl=100, slots=100, o=P, lse=P, B=2, Hq=8, Hkv=2,
+                Nq=1, d=128, scale=0.088, causal=0, dtype=0, ws=P, wsb=1 << 30, split=0)
+
+    def call(**kw):
+        a = dict(base, **kw)
+        return lib.attn_fwd_varlen_kvcache(a["q"], a["k"], a["v"], a["cu"], a["sl"], a["maxl"],
+                                           a["slots"], a["o"], a["lse"], a["B"], a["Hq"],
+                                           a["Hkv"], a["Nq"], a["d"], a["scale"], a["causal"],
+                                           a["dtype"], a["ws"], a["wsb"], a["split"], None)
+
+    assert call(Nq=17) == -1         # at most 16 new tokens
+    assert call(Nq=0) == -1
+    assert call(Hq=6, Hkv=4) == -1
+    assert call(split=100) == -1     # split not a multiple of 64
+    assert call(slots=0) == -1
+    assert call(cu=P + 2) == -1
+    assert call(d=80) == -2
+    # host-only size query (no GPU needed)
+    need = attn.decode_workspace_bytes(2, 8, 2, 1, 128, 100)
+    assert need > 0
+    assert attn.decode_workspace_bytes(2, 8, 2, 17, 128, 100) == 0
+    assert attn.decode_workspace_bytes(2, 8, 2, 1, 128, 100, split_keys=96) == 0
+
+
+def test_decode_workspace_accounting():
+    # B=32, Hkv=8 one row group (8 query rows), auto split of 1024 keys over
+    # 32768 keys: 32 splits x 16 padded rows x (128 + 1) floats + counters
+    n = attn.decode_workspace_bytes(32, 64, 8, 1, 128, 32768)
+    units, splits = 32 * 8, 32
+    expect = units * splits * 16 * 128 * 4 + units * splits * 16 * 4 + units * 4
+    assert expect <= n <= expect + 3 * 256
+
+
+def test_python_binding_fails_loudly_without_cuda_tensors():
+    import torch
+    q = torch.zeros(1, 128, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        attn.attn_fwd(q, q, q)

@@ -1,0 +1,113 @@
+"""KV-cache decode kernel (split-K over a packed variable-length cache)
+against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from io_aware_exact_29_b200 import attn
+from io_aware_exact_29_b200.workloads import DECODE_CASES, DecodeCase, kvcache_inputs
+from tests.parity import compare
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(inp, case, split_keys=0, max_seqlen=None):
+    dev = {k: v.cuda() for k, v in inp.items()}
+    ml = int(inp["seqlens_k"].max().item()) if max_seqlen is None else max_seqlen
+    o, lse = attn.attn_fwd_varlen_kvcache(dev["q"], dev["k_cache"], dev["v_cache"],
+                                          dev["cu_seqlens_k"], dev["seqlens_k"], ml,
+                                          scale=case.scale, causal=case.causal,
+                                          split_keys=split_keys)
+    torch.cuda.synchronize()
+    assert attn.get_device_error() == 0
+    return o, lse
+
+
+def _check(inp, case, split_keys=0, what=""):
+    o, lse = _run(inp, case, split_keys)
+    o_ref, lse_ref = oracle.attn_kvcache(inp["q"], inp["k_cache"], inp["v_cache"],
+                                         inp["cu_seqlens_k"], inp["seqlens_k"], case.scale,
+                                         case.causal)
+    return compare(o, lse, o_ref, lse_ref, what=what), o, lse
+
+
+def test_tiny_decode():
+    c = DecodeCase("t", 3, 8, 2, 1, 128, (1, 200), False)
+    inp = kvcache_inputs(c, seed=1, seqlens=[1, 64, 200])
+    _check(inp, c, what="tiny decode")
+
+
+@pytest.mark.parametrize("split", [0, 64, 256, 1024, 8192])
+def test_tile_and_split_boundaries(split):
+    lens = [1, 63, 64, 65, 127, 128, 129, 1023, 1024, 1025, 4097, 0]
+    c = DecodeCase("b", len(lens), 16, 2, 1, 128, (0, 4097), False, slack=3)
+    inp = kvcache_inputs(c, seed=2, seqlens=lens)
+    _check(inp, c, split_keys=split, what=f"split {split}")
+
+
+def test_split_results_agree():
+    c = DecodeCase("s", 4, 8, 1, 1, 128, (1, 3000), False)
+    inp = kvcache_inputs(c, seed=3, seqlens=[3000, 1500, 777, 64])
+    (_, o1, l1) = _check(inp, c, split_keys=64, what="split 64")
+    (_, o2, l2) = _check(inp, c, split_keys=4096, what="one split")
+    assert (o1.float() - o2.float()).abs().max().item() <= 1.6e-2
+    assert (l1 - l2).abs().max().item() <= 1e-4
+
+
+def test_unfilled_slots_hold_nan():
+    c = DecodeCase("n", 6, 8, 2, 1, 128, (1, 700), False, slack=40)
+    clean = kvcache_inputs(c, seed=4)
+    dirty = kvcache_inputs(c, seed=4, slack_fill=float("nan"))
+    (_, o1, l1) = _check(clean, c, split_keys=256, what="clean")
+    (_, o2, l2) = _check(dirty, c, split_keys=256, what="NaN in unfilled slots")
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("d,dtype", [(64, "bf16"), (128, "fp16"), (64, "fp16")])
+def test_head_dims_and_fp16(d, dtype):
+    c = DecodeCase("h", 5, 12, 3, 1, d, (1, 2500), False, dtype=dtype)
+    _check(kvcache_inputs(c, seed=5), c, what=f"d{d} {dtype}")
+
+
+@pytest.mark.parametrize("nq", [2, 5, 16])
+def test_chunk_causal_bottom_right(nq):
+    lens = [nq, nq + 1, 100, 2000, 3]  # the last one: some tokens see no key
+    c = DecodeCase("c", len(lens), 16, 2, nq, 128, (1, 2000), True)
+    inp = kvcache_inputs(c, seed=6, seqlens=lens)
+    _, o, lse = _check(inp, c, split_keys=256, what=f"chunk {nq}")
+    if nq > 3:
+        # last sequence has 3 keys: tokens 0..nq-4 see nothing
+        assert torch.all(o[4, : nq - 3] == 0)
+        assert torch.all(torch.isneginf(lse[4, :, : nq - 3]))
+
+
+@pytest.mark.parametrize("name", ["llama70b_decode", "llama70b_chunk16"])
+def test_llama70b_shape_sampled_sequences(name):
+    # full-size launch (B=32, Hq=64, Hkv=8, d=128, lengths up to 32768);
+    # the oracle checks a sample of sequences, the shortest and longest included
+    c = DECODE_CASES[name]
+    inp = kvcache_inputs(c, seed=0)
+    o, lse = _run(inp, c)
+    lens = inp["seqlens_k"].tolist()
+    pick = sorted(set([int(np.argmin(lens)), int(np.argmax(lens)), 0, 7, 19]))
+    cu = inp["cu_seqlens_k"].tolist()
+    for b in pick:
+        sub_k = inp["k_cache"][cu[b]:cu[b + 1]]
+        sub_v = inp["v_cache"][cu[b]:cu[b + 1]]
+        o_ref, lse_ref = oracle.attn_kvcache(inp["q"][b:b + 1], sub_k, sub_v,
+                                             torch.tensor([0, cu[b + 1] - cu[b]]),
+                                             inp["seqlens_k"][b:b + 1], c.scale, c.causal)
+        compare(o[b:b + 1], lse[b:b + 1], o_ref, lse_ref, what=f"{name} seq {b} len {lens[b]}")
+
+
+def test_max_seqlen_too_small_is_reported():
+    c = DecodeCase("e", 2, 8, 2, 1, 128, (1, 3000), False)
+    inp = kvcache_inputs(c, seed=8, seqlens=[3000, 10])
+    attn.get_device_error()
+    _run_ok = True
+    dev = {k: v.cuda() for k, v in inp.items()}
+    attn.attn_fwd_varlen_kvcache(dev["q"], dev["k_cache"], dev["v_cache"], dev["cu_seqlens_k"],
+                                 dev["seqlens_k"], 1000, scale=c.scale, split_keys=256)
+    torch.cuda.synchronize()
+    assert attn.get_device_error() == attn.ERR_DECODE_BASE + 1

@@ -1,0 +1,125 @@
+"""Forward kernel (tcgen05) against the fp64 oracle, element by element.
+
+Full comparisons on shapes the oracle finishes in seconds (several 128-row
+tiles and ragged tails), the tiny / BERT-large / GPT-2 workloads in full, and
+the long-sequence sweep on sampled query rows at its full sizes in the launch
+configuration the bench times.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from io_aware_exact_29_b200 import attn
+from io_aware_exact_29_b200.workloads import FWD_CASES, FwdCase, default_scale, fwd_inputs
+from tests.parity import check_fwd, compare, run_fwd, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_tiny(causal):
+    c = FWD_CASES["tiny_causal" if causal else "tiny"]
+    check_fwd(fwd_inputs(c), c.causal, c.scale, what=c.name)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk", [(1, 1, 1, 128, 128), (2, 3, 3, 200, 333),
+                                            (1, 8, 2, 257, 257), (2, 4, 1, 77, 300),
+                                            (1, 2, 2, 300, 77), (3, 2, 1, 1, 129),
+                                            (1, 2, 2, 513, 1)])
+def test_ragged_and_grouped(B, Hq, Hkv, Nq, Nk, d, causal):
+    c = FwdCase("r", B, Hq, Hkv, Nq, Nk, d, causal)
+    check_fwd(fwd_inputs(c, seed=Nq + Nk + d), causal, c.scale,
+              what=f"B{B} Hq{Hq} Hkv{Hkv} Nq{Nq} Nk{Nk} d{d} causal{causal}")
+
+
+@pytest.mark.parametrize("name", ["bert_large", "bert_large_varlen", "gpt2", "gpt2_fp16"])
+def test_workloads_in_full(name):
+    c = FWD_CASES[name]
+    check_fwd(fwd_inputs(c), c.causal, c.scale, what=name)
+
+
+@pytest.mark.parametrize("name", sorted(n for n in FWD_CASES if n.startswith("sweep_")))
+def test_long_sequence_sweep_sampled_rows(name):
+    c = FWD_CASES[name]
+    rows = sample_rows(c.Nq, 48, seed=c.Nq)
+    check_fwd(fwd_inputs(c), c.causal, c.scale, rows=rows, what=name)
+
+
+def test_fp16_head128_causal_gqa():
+    c = FwdCase("h", 2, 8, 2, 384, 384, 128, True, dtype="fp16")
+    check_fwd(fwd_inputs(c, seed=3), True, c.scale, what="fp16 d128 gqa causal")
+
+
+def test_key_padding_ignores_nan_behind_the_length():
+    c = FwdCase("k", 4, 2, 2, 200, 300, 128, False, kpad_range=(1, 300))
+    inp = fwd_inputs(c, seed=11)
+    inp["seqlens_k"] = torch.tensor([300, 129, 128, 1], dtype=torch.int32)
+    clean = check_fwd(inp, False, c.scale, what="kpad clean")
+    for b, L in enumerate(inp["seqlens_k"].tolist()):
+        inp["k"][b, L:] = float("nan")
+        inp["v"][b, L:] = float("nan")
+    dirty = check_fwd(inp, False, c.scale, what="kpad with NaN padding")
+    assert dirty == clean
+    for causal in (True,):
+        check_fwd(inp, causal, c.scale, what="kpad causal with NaN padding")
+
+
+def test_zero_query_gives_prefix_means():
+    # closed form on the GPU: Q = 0 makes every visible key equally likely
+    c = FwdCase("z", 1, 2, 2, 300, 300, 64, True)
+    inp = fwd_inputs(c, seed=5)
+    inp["q"].zero_()
+    o, lse = run_fwd(inp, True, c.scale)
+    v = inp["v"].double()
+    means = torch.cumsum(v[0], 0) / torch.arange(1, 301, dtype=torch.float64)[:, None, None]
+    assert (o[0].double().cpu() - means).abs().max().item() <= 1e-2
+    expect = torch.log(torch.arange(1, 301, dtype=torch.float64))
+    assert (lse[0].double().cpu() - expect).abs().max().item() <= 1e-3
+    # causal row 0 is V[0] up to the output rounding
+    assert torch.equal(o[0, 0].cpu(), inp["v"][0, 0])
+
+
+def test_no_keys_and_fully_masked_rows():
+    c = FwdCase("m", 1, 2, 2, 256, 100, 64, True)
+    inp = fwd_inputs(c, seed=9)
+    o, lse = run_fwd(inp, True, c.scale)  # rows i < 156 see no key (bottom-right)
+    assert torch.all(o[0, :156] == 0)
+    assert torch.all(torch.isneginf(lse[0, :, :156]))
+    check_fwd(inp, True, c.scale, what="causal Nq > Nk")
+    inp0 = dict(inp)
+    inp0["k"] = inp["k"][:, :0].contiguous()
+    inp0["v"] = inp["v"][:, :0].contiguous()
+    # no keys at all: pass any valid pointer for k/v
+    q = inp["q"].cuda()
+    kv = torch.empty((1, 0, 2, 64), dtype=torch.bfloat16, device="cuda")
+    o, lse = attn.attn_fwd(q, kv, kv, causal=False)
+    torch.cuda.synchronize()
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_repeatable_bit_for_bit():
+    c = FWD_CASES["gpt2"]
+    inp = fwd_inputs(FwdCase("d", 2, 4, 4, 1024, 1024, 128, True), seed=1)
+    o1, l1 = run_fwd(inp, True, default_scale(128))
+    o2, l2 = run_fwd(inp, True, default_scale(128))
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_bounded_wait_reports_instead_of_hanging():
+    # the loader is told to skip its work: every consumer wait runs out after
+    # 100 ms, the kernel records the site, frees tensor memory and returns
+    q = torch.randn(1, 128, 1, 64, device="cuda").to(torch.bfloat16)
+    o = torch.empty_like(q)
+    lse = torch.empty(1, 1, 128, device="cuda")
+    attn.get_device_error()  # clear
+    attn.selftest_watchdog(q, q, q, o, lse, limit_ms=100)
+    code = attn.get_device_error()
+    assert code // 16 == 1 and code % 16 != 0, code
+    # the context is still usable and the word is clear again
+    check_fwd(fwd_inputs(FWD_CASES["tiny"]), False, 0.125, what="after watchdog")
+    assert attn.get_device_error() == 0
