@@ -1,0 +1,476 @@
+"""Throughput of the attention path on B200: one JSON line on rank 0.
+
+A step is one pass of the whole path over one batch of synthetic inputs:
+  forward  : B=4, H=16, N=4096, d=128, bf16, non-causal (the long-sequence
+             sweep point at which the forward target is stated), then
+  decode   : Llama2-70B shape, B=32, Hq=64, Hkv=8, d=128, one new token per
+             sequence, packed bf16 KV cache with lengths ~ U[1, 32768].
+`value` is the forward's TFLOP/s (algorithmic FLOPs / device time of the
+forward launches, summed over ranks); the decode's GB/s is reported beside it.
+All inputs are larger than L2 (126 MB), so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs the same per-rank workload on its own GPU with
+no collective on the data path (weak scaling); the timed region is bracketed
+by a barrier and a device synchronisation, and the max over ranks is taken.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
+workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from io_aware_exact_29_b200 import accounting  # noqa: E402
+from io_aware_exact_29_b200.workloads import (DECODE_CASES, FWD_CASES, fwd_inputs,  # noqa: E402
+                                              kvcache_inputs)
+
+FWD_CASE = FWD_CASES["sweep_d128_n4096"]
+DEC_CASE = DECODE_CASES["llama70b_decode"]
+METRIC = "attn fwd TFLOP/s & % of BF16 TC peak; KV-cache decode GB/s & % of HBM peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = {
+    "fwd": os.path.join(ROOT, "io_aware_exact_29_b200", "csrc", "attn_fwd_sm100a.cu"),
+    "decode": os.path.join(ROOT, "io_aware_exact_29_b200", "csrc", "attn_decode_sm100a.cu"),
+}
+L2_BYTES = 126 * 2 ** 20
+
+
+def source_hash(path: str) -> str:
+    with open(path, "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; None otherwise."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        rec = json.load(fh).get(kernel)
+    if not rec or rec.get("source_sha256_16") != source_hash(KERNEL_SOURCES[kernel]):
+        return None
+    return rec.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ helpers
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def reduce_max(values, world: int, device=None):
+    """Element-wise max of a list of floats over all ranks (timing only)."""
+    if world <= 1:
+        return list(values)
+    import torch.distributed as dist
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def fwd_work(case):
+    return accounting.fwd_flops(case.B, case.Hq, case.Nq, case.Nk, case.d, case.causal)
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local):
+    from io_aware_exact_29_b200 import attn
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # inputs, seeded per rank (independent problems), generated on the device
+    fc, dc = FWD_CASE, DEC_CASE
+    fin = fwd_inputs(fc, seed=1000 * rank, device=str(dev))
+    q, k, v = fin["q"], fin["k"], fin["v"]
+    o = torch.empty_like(q)
+    lse = torch.empty((fc.B, fc.Hq, fc.Nq), dtype=torch.float32, device=dev)
+    din = kvcache_inputs(dc, seed=1000 * rank, device=str(dev))
+    dq, kc, vc = din["q"], din["k_cache"], din["v_cache"]
+    cu, sl = din["cu_seqlens_k"], din["seqlens_k"]
+    max_len = int(sl.max().item())
+    do = torch.empty_like(dq)
+    dlse = torch.empty((dc.B, dc.Hq, dc.Nq), dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.decode_workspace_bytes(dc.B, dc.Hq, dc.Hkv, dc.Nq, dc.d, max_len),
+                     dtype=torch.uint8, device=dev)
+    fflops = fwd_work(fc)
+    dbytes = accounting.decode_bytes(sl.tolist(), dc.B, dc.Hq, dc.Hkv, dc.Nq, dc.d)
+
+    def step(ev):
+        ev[0].record(stream)
+        attn.attn_fwd(q, k, v, scale=fc.scale, causal=fc.causal, out=o, lse=lse, stream=stream)
+        ev[1].record(stream)
+        attn.attn_fwd_varlen_kvcache(dq, kc, vc, cu, sl, max_len, scale=dc.scale,
+                                     causal=dc.causal, workspace=ws, out=do, lse=dlse,
+                                     stream=stream)
+        ev[2].record(stream)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for _ in range(args.warmup):
+        step(evs[0])
+    torch.cuda.synchronize()
+    assert attn.get_device_error() == 0
+
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        barrier(world)
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    total_ms = t0.elapsed_time(t1)
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    dec_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    total_ms, fwd_ms, dec_ms = reduce_max([total_ms, fwd_ms, dec_ms], world, dev)
+    assert attn.get_device_error() == 0
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(args, attn, fin, din, max_len, stream, dev)
+    e2e_fwd_ms, e2e_dec_ms = reduce_max([e2e["fwd_ms"], e2e["dec_ms"]], world, dev)
+
+    peaks, peak_src = load_peaks()
+    fwd_tflops = fflops * args.steps * world / (fwd_ms * 1e-3) / 1e12
+    dec_gbs = dbytes * args.steps * world / (dec_ms * 1e-3) / 1e9
+    per_launch_ms = fwd_ms / args.steps
+    achieved = fflops / (per_launch_ms * 1e-3) / 1e12
+    peak_t = peaks["bf16_tflops_sustained"]
+    dec_launch_ms = dec_ms / args.steps
+    dec_achieved = dbytes / (dec_launch_ms * 1e-3) / 1e9
+
+    out = {
+        "metric": METRIC,
+        "value": round(fwd_tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16; decode lengths ~U[1,32768])",
+        "config": {
+            "workload": ("fwd: long-sequence sweep point B=4 H=16 N=4096 d=128 non-causal; "
+                         "decode: Llama2-70B shape B=32 Hq=64 Hkv=8 d=128 Nq=1 "
+                         "lengths U[1,32768] packed bf16 cache"),
+            "fwd": {"B": fc.B, "H": fc.Hq, "N": fc.Nq, "d": fc.d, "causal": fc.causal},
+            "decode": {"B": dc.B, "Hq": dc.Hq, "Hkv": dc.Hkv, "d": dc.d, "Nq": dc.Nq,
+                       "sum_len": int(sl.sum().item()), "max_len": max_len},
+            "l2": "inputs larger than L2 (fwd 268 MB, decode cache 2.1 GB); no flush",
+            "parallelism": f"replicas x{world} (independent problems per GPU, no collective)",
+        },
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "attn_fwd_kernel<128, bf16>",
+            "achieved": round(achieved, 2),
+            "peak": peak_t,
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak_t, 4),
+            "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed in a back-to-back loop)",
+            "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4),
+            "flops_per_launch": fflops,
+            "traffic": load_traffic("fwd"),
+        },
+        "decode": {
+            "value": round(dec_gbs, 1),
+            "unit": "GB/s",
+            "achieved_per_launch": round(dec_achieved, 1),
+            "peak": peaks["hbm_gbs"],
+            "frac": round(dec_achieved / peaks["hbm_gbs"], 4),
+            "bytes_per_launch": dbytes,
+            "ms_per_launch": round(dec_launch_ms, 4),
+            "bound": "hbm",
+            "traffic": load_traffic("decode"),
+            "e2e": {"value": round(dbytes * world / (e2e_dec_ms * 1e-3) / 1e9, 1),
+                    "unit": "GB/s", "h2d_bytes_per_step": e2e["dec_h2d"],
+                    "d2h_bytes_per_step": e2e["dec_d2h"]},
+        },
+        "e2e": {"value": round(fflops * world / (e2e_fwd_ms * 1e-3) / 1e12, 2),
+                "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["fwd_h2d"],
+                "d2h_bytes_per_step": e2e["fwd_d2h"]},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+        "fwd_ms_per_launch": round(per_launch_ms, 4),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget)
+    return out
+
+
+def run_e2e(args, attn, fin, din, max_len, stream, dev):
+    """Same workload through the public calls with pinned host buffers: every
+    step copies its inputs host->device and its outputs device->host."""
+    fc, dc = FWD_CASE, DEC_CASE
+    h = {n: fin[n].cpu().pin_memory() for n in ("q", "k", "v")}
+    hq = din["q"].cpu().pin_memory()
+    hcu = din["cu_seqlens_k"].cpu().pin_memory()
+    hsl = din["seqlens_k"].cpu().pin_memory()
+    dq = {n: torch.empty_like(fin[n]) for n in ("q", "k", "v")}
+    o = torch.empty_like(fin["q"])
+    lse = torch.empty((fc.B, fc.Hq, fc.Nq), dtype=torch.float32, device=dev)
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    kc, vc = din["k_cache"], din["v_cache"]  # resident cache (built on device by prefill)
+    ddq = torch.empty_like(din["q"])
+    dcu = torch.empty_like(din["cu_seqlens_k"])
+    dsl = torch.empty_like(din["seqlens_k"])
+    do = torch.empty_like(din["q"])
+    dl = torch.empty((dc.B, dc.Hq, dc.Nq), dtype=torch.float32, device=dev)
+    hdo = torch.empty(do.shape, dtype=do.dtype).pin_memory()
+    hdl = torch.empty(dl.shape, dtype=dl.dtype).pin_memory()
+    ws = torch.empty(attn.decode_workspace_bytes(dc.B, dc.Hq, dc.Hkv, dc.Nq, dc.d, max_len),
+                     dtype=torch.uint8, device=dev)
+    steps = max(3, min(args.steps, 10))
+
+    def fwd_step():
+        for n in ("q", "k", "v"):
+            dq[n].copy_(h[n], non_blocking=True)
+        attn.attn_fwd(dq["q"], dq["k"], dq["v"], scale=fc.scale, causal=fc.causal, out=o,
+                      lse=lse, stream=stream)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    def dec_step():
+        ddq.copy_(hq, non_blocking=True)
+        dcu.copy_(hcu, non_blocking=True)
+        dsl.copy_(hsl, non_blocking=True)
+        attn.attn_fwd_varlen_kvcache(ddq, kc, vc, dcu, dsl, max_len, scale=dc.scale,
+                                     causal=dc.causal, workspace=ws, out=do, lse=dl,
+                                     stream=stream)
+        hdo.copy_(do, non_blocking=True)
+        hdl.copy_(dl, non_blocking=True)
+
+    res = {}
+    for name, fn in (("fwd", fwd_step), ("dec", dec_step)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        res[name + "_ms"] = a.elapsed_time(b) / steps
+    res["fwd_h2d"] = sum(t.numel() * t.element_size() for t in h.values())
+    res["fwd_d2h"] = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    res["dec_h2d"] = sum(t.numel() * t.element_size() for t in (hq, hcu, hsl))
+    res["dec_d2h"] = hdo.numel() * hdo.element_size() + hdl.numel() * hdl.element_size()
+    return res
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(rows_per_head: int, seed: int = 0):
+    """A bounded sample of the forward workload: every (batch, head), a seeded
+    subset of query rows against all keys."""
+    fc = FWD_CASE
+    inp = fwd_inputs(fc, seed=seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    rows = sorted(torch.randperm(fc.Nq, generator=g)[:rows_per_head].tolist())
+    flops = 4 * fc.d * fc.B * fc.Hq * len(rows) * fc.Nk  # non-causal: every key visible
+    return inp, rows, flops
+
+
+def cpu_baseline(budget_s: float = 15.0):
+    import oracle
+
+    fc = FWD_CASE
+    rows_per_head = 16
+    inp, rows, flops = oracle_sample(rows_per_head)
+    t = time.perf_counter()
+    oracle.attn_fwd(inp["q"], inp["k"], inp["v"], fc.scale, fc.causal, rows=rows)
+    dt = time.perf_counter() - t
+    # grow the sample to fill about `budget_s` of CPU time, then time it once
+    scale = max(1, min(int(budget_s / max(dt, 1e-3)), fc.Nq // rows_per_head))
+    if scale > 1:
+        inp, rows, flops = oracle_sample(rows_per_head * scale)
+        t = time.perf_counter()
+        oracle.attn_fwd(inp["q"], inp["k"], inp["v"], fc.scale, fc.causal, rows=rows)
+        dt = time.perf_counter() - t
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s",
+            "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": (f"fwd workload B=4 H=16 N=4096 d=128: {len(rows)} seeded query rows "
+                       f"per head x all 64 heads x all 4096 keys, fp64 ({dt:.1f} s)")}
+
+
+def run_reference(args, rank, world):
+    """The oracle arm: the fp64 CPU oracle on the host cores, each step a
+    bounded sample of the forward workload."""
+    import oracle
+
+    fc = FWD_CASE
+    inp, rows, flops = oracle_sample(args.ref_rows)
+    for _ in range(args.warmup):
+        oracle.attn_fwd(inp["q"], inp["k"], inp["v"], fc.scale, fc.causal, rows=rows[:4])
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attn_fwd(inp["q"], inp["k"], inp["v"], fc.scale, fc.causal, rows=rows)
+    dt = time.perf_counter() - t
+    value = flops * args.steps / dt / 1e12
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 6),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16 inputs widened to fp64)",
+        "config": {"workload": "fwd: B=4 H=16 N=4096 d=128 non-causal (sampled query rows)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
+                         "cores": oracle.max_threads(), "kind": "oracle",
+                         "sample": f"{len(rows)} query rows per head x 64 heads x 4096 keys"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=32)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        # the oracle arm runs on rank 0's host cores only; other ranks leave
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return 0
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        out = run_ours(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+        return 0
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -25,7 +25,8 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, rows=None, what=""):
     err = np.abs(og - o_ref)
     max_err, mean_err = float(err.max(initial=0.0)), float(err.mean()) if err.size else 0.0
     both_inf = np.isneginf(lg) & np.isneginf(lse_ref)
-    lerr = np.where(both_inf, 0.0, np.abs(lg - lse_ref))
+    with np.errstate(invalid="ignore"):
+        lerr = np.where(both_inf, 0.0, np.abs(lg - lse_ref))
     lse_err = float(np.nan_to_num(lerr, nan=np.inf).max(initial=0.0))
     worst = np.unravel_index(np.argmax(err), err.shape) if err.size else None
     msg = (f"{what}: O max {max_err:.3e} (at {worst}) mean {mean_err:.3e}, "
