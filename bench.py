@@ -440,6 +440,34 @@ def run_reference(args, rank, world):
     }
 
 
+def run_profile_case(kernel: str, launches: int):
+    """Small, self-contained launches for ncu captures: the forward of the
+    bench workload (268 MB of inputs), or a decode of the Llama2-70B shape with
+    lengths up to 8192 (about 0.5 GB of cache); both larger than L2."""
+    from io_aware_exact_29_b200 import attn
+    from io_aware_exact_29_b200.workloads import DecodeCase
+
+    dev = torch.device("cuda", 0)
+    if kernel == "fwd":
+        fc = FWD_CASE
+        fin = fwd_inputs(fc, seed=0, device="cuda")
+        for _ in range(2 + launches):
+            attn.attn_fwd(fin["q"], fin["k"], fin["v"], scale=fc.scale, causal=fc.causal)
+    else:
+        dc = DecodeCase("profile", 32, 64, 8, 1, 128, (1, 8192), False)
+        din = kvcache_inputs(dc, seed=0, device="cuda")
+        ml = int(din["seqlens_k"].max().item())
+        ws = torch.empty(attn.decode_workspace_bytes(dc.B, dc.Hq, dc.Hkv, dc.Nq, dc.d, ml),
+                         dtype=torch.uint8, device=dev)
+        for _ in range(2 + launches):
+            attn.attn_fwd_varlen_kvcache(din["q"], din["k_cache"], din["v_cache"],
+                                         din["cu_seqlens_k"], din["seqlens_k"], ml,
+                                         scale=dc.scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert attn.get_device_error() == 0
+    print(f"profile case {kernel}: {2 + launches} launches ok")
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -449,7 +477,13 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--profile", choices=["fwd", "decode"], default=None,
+                    help="run a small case of one kernel for an ncu capture and exit")
+    ap.add_argument("--profile-launches", type=int, default=3)
     args = ap.parse_args(argv)
+    if args.profile:
+        run_profile_case(args.profile, args.profile_launches)
+        return 0
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
