@@ -105,6 +105,51 @@ __device__ __forceinline__ int tiles_for(int q_first, int Nq, int Lk, int causal
     return nt;
 }
 
+// Running maxima of 64 score columns (two 32-column TMEM loads) into eight
+// independent chains of three-input maxima.  kMask: the tile reaches past
+// the row's last visible key (key_base + c > row_lim is masked).
+template <bool kMask>
+__device__ __forceinline__ void half_max(const uint32_t (&r)[2][32], int key_base, int row_lim,
+                                         float (&mx8)[8]) {
+#pragma unroll
+    for (int c = 0; c < 64; c += 16) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int c0 = c + u, c1 = c + 8 + u;
+            float v0 = __uint_as_float(r[c0 >> 5][c0 & 31]);
+            float v1 = __uint_as_float(r[c1 >> 5][c1 & 31]);
+            if (kMask) {
+                if (key_base + c0 > row_lim) v0 = -INFINITY;
+                if (key_base + c1 > row_lim) v1 = -INFINITY;
+            }
+            mx8[u] = ptx::max3(mx8[u], v0, v1);
+        }
+    }
+}
+
+// p = 2^(s * scale_log2 - m) for 64 score columns, accumulated into four
+// pair sums and packed two per 32-bit word (bf16 or fp16).
+template <bool kMask, bool BF16>
+__device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_base, int row_lim,
+                                         uint64_t sl2_2, uint64_t nm_2, uint64_t (&acc2)[4],
+                                         uint32_t (&pk)[32]) {
+#pragma unroll
+    for (int c = 0; c < 64; c += 2) {
+        float v0 = __uint_as_float(r[c >> 5][c & 31]);
+        float v1 = __uint_as_float(r[c >> 5][(c & 31) + 1]);
+        if (kMask) {
+            if (key_base + c > row_lim) v0 = -INFINITY;
+            if (key_base + c + 1 > row_lim) v1 = -INFINITY;
+        }
+        float t0, t1;
+        ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(v0, v1), sl2_2, nm_2), t0, t1);
+        const float p0 = ptx::ex2_approx(t0);
+        const float p1 = ptx::ex2_approx(t1);
+        acc2[(c >> 1) & 3] = ptx::f2_add(acc2[(c >> 1) & 3], ptx::f2_pack(p0, p1));
+        pk[c >> 1] = ptx::pack2<BF16>(p0, p1);
+    }
+}
+
 template <int D, bool BF16, int KST, int VST>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -337,20 +382,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tmem_ld32(t_s + hf * 64 + 32, r[1]);
                 ptx::tmem_wait_ld_dep(r[0]);
                 ptx::tmem_wait_ld_dep(r[1]);
-#pragma unroll
-                for (int c = 0; c < 64; c += 16) {
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int c0 = c + u, c1 = c + 8 + u;
-                        float v0 = __uint_as_float(r[c0 >> 5][c0 & 31]);
-                        float v1 = __uint_as_float(r[c1 >> 5][c1 & 31]);
-                        if (masked) {
-                            if (key0 + hf * 64 + c0 > row_lim) v0 = -INFINITY;
-                            if (key0 + hf * 64 + c1 > row_lim) v1 = -INFINITY;
-                        }
-                        mx8[u] = ptx::max3(mx8[u], v0, v1);
-                    }
-                }
+                if (masked)
+                    half_max<true>(r, key0 + hf * 64, row_lim, mx8);
+                else
+                    half_max<false>(r, key0 + hf * 64, row_lim, mx8);
             }
             const float mx = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]),
                                        ptx::max3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
@@ -376,21 +411,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tmem_wait_ld_dep(r[0]);
                 ptx::tmem_wait_ld_dep(r[1]);
                 uint32_t pk[32];
-#pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    float v0 = __uint_as_float(r[c >> 5][c & 31]);
-                    float v1 = __uint_as_float(r[c >> 5][(c & 31) + 1]);
-                    if (masked) {
-                        if (key0 + hf * 64 + c > row_lim) v0 = -INFINITY;
-                        if (key0 + hf * 64 + c + 1 > row_lim) v1 = -INFINITY;
-                    }
-                    float t0, t1;
-                    ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(v0, v1), sl2_2, nm_2), t0, t1);
-                    const float p0 = ptx::ex2_approx(t0);
-                    const float p1 = ptx::ex2_approx(t1);
-                    acc2[(c >> 1) & 3] = ptx::f2_add(acc2[(c >> 1) & 3], ptx::f2_pack(p0, p1));
-                    pk[c >> 1] = ptx::pack2<BF16>(p0, p1);
-                }
+                if (masked)
+                    half_exp<true, BF16>(r, key0 + hf * 64, row_lim, sl2_2, nm_2, acc2, pk);
+                else
+                    half_exp<false, BF16>(r, key0 + hf * 64, row_lim, sl2_2, nm_2, acc2, pk);
                 ptx::tmem_st32(t_s + hf * 32, pk);
             }
             float s0, s1, s2, s3, s4, s5, s6, s7;
