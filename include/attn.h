@@ -130,6 +130,42 @@ ATTN_API int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const v
                             float scale, int causal, int dtype, void* workspace,
                             size_t workspace_bytes, int split_keys, void* stream);
 
+/* Size in bytes of the scratch area built into the library for
+ * attn_fwd_varlen_kvcache_noalloc (32 MiB). */
+#define ATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * attn_fwd_varlen_kvcache for callers that cannot allocate device memory.
+ * (An addition of this library: the pages have no counterpart.)
+ *
+ * The decode needs a workspace for its split-K partial results.  Some callers
+ * cannot provide one: code embedded in a host program that plans and owns all
+ * device memory without giving it an allocator, or a decode loop that must
+ * not call cudaMalloc because that call can synchronise the whole device.
+ * This entry point takes the same arguments as attn_fwd_varlen_kvcache minus
+ * the workspace and uses a scratch area of ATTN_NOALLOC_SCRATCH_BYTES that the
+ * library keeps in a static device array; it calls no cudaMalloc, cudaFree or
+ * other allocating routine.  The caller still passes every input and output.
+ *  - Limit: if the sizes need more scratch than ATTN_NOALLOC_SCRATCH_BYTES
+ *    (see attn_decode_workspace_bytes; a larger split_keys needs less), the
+ *    call returns ATTN_ERR_WORKSPACE before queuing any work.
+ *  - Set-up: the first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make
+ *    that first call before any stream capture on the device.
+ *  - Sharing: every GPU that loads the library holds the array until the
+ *    process exits, and all calls on a device share it.  It keeps whatever the
+ *    last call left; each call clears the parts that must start at zero (the
+ *    split counters) on `stream` before its kernel.  Calls that overlap on the
+ *    GPU (other streams, other host threads) race on it: serialise them.
+ * Returns the same status codes as attn_fwd_varlen_kvcache.
+ */
+ATTN_API int attn_fwd_varlen_kvcache_noalloc(const void* q, const void* k_cache,
+                                             const void* v_cache, const int* cu_seqlens_k,
+                                             const int* seqlens_k, int max_seqlen_k,
+                                             int cache_slots, void* o, float* lse, int B, int Hq,
+                                             int Hkv, int Nq, int d, float scale, int causal,
+                                             int dtype, int split_keys, void* stream);
+
 /* Human-readable text of a status code (static storage). */
 ATTN_API const char* attn_status_string(int status);
 
