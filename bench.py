@@ -463,6 +463,9 @@ def run_profile_case(kernel: str, launches: int):
             attn.attn_fwd_varlen_kvcache(din["q"], din["k_cache"], din["v_cache"],
                                          din["cu_seqlens_k"], din["seqlens_k"], ml,
                                          scale=dc.scale, workspace=ws)
+        lens = din["seqlens_k"].tolist()
+        print("decode profile case: sum_len", sum(lens), "algorithmic bytes per launch",
+              accounting.decode_bytes(lens, dc.B, dc.Hq, dc.Hkv, dc.Nq, dc.d))
     torch.cuda.synchronize()
     assert attn.get_device_error() == 0
     print(f"profile case {kernel}: {2 + launches} launches ok")

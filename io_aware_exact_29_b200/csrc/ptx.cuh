@@ -322,6 +322,40 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     return d;
 }
 
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^x for two lanes on the FMA pipe (no MUFU).  Cody & Waite range
+// reduction x = n + f, n = round(x), f in [-1/2, 1/2]; 2^f by a cubic whose
+// coefficients minimise the maximum relative error on that interval (Remez
+// exchange; io_aware_exact_29_b200/fit_exp2.py; max relative error 7.5e-5);
+// 2^n built directly in the exponent field.  Inputs are clamped at -127, where
+// 2^n's bit pattern is +0, so -inf and anything below -127 give exactly 0.
+// Valid for x <= 127.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+    constexpr float kC0 = 0.999928057f, kC1 = 0.693260968f, kC2 = 0.242611125f,
+                    kC3 = 0.0551716685f;
+    // 1.5 * 2^23 + 127: adding it rounds x to an integer held in the low
+    // mantissa bits, pre-biased by 127 for the exponent field.
+    constexpr float kRound = 12583039.0f;
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    const uint64_t xc = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+    const uint64_t rr = f2_add(xc, f2_pack(kRound, kRound));
+    const uint64_t fr = f2_sub(xc, f2_sub(rr, f2_pack(kRound, kRound)));
+    uint64_t q = f2_fma(fr, f2_pack(kC3, kC3), f2_pack(kC2, kC2));
+    q = f2_fma(q, fr, f2_pack(kC1, kC1));
+    q = f2_fma(q, fr, f2_pack(kC0, kC0));
+    float r0, r1;
+    f2_unpack(rr, r0, r1);
+    const uint64_t scale =
+        f2_pack(__int_as_float(__float_as_int(r0) << 23), __int_as_float(__float_as_int(r1) << 23));
+    return f2_mul(q, scale);
+}
+
 template <bool kBF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     if constexpr (kBF16) {
