@@ -471,6 +471,66 @@ def run_profile_case(kernel: str, launches: int):
     print(f"profile case {kernel}: {2 + launches} launches ok")
 
 
+def run_sweep(reps: int = 20):
+    """One JSON line per configured workload (forward TFLOP/s, decode GB/s),
+    each timed with CUDA events over `reps` back-to-back launches after 3
+    warm-ups; inputs seeded on the device.  Not the default line."""
+    from io_aware_exact_29_b200 import attn
+
+    peaks, _ = load_peaks()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    for name, c in FWD_CASES.items():
+        fin = fwd_inputs(c, seed=0, device="cuda")
+        sl = fin["seqlens_k"]
+        o = torch.empty_like(fin["q"])
+        lse = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)
+        ms = timed(lambda: attn.attn_fwd(fin["q"], fin["k"], fin["v"], scale=c.scale,
+                                         causal=c.causal, seqlens_k=sl, out=o, lse=lse))
+        flops = accounting.fwd_flops(c.B, c.Hq, c.Nq, c.Nk, c.d, c.causal,
+                                     None if sl is None else sl.tolist())
+        tf = flops / (ms * 1e-3) / 1e12
+        print(json.dumps({"sweep": name, "kind": "fwd", "dtype": c.dtype, "causal": c.causal,
+                          "B": c.B, "H": c.Hq, "N": c.Nq, "d": c.d, "ms": round(ms, 4),
+                          "TFLOP/s": round(tf, 1),
+                          "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 3),
+                          "frac_burst": round(tf / peaks["bf16_tflops"], 3)}), flush=True)
+        del fin, o, lse
+    for name, c in DECODE_CASES.items():
+        din = kvcache_inputs(c, seed=0, device="cuda")
+        ml = int(din["seqlens_k"].max().item())
+        ws = torch.empty(attn.decode_workspace_bytes(c.B, c.Hq, c.Hkv, c.Nq, c.d, ml),
+                         dtype=torch.uint8, device=dev)
+        o = torch.empty_like(din["q"])
+        lse = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)
+        ms = timed(lambda: attn.attn_fwd_varlen_kvcache(
+            din["q"], din["k_cache"], din["v_cache"], din["cu_seqlens_k"], din["seqlens_k"], ml,
+            scale=c.scale, causal=c.causal, workspace=ws, out=o, lse=lse))
+        lens = din["seqlens_k"].tolist()
+        by = accounting.decode_bytes(lens, c.B, c.Hq, c.Hkv, c.Nq, c.d)
+        fl = accounting.decode_flops(lens, c.Hq, c.Nq, c.d, c.causal)
+        gbs = by / (ms * 1e-3) / 1e9
+        print(json.dumps({"sweep": name, "kind": "decode", "Nq": c.Nq, "ms": round(ms, 4),
+                          "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 3),
+                          "TFLOP/s": round(fl / (ms * 1e-3) / 1e12, 1)}), flush=True)
+        del din, ws, o, lse
+    assert attn.get_device_error() == 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -483,7 +543,12 @@ def main(argv=None):
     ap.add_argument("--profile", choices=["fwd", "decode"], default=None,
                     help="run a small case of one kernel for an ncu capture and exit")
     ap.add_argument("--profile-launches", type=int, default=3)
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every configured workload, one JSON line each, and exit")
     args = ap.parse_args(argv)
+    if args.sweep:
+        run_sweep()
+        return 0
     if args.profile:
         run_profile_case(args.profile, args.profile_launches)
         return 0

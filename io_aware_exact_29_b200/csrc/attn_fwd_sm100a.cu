@@ -8,11 +8,13 @@
 // only O; the effectstory.com article "FlashAttention：IO 感知的精確注意力演算
 // 法..." states the same single pass: Q, K, V loaded once, O written once).
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warps 0-3   softmax of Q0 (thread t owns query row t = TMEM lane t)
 //   warps 4-7   softmax of Q1
 //   warp 8      TMA loader: Q0, Q1 once, then K_j / V_j into rings
 //   warp 9      tensor-memory owner and single-thread tcgen05.mma issuer
+//   warps 10-11 idle (they complete the third warpgroup, whose registers
+//               move to the softmax warpgroups)
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
 // O1 [256+D, 256+2D).  Each softmax thread reads its score row from S_a,
 // keeps the running max m and sum l (the online softmax of the section above),
@@ -42,7 +44,15 @@ namespace {
 
 constexpr int kBlockM = 128;  // rows per Q tile
 constexpr int kBlockN = 128;  // keys per K/V tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+// Register split (setmaxnreg): the kernel launches with 168 registers per
+// thread; the two softmax warpgroups grow to 216, the loader/MMA warpgroup
+// shrinks to 72.  The shares add up to the launch allocation exactly.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsSoftmax = 216;
+constexpr int kRegsOther = 72;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsLaunch,
+              "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 
@@ -227,7 +237,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
-
+    if (warp >= 8) {
+        ptx::setmaxnreg_dec<kRegsOther>();
+    }
     if (warp == 8) {
         // ================================================= TMA loader
         if (lane == 0 && nt > 0 && !p.inject) {
@@ -351,8 +363,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::mbar_wait(&bars->drain, 0, p.limit_ns, no_abort);
             }
         }
-    } else {
+    } else if (warp < 8) {
         // ================================================= softmax warpgroups
+        ptx::setmaxnreg_inc<kRegsSoftmax>();
         const int a = warp >> 2;  // which Q tile
         const int nta = a == 0 ? nt0 : nt1;
         const uint32_t quarter = (uint32_t)(warp & 3);
@@ -378,27 +391,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_after();
             const int key0 = j * kBlockN;
             const bool masked = key0 + kBlockN - 1 > row_lim;
-            // pass 1: row maximum, two halves of 64 columns, eight independent
-            // chains of three-input maxima
+            // the whole score row in registers: four loads, one wait
+            uint32_t r[2][2][32];
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                ptx::tmem_ld32(t_s + hf * 64, r[hf][0]);
+                ptx::tmem_ld32(t_s + hf * 64 + 32, r[hf][1]);
+            }
+            // row maximum: eight independent chains of three-input maxima
             float mx8[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
-            {
-                uint32_t r[2][2][32];
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    ptx::tmem_ld32(t_s + hf * 64, r[hf][0]);
-                    ptx::tmem_ld32(t_s + hf * 64 + 32, r[hf][1]);
-                }
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    ptx::tmem_wait_ld_dep(r[hf][0]);
-                    ptx::tmem_wait_ld_dep(r[hf][1]);
-                    if (masked)
-                        half_max<true>(r[hf], key0 + hf * 64, row_lim, mx8);
-                    else
-                        half_max<false>(r[hf], key0 + hf * 64, row_lim, mx8);
-                }
+            for (int hf = 0; hf < 2; ++hf) {
+                ptx::tmem_wait_ld_dep(r[hf][0]);
+                ptx::tmem_wait_ld_dep(r[hf][1]);
+                if (masked)
+                    half_max<true>(r[hf], key0 + hf * 64, row_lim, mx8);
+                else
+                    half_max<false>(r[hf], key0 + hf * 64, row_lim, mx8);
             }
             const float mx = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]),
                                        ptx::max3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
@@ -414,20 +425,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
             const uint64_t nm_2 = ptx::f2_pack(-m_use, -m_use);
             uint64_t acc2[4] = {0, 0, 0, 0};  // four pair accumulators of the row sum
-            // pass 2: exponentials per half; P of half hf goes to columns
-            // [32 hf, 32 hf + 32) of S_a, which pass 2 has already consumed
+            // exponentials; P of keys [64 hf, 64 hf + 64) goes to columns
+            // [32 hf, 32 hf + 32) of S_a (every score is already in registers)
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                uint32_t r[2][32];
-                ptx::tmem_ld32(t_s + hf * 64, r[0]);
-                ptx::tmem_ld32(t_s + hf * 64 + 32, r[1]);
-                ptx::tmem_wait_ld_dep(r[0]);
-                ptx::tmem_wait_ld_dep(r[1]);
                 uint32_t pk[32];
                 if (masked)
-                    half_exp<true, BF16>(r, key0 + hf * 64, row_lim, sl2_2, nm_2, acc2, pk);
+                    half_exp<true, BF16>(r[hf], key0 + hf * 64, row_lim, sl2_2, nm_2, acc2, pk);
                 else
-                    half_exp<false, BF16>(r, key0 + hf * 64, row_lim, sl2_2, nm_2, acc2, pk);
+                    half_exp<false, BF16>(r[hf], key0 + hf * 64, row_lim, sl2_2, nm_2, acc2, pk);
                 ptx::tmem_st32(t_s + hf * 32, pk);
             }
             float s0, s1, s2, s3, s4, s5, s6, s7;
@@ -546,8 +552,14 @@ cudaError_t launch_fwd_t(const FwdMaps& maps, const FwdParams& p, cudaStream_t s
     using L = FwdSmem<D, KST, VST>;
     static_assert(L::kAlloc <= 227 * 1024, "shared memory budget");
     auto kern = attn_fwd_kernel<D, BF16, KST, VST>;
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc);
+    // The register split assumes exactly kRegsLaunch registers per thread at
+    // launch; with fewer, setmaxnreg.inc could never be satisfied.  Refuse to
+    // launch a build that does not match.
+    cudaFuncAttributes attr;
+    cudaError_t e = cudaFuncGetAttributes(&attr, kern);
+    if (e != cudaSuccess) return e;
+    if (attr.numRegs != kRegsLaunch) return cudaErrorInvalidKernelImage;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc);
     if (e != cudaSuccess) return e;
     dim3 grid((p.Nq + 2 * kBlockM - 1) / (2 * kBlockM), p.Hq, p.B);
     kern<<<grid, kThreads, L::kAlloc, stream>>>(maps.q, maps.k, maps.v, maps.o, p);

@@ -149,6 +149,22 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr) {
                  : "memory");
 }
 
+// Move registers between the warpgroups of a CTA (all warps of a warpgroup
+// execute the same instruction).  `inc` waits until other warpgroups have
+// released enough with `dec`: the per-thread targets, times the warpgroups'
+// threads, must add up to at most the block's launch allocation.
+template <uint32_t kRegs>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    static_assert(kRegs % 8 == 0 && kRegs >= 24 && kRegs <= 256, "bad register target");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
+template <uint32_t kRegs>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    static_assert(kRegs % 8 == 0 && kRegs >= 24 && kRegs <= 256, "bad register target");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
