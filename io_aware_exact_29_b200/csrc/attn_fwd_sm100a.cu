@@ -46,11 +46,11 @@ constexpr int kBlockM = 128;  // rows per Q tile
 constexpr int kBlockN = 128;  // keys per K/V tile
 constexpr int kThreads = 384;
 // Register split (setmaxnreg): the kernel launches with 168 registers per
-// thread; the two softmax warpgroups grow to 216, the loader/MMA warpgroup
-// shrinks to 72.  The shares add up to the launch allocation exactly.
+// thread; the two softmax warpgroups grow to 208, the loader/MMA warpgroup
+// shrinks to 88.  The shares add up to the launch allocation exactly.
 constexpr int kRegsLaunch = 168;
-constexpr int kRegsSoftmax = 216;
-constexpr int kRegsOther = 72;
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsOther = 88;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
@@ -293,10 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ================================================= MMA issuer
         if (lane == 0 && nt > 0) {
             bool ok = true;
-            bool q_ready[2] = {false, false};
-            const uint32_t col_s[2] = {0u, 128u};
-            const uint32_t col_o[2] = {256u, 256u + D};
-            const uint32_t q_addr[2] = {sbase + L::kQ, sbase + L::kQ + kTileBytes};
+            bool q0_ready = false, q1_ready = false;
             auto wait_or_fail = [&](uint64_t* bar, uint32_t parity, unsigned site) {
                 if (!ptx::mbar_wait(bar, parity, p.limit_ns, abort_flag)) {
                     record_error(p.err, kErrFwdBase + site, &bars->abort);
@@ -304,18 +301,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 return ok;
             };
+            // Descriptors are built once; inside the loop each MMA only adds a
+            // compile-time offset (in 16-byte units) to a base descriptor, so
+            // that the issuing thread keeps the tensor pipe fed.
+            const uint64_t q_desc0 = ptx::sdesc_sw128(sbase + L::kQ, 16, 1024);
+            const uint64_t k_desc0 = ptx::sdesc_sw128(sbase + L::kK, 16, 1024);
+            const uint64_t v_desc0 = ptx::sdesc_sw128(sbase + L::kV, kBlockBytes, 1024);
+            constexpr uint64_t kTileUnits = kTileBytes >> 4;  // one tile, in 16-byte units
             auto issue_s = [&](int a, int j) {
-                if (!q_ready[a]) {
+                bool& ready = a == 0 ? q0_ready : q1_ready;
+                if (!ready) {
                     if (!wait_or_fail(&bars->q_full[a], 0, 3)) return;
                     ptx::tc_fence_after();
-                    q_ready[a] = true;
+                    ready = true;
                 }
-                const uint32_t k_addr = sbase + L::kK + (j % KST) * kTileBytes;
+                const uint64_t qd = q_desc0 + (uint64_t)a * kTileUnits;
+                const uint64_t kd = k_desc0 + (uint64_t)(j % KST) * kTileUnits;
+                const uint32_t d_s = tmem + (a == 0 ? 0u : 128u);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
-                    ptx::umma_ss(tmem + col_s[a], ptx::sdesc_sw128(q_addr[a] + off, 16, 1024),
-                                 ptx::sdesc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0);
+                    // K-major: +32 B per 16 elements, +16 KB per 64-column block
+                    const uint64_t off = (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
+                    ptx::umma_ss(d_s, qd + off, kd + off, kIdescS, kk > 0);
                 }
                 ptx::umma_commit(&bars->s_full[a]);
             };
@@ -323,12 +330,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_or_fail(&bars->p_full[a], j & 1, 5)) return;
                 if (!wait_or_fail(&bars->v_full[j % VST], (j / VST) & 1, 6)) return;
                 ptx::tc_fence_after();
-                const uint32_t v_addr = sbase + L::kV + (j % VST) * kTileBytes;
+                const uint64_t vd = v_desc0 + (uint64_t)(j % VST) * kTileUnits;
+                const uint32_t d_o = tmem + (a == 0 ? 256u : 256u + D);
+                const uint32_t a_p = tmem + (a == 0 ? 0u : 128u);
+                const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
                 for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                    ptx::umma_ts(tmem + col_o[a], tmem + col_s[a] + kk * 8,
-                                 ptx::sdesc_sw128(v_addr + kk * 16 * 128, kBlockBytes, 1024),
-                                 kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+                    // MN-major V: +16 keys = +2 KB per step
+                    ptx::umma_ts(d_o, a_p + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), kIdescO,
+                                 kk > 0 ? 1u : acc0);
                 }
                 if (j == (a == 0 ? nt0 : nt1) - 1) ptx::umma_commit(&bars->o_done[a]);
             };
