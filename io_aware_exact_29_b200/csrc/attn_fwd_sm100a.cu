@@ -240,41 +240,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp >= 8) {
         ptx::setmaxnreg_dec<kRegsOther>();
     }
+    // The loader and MMA loops run on all 32 lanes of their warp (no
+    // divergence between a working lane and lanes parked at a barrier); one
+    // lane issues the copies and MMAs, and every wait's outcome is made
+    // warp-uniform.
     if (warp == 8) {
         // ================================================= TMA loader
-        if (lane == 0 && nt > 0 && !p.inject) {
+        if (nt > 0 && !p.inject) {
             int issued_k = 0, issued_v = 0;
-            bool issued_q[2] = {false, false};
             for (int a = 0; a < 2; ++a) {
                 if ((a == 0 ? nt0 : nt1) == 0) continue;
-                ptx::mbar_arrive_expect_tx(&bars->q_full[a], kTileBytes);
-                for (int c = 0; c < kDBlocks; ++c)
-                    ptx::tma_load_4d(smem + L::kQ + a * kTileBytes + c * kBlockBytes, &tm_q,
-                                     &bars->q_full[a], c * 64, h, qbase + a * kBlockM, b);
-                issued_q[a] = true;
+                if (lane == 0) {
+                    ptx::mbar_arrive_expect_tx(&bars->q_full[a], kTileBytes);
+                    for (int c = 0; c < kDBlocks; ++c)
+                        ptx::tma_load_4d(smem + L::kQ + a * kTileBytes + c * kBlockBytes, &tm_q,
+                                         &bars->q_full[a], c * 64, h, qbase + a * kBlockM, b);
+                }
+                __syncwarp();
             }
             for (int j = 0; j < nt; ++j) {
                 const int sk = j % KST;
-                if (!ptx::mbar_wait(&bars->k_empty[sk], ((j / KST) & 1) ^ 1, p.limit_ns,
-                                    abort_flag)) {
+                if (!warp_wait(&bars->k_empty[sk], ((j / KST) & 1) ^ 1, p.limit_ns, abort_flag)) {
                     record_error(p.err, kErrFwdBase + 1, &bars->abort);
                     break;
                 }
-                ptx::mbar_arrive_expect_tx(&bars->k_full[sk], kTileBytes);
-                for (int c = 0; c < kDBlocks; ++c)
-                    ptx::tma_load_4d(smem + L::kK + sk * kTileBytes + c * kBlockBytes, &tm_k,
-                                     &bars->k_full[sk], c * 64, g, j * kBlockN, b);
+                if (lane == 0) {
+                    ptx::mbar_arrive_expect_tx(&bars->k_full[sk], kTileBytes);
+                    for (int c = 0; c < kDBlocks; ++c)
+                        ptx::tma_load_4d(smem + L::kK + sk * kTileBytes + c * kBlockBytes, &tm_k,
+                                         &bars->k_full[sk], c * 64, g, j * kBlockN, b);
+                }
+                __syncwarp();
                 ++issued_k;
                 const int sv = j % VST;
-                if (!ptx::mbar_wait(&bars->v_empty[sv], ((j / VST) & 1) ^ 1, p.limit_ns,
-                                    abort_flag)) {
+                if (!warp_wait(&bars->v_empty[sv], ((j / VST) & 1) ^ 1, p.limit_ns, abort_flag)) {
                     record_error(p.err, kErrFwdBase + 2, &bars->abort);
                     break;
                 }
-                ptx::mbar_arrive_expect_tx(&bars->v_full[sv], kTileBytes);
-                for (int c = 0; c < kDBlocks; ++c)
-                    ptx::tma_load_4d(smem + L::kV + sv * kTileBytes + c * kBlockBytes, &tm_v,
-                                     &bars->v_full[sv], c * 64, g, j * kBlockN, b);
+                if (lane == 0) {
+                    ptx::mbar_arrive_expect_tx(&bars->v_full[sv], kTileBytes);
+                    for (int c = 0; c < kDBlocks; ++c)
+                        ptx::tma_load_4d(smem + L::kV + sv * kTileBytes + c * kBlockBytes, &tm_v,
+                                         &bars->v_full[sv], c * 64, g, j * kBlockN, b);
+                }
+                __syncwarp();
                 ++issued_v;
             }
             // Never leave the CTA with a copy in flight: wait (bounded, and
@@ -283,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int zero = 0;
             volatile int* no_abort = &zero;
             for (int a = 0; a < 2; ++a)
-                if (issued_q[a]) ptx::mbar_wait(&bars->q_full[a], 0, p.limit_ns, no_abort);
+                if ((a == 0 ? nt0 : nt1) > 0) ptx::mbar_wait(&bars->q_full[a], 0, p.limit_ns, no_abort);
             for (int j = max(0, issued_k - KST); j < issued_k; ++j)
                 ptx::mbar_wait(&bars->k_full[j % KST], (j / KST) & 1, p.limit_ns, no_abort);
             for (int j = max(0, issued_v - VST); j < issued_v; ++j)
@@ -291,19 +300,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 9) {
         // ================================================= MMA issuer
-        if (lane == 0 && nt > 0) {
+        if (nt > 0) {
             bool ok = true;
             bool q0_ready = false, q1_ready = false;
             auto wait_or_fail = [&](uint64_t* bar, uint32_t parity, unsigned site) {
-                if (!ptx::mbar_wait(bar, parity, p.limit_ns, abort_flag)) {
+                if (!warp_wait(bar, parity, p.limit_ns, abort_flag)) {
                     record_error(p.err, kErrFwdBase + site, &bars->abort);
                     ok = false;
                 }
                 return ok;
             };
             // Descriptors are built once; inside the loop each MMA only adds a
-            // compile-time offset (in 16-byte units) to a base descriptor, so
-            // that the issuing thread keeps the tensor pipe fed.
+            // compile-time offset (in 16-byte units) to a base descriptor.
             const uint64_t q_desc0 = ptx::sdesc_sw128(sbase + L::kQ, 16, 1024);
             const uint64_t k_desc0 = ptx::sdesc_sw128(sbase + L::kK, 16, 1024);
             const uint64_t v_desc0 = ptx::sdesc_sw128(sbase + L::kV, kBlockBytes, 1024);
@@ -315,32 +323,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tc_fence_after();
                     ready = true;
                 }
-                const uint64_t qd = q_desc0 + (uint64_t)a * kTileUnits;
-                const uint64_t kd = k_desc0 + (uint64_t)(j % KST) * kTileUnits;
-                const uint32_t d_s = tmem + (a == 0 ? 0u : 128u);
+                if (lane == 0) {
+                    const uint64_t qd = q_desc0 + (uint64_t)a * kTileUnits;
+                    const uint64_t kd = k_desc0 + (uint64_t)(j % KST) * kTileUnits;
+                    const uint32_t d_s = tmem + (a == 0 ? 0u : 128u);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    // K-major: +32 B per 16 elements, +16 KB per 64-column block
-                    const uint64_t off = (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
-                    ptx::umma_ss(d_s, qd + off, kd + off, kIdescS, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        // K-major: +32 B per 16 elements, +16 KB per 64-column block
+                        const uint64_t off =
+                            (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
+                        ptx::umma_ss(d_s, qd + off, kd + off, kIdescS, kk > 0);
+                    }
+                    ptx::umma_commit(&bars->s_full[a]);
                 }
-                ptx::umma_commit(&bars->s_full[a]);
+                __syncwarp();
             };
             auto issue_pv = [&](int a, int j) {
                 if (!wait_or_fail(&bars->p_full[a], j & 1, 5)) return;
                 if (!wait_or_fail(&bars->v_full[j % VST], (j / VST) & 1, 6)) return;
                 ptx::tc_fence_after();
-                const uint64_t vd = v_desc0 + (uint64_t)(j % VST) * kTileUnits;
-                const uint32_t d_o = tmem + (a == 0 ? 256u : 256u + D);
-                const uint32_t a_p = tmem + (a == 0 ? 0u : 128u);
-                const uint32_t acc0 = j > 0 ? 1u : 0u;
+                if (lane == 0) {
+                    const uint64_t vd = v_desc0 + (uint64_t)(j % VST) * kTileUnits;
+                    const uint32_t d_o = tmem + (a == 0 ? 256u : 256u + D);
+                    const uint32_t a_p = tmem + (a == 0 ? 0u : 128u);
+                    const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                    // MN-major V: +16 keys = +2 KB per step
-                    ptx::umma_ts(d_o, a_p + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), kIdescO,
-                                 kk > 0 ? 1u : acc0);
+                    for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                        // MN-major V: +16 keys = +2 KB per step
+                        ptx::umma_ts(d_o, a_p + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4),
+                                     kIdescO, kk > 0 ? 1u : acc0);
+                    }
+                    if (j == (a == 0 ? nt0 : nt1) - 1) ptx::umma_commit(&bars->o_done[a]);
                 }
-                if (j == (a == 0 ? nt0 : nt1) - 1) ptx::umma_commit(&bars->o_done[a]);
+                __syncwarp();
+            };
+            auto commit = [&](uint64_t* bar) {
+                if (lane == 0) ptx::umma_commit(bar);
+                __syncwarp();
             };
             for (int j = 0; ok && j <= nt; ++j) {
                 if (j < nt) {
@@ -352,16 +371,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (j >= 1 && j - 1 < nt1) {
                     issue_pv(1, j - 1);
                     if (!ok) break;
-                    ptx::umma_commit(&bars->v_empty[(j - 1) % VST]);
+                    commit(&bars->v_empty[(j - 1) % VST]);
                 }
                 if (j < nt) {
                     if (j < nt1) issue_s(1, j);
                     if (!ok) break;
-                    ptx::umma_commit(&bars->k_empty[j % KST]);
+                    commit(&bars->k_empty[j % KST]);
                     if (j < nt0) {
                         issue_pv(0, j);
                         if (!ok) break;
-                        if (j >= nt1) ptx::umma_commit(&bars->v_empty[j % VST]);
+                        if (j >= nt1) commit(&bars->v_empty[j % VST]);
                     }
                 }
             }
@@ -369,7 +388,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // make sure no MMA is still running before TMEM is freed
                 int zero = 0;
                 volatile int* no_abort = &zero;
-                ptx::umma_commit(&bars->drain);
+                if (lane == 0) ptx::umma_commit(&bars->drain);
+                __syncwarp();
                 ptx::mbar_wait(&bars->drain, 0, p.limit_ns, no_abort);
             }
         }
