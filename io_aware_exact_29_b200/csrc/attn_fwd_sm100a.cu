@@ -435,7 +435,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             l_half = l_half * alpha + (((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
             if (__any_sync(0xffffffffu, rescale)) {
                 // O must hold P_{j-1} V_{j-1} before it is rescaled (both
-                // halves of a row take the same decision)
+                // halves of a row take the same decision).  S_j being done
+                // implies P_{j-2} V_{j-2} is, so phase j-1 is the current or
+                // the previous phase of o_done and a parity wait is exact.
                 if (!warp_wait(&bars->o_done, (j - 1) & 1, p.limit_ns, abort_flag)) {
                     record_error(p.err, kErrFwdBase + 10, &bars->abort);
                     ok = false;
@@ -482,8 +484,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // ---- epilogue: O / l -> bf16/fp16 -> swizzled staging (the Q
         // buffer, free once the last S MMA is done) -> TMA store
+        // o_done completes once per P·V.  When the last tile's softmax ends,
+        // P_{nt-2}·V may still be pending (S_{nt-1} was issued before it), and a
+        // parity wait only tells the current phase from the one before it:
+        // wait for phase nt-2, then for phase nt-1.
         if (ok && nt > 0) {
-            if (!warp_wait(&bars->o_done, (nt - 1) & 1, p.limit_ns, abort_flag)) {
+            if ((nt >= 2 && !warp_wait(&bars->o_done, (nt - 2) & 1, p.limit_ns, abort_flag)) ||
+                !warp_wait(&bars->o_done, (nt - 1) & 1, p.limit_ns, abort_flag)) {
                 record_error(p.err, kErrFwdBase + 9, &bars->abort);
                 ok = false;
             }

@@ -30,7 +30,8 @@ def test_tiny(causal):
 @pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk", [(1, 1, 1, 128, 128), (2, 3, 3, 200, 333),
                                             (1, 8, 2, 257, 257), (2, 4, 1, 77, 300),
                                             (1, 2, 2, 300, 77), (3, 2, 1, 1, 129),
-                                            (1, 2, 2, 513, 1)])
+                                            (1, 2, 2, 513, 1), (4, 2, 2, 200, 300),
+                                            (1, 2, 1, 256, 256)])
 def test_ragged_and_grouped(B, Hq, Hkv, Nq, Nk, d, causal):
     c = FwdCase("r", B, Hq, Hkv, Nq, Nk, d, causal)
     check_fwd(fwd_inputs(c, seed=Nq + Nk + d), causal, c.scale,
