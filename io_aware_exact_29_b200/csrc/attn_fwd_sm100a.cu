@@ -8,21 +8,23 @@
 // effectstory.com article "FlashAttention：IO 感知的精確注意力演算法..." states
 // the same single pass: Q, K, V loaded once, O written once).
 //
-// Warp roles (320 threads):
-//   warps 0-7   softmax: warp w owns query rows 32*(w%4) .. +31 (its TMEM lane
-//               quarter) and score columns 64*(w/4) .. +63 of every tile, so
-//               two warps share each row and each SM sub-partition runs two
-//               softmax warps at once
-//   warp 8      TMA loader: Q once, then K_j / V_j into rings
-//   warp 9      tensor-memory owner and tcgen05.mma issuer (one lane)
+// Warp roles (576 threads):
+//   warps 0-15  softmax: warp w owns query rows 32*(w%4) .. +31 (its TMEM lane
+//               quarter) and score columns 32*(w/4) .. +31 of every tile:
+//               four warps share each row, four softmax warps per SM
+//               sub-partition hide each other's latencies
+//   warp 16     TMA loader: Q once, then K_j / V_j into rings
+//   warp 17     tensor-memory owner and tcgen05.mma issuer (one lane)
 // Tensor memory (512 columns): score buffers S[0] = [0,128) and S[1] =
 // [128,256) (double-buffered: S_{j+1} is computed while the softmax of tile j
-// runs), O accumulator [256, 256+D).  Each softmax thread reads its 64 scores
-// of S[j%2], agrees on the row maximum with its partner warp through shared
-// memory, keeps the running max m and its half of the running sum l (the
-// online softmax of the section above), and writes P (bf16/fp16) back over
-// the first 64 columns of S[j%2]; the P·V MMA reads P from tensor memory as its
-// A operand and V from shared memory.
+// runs), O accumulator [256, 256+D), Q [384, 384+D/2) (two 16-bit values per
+// column).  The softmax warps copy Q from shared memory into tensor memory
+// once, so S = Q·Kᵀ reads only K from shared memory.  Each softmax thread
+// reads its 32 scores of S[j%2], agrees on the row maximum with the three
+// other warps of its rows through shared memory, keeps the running max m and
+// its share of the running sum l (the online softmax of the section above),
+// and writes P (bf16/fp16) back over the first 64 columns of S[j%2]; the P·V
+// MMA reads P from tensor memory as its A operand and V from shared memory.
 //
 // MMA issue order: S_0, then per tile j: S_{j+1}, P_j·V_j.  MMAs from one
 // thread execute in issue order, so S_{j+1} (into the buffer of P_{j-1}) never
@@ -44,7 +46,8 @@ namespace {
 
 constexpr int kBlockM = 128;  // rows per Q tile
 constexpr int kBlockN = 128;  // keys per K/V tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
+constexpr int kSoftmaxWarps = 16;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 
@@ -54,9 +57,9 @@ struct FwdSmem {
     static constexpr uint32_t kQ = 0;
     static constexpr uint32_t kK = kQ + kTileBytes;
     static constexpr uint32_t kV = kK + KST * kTileBytes;
-    static constexpr uint32_t kRedMax = kV + VST * kTileBytes;  // [2 slots][2 halves][128] fp32
-    static constexpr uint32_t kRedSum = kRedMax + 2 * 2 * 128 * 4;  // [2 halves][128] fp32
-    static constexpr uint32_t kBars = kRedSum + 2 * 128 * 4;
+    static constexpr uint32_t kRedMax = kV + VST * kTileBytes;  // [2 slots][4 parts][128] fp32
+    static constexpr uint32_t kRedSum = kRedMax + 2 * 4 * 128 * 4;  // [4 parts][128] fp32
+    static constexpr uint32_t kBars = kRedSum + 4 * 128 * 4;
     static constexpr uint32_t kTotal = kBars + 512;
     static constexpr uint32_t kAlloc = kTotal + 1024;  // manual 1024-B alignment
 };
@@ -71,6 +74,7 @@ struct FwdBars {
     uint64_t s_full[2];
     uint64_t p_full[2];
     uint64_t o_done;
+    uint64_t q_tmem;  // Q copied into tensor memory
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -109,38 +113,37 @@ __device__ __forceinline__ int tiles_for(int q_first, int Nq, int Lk, int causal
     return nt;
 }
 
-// Running maxima of 64 score columns (two 32-column TMEM loads) into eight
-// independent chains of three-input maxima.  kMask: the tile reaches past
-// the row's last visible key (key_base + c > row_lim is masked).
+// Running maxima of 32 score columns (one 32-column TMEM load) into eight
+// independent chains.  kMask: the tile reaches past the row's last visible
+// key (key_base + c > row_lim is masked).
 template <bool kMask>
-__device__ __forceinline__ void half_max(const uint32_t (&r)[2][32], int key_base, int row_lim,
+__device__ __forceinline__ void part_max(const uint32_t (&r)[32], int key_base, int row_lim,
                                          float (&mx8)[8]) {
 #pragma unroll
-    for (int c = 0; c < 64; c += 16) {
+    for (int c = 0; c < 32; c += 16) {
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const int c0 = c + u, c1 = c + 8 + u;
-            float v0 = __uint_as_float(r[c0 >> 5][c0 & 31]);
-            float v1 = __uint_as_float(r[c1 >> 5][c1 & 31]);
+            float v0 = __uint_as_float(r[c + u]);
+            float v1 = __uint_as_float(r[c + 8 + u]);
             if (kMask) {
-                if (key_base + c0 > row_lim) v0 = -INFINITY;
-                if (key_base + c1 > row_lim) v1 = -INFINITY;
+                if (key_base + c + u > row_lim) v0 = -INFINITY;
+                if (key_base + c + 8 + u > row_lim) v1 = -INFINITY;
             }
             mx8[u] = ptx::max3(mx8[u], v0, v1);
         }
     }
 }
 
-// p = 2^(s * scale_log2 - m) for 64 score columns, accumulated into four
+// p = 2^(s * scale_log2 - m) for 32 score columns, accumulated into four
 // pair sums and packed two per 32-bit word (bf16 or fp16).
 template <bool kMask, bool BF16>
-__device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_base, int row_lim,
+__device__ __forceinline__ void part_exp(const uint32_t (&r)[32], int key_base, int row_lim,
                                          uint64_t sl2_2, uint64_t nm_2, uint64_t (&acc2)[4],
-                                         uint32_t (&pk)[32]) {
+                                         uint32_t (&pk)[16]) {
 #pragma unroll
-    for (int c = 0; c < 64; c += 2) {
-        float v0 = __uint_as_float(r[c >> 5][c & 31]);
-        float v1 = __uint_as_float(r[c >> 5][(c & 31) + 1]);
+    for (int c = 0; c < 32; c += 2) {
+        float v0 = __uint_as_float(r[c]);
+        float v1 = __uint_as_float(r[c + 1]);
         if (kMask) {
             if (key_base + c > row_lim) v0 = -INFINITY;
             if (key_base + c + 1 > row_lim) v1 = -INFINITY;
@@ -175,7 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kIdescS = ptx::idesc_f16(kBlockM, kBlockN, BF16, false);
     constexpr uint32_t kIdescO = ptx::idesc_f16(kBlockM, D, BF16, true);
     constexpr uint32_t kColO = 256;
-    constexpr int kHalfD = D / 2;  // O columns per softmax half
+    constexpr uint32_t kColQ = 384;
+    constexpr int kPartD = D / 4;  // O columns per softmax warp
+    constexpr int kLoaderWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = ptx::smem_u32(smem_raw);
@@ -209,20 +214,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(&bars->s_full[s], 1);
-            ptx::mbar_init(&bars->p_full[s], 256);
+            ptx::mbar_init(&bars->p_full[s], 32 * kSoftmaxWarps);
         }
         ptx::mbar_init(&bars->o_done, 1);
+        ptx::mbar_init(&bars->q_tmem, 32 * kSoftmaxWarps);
         ptx::mbar_init(&bars->drain, 1);
         bars->abort = 0;
         ptx::fence_barrier_init();
     }
-    if (warp == 8 && lane == 0) {
+    if (warp == kLoaderWarp && lane == 0) {
         ptx::prefetch_tmap(&tm_q);
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_v);
         ptx::prefetch_tmap(&tm_o);
     }
-    if (warp == 9) {
+    if (warp == kMmaWarp) {
         ptx::tmem_alloc<kTmemCols>(&bars->tmem_base);
         ptx::tmem_relinquish();
     }
@@ -233,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // The loader and MMA loops run on all 32 lanes of their warp; one lane
     // issues the copies and MMAs, and every wait's outcome is warp-uniform.
-    if (warp == 8) {
+    if (warp == kLoaderWarp) {
         // ================================================= TMA loader
         if (nt > 0 && !p.inject) {
             int issued_k = 0, issued_v = 0;
@@ -283,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = max(0, issued_v - VST); j < issued_v; ++j)
                 ptx::mbar_wait(&bars->v_full[j % VST], (j / VST) & 1, p.limit_ns, no_abort);
         }
-    } else if (warp == 9) {
+    } else if (warp == kMmaWarp) {
         // ================================================= MMA issuer
         if (nt > 0) {
             bool ok = true;
@@ -296,7 +302,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             // Descriptors are built once; each MMA adds a compile-time offset
             // (in 16-byte units) to a base descriptor.
-            const uint64_t q_desc = ptx::sdesc_sw128(sbase + L::kQ, 16, 1024);
             const uint64_t k_desc0 = ptx::sdesc_sw128(sbase + L::kK, 16, 1024);
             const uint64_t v_desc0 = ptx::sdesc_sw128(sbase + L::kV, kBlockBytes, 1024);
             constexpr uint64_t kTileUnits = kTileBytes >> 4;
@@ -308,17 +313,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t d_s = tmem + (uint32_t)((j & 1) * kBlockN);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        // K-major: +32 B per 16 elements, +16 KB per 64-column block
+                        // A = Q from tensor memory (8 columns per 16 values);
+                        // B = K, K-major: +32 B per 16 values, +16 KB per block
                         const uint64_t off =
                             (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
-                        ptx::umma_ss(d_s, q_desc + off, kd + off, kIdescS, kk > 0);
+                        ptx::umma_ts(d_s, tmem + kColQ + kk * 8, kd + off, kIdescS, kk > 0);
                     }
                     ptx::umma_commit(&bars->s_full[j & 1]);
                     ptx::umma_commit(&bars->k_empty[j % KST]);
                 }
                 __syncwarp();
             };
-            if (wait_or_fail(&bars->q_full, 0, 3)) {
+            if (wait_or_fail(&bars->q_tmem, 0, 3)) {
                 ptx::tc_fence_after();
                 issue_s(0);
             }
@@ -358,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ================================================= softmax warps
         const uint32_t quarter = (uint32_t)(warp & 3);
-        const int hf = warp >> 2;  // which 64 score columns
+        const int part = warp >> 2;  // which 32 score columns / D/4 output columns
         const uint32_t row = quarter * 32u + (uint32_t)lane;
         const uint32_t lane_addr = (quarter * 32u) << 16;
         const int i = q0 + (int)row;
@@ -366,16 +372,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p.causal) row_lim = min(row_lim, i + Lk - p.Nq);
         const float sl2 = p.scale_log2;
         float m_ref = -INFINITY;  // running reference max, scale*log2 units
-        float l_half = 0.f;       // this half's running sum of exp2(s*sl2 - m_ref)
+        float l_part = 0.f;       // this warp's share of the running sum
         bool ok = true;
         float* red_max = reinterpret_cast<float*>(smem + L::kRedMax);
         float* red_sum = reinterpret_cast<float*>(smem + L::kRedSum);
-        const uint32_t pair_bar = 1 + quarter;  // warps quarter and quarter + 4
-        const uint32_t t_o = tmem + lane_addr + kColO + (uint32_t)(hf * kHalfD);
+        const uint32_t row_bar = 1 + quarter;  // the four warps of these rows
+        const uint32_t t_o = tmem + lane_addr + kColO + (uint32_t)(part * kPartD);
 
-        // Every warp walks all nt iterations and reaches every pair barrier,
+        // ---- Q -> tensor memory (A operand of S = Q Kᵀ): this warp copies
+        // d values [32 part, 32 part + 32) of its rows, two per column
+        if (nt > 0) {
+            if (!warp_wait(&bars->q_full, 0, p.limit_ns, abort_flag)) {
+                record_error(p.err, kErrFwdBase + 11, &bars->abort);
+                ok = false;
+            } else if (part * 32 < D) {
+                const int c0 = part * 32;  // first d value
+                const uint8_t* qrow = smem + L::kQ + (c0 >> 6) * kBlockBytes;
+                uint32_t qv[16];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const uint4 v4 = *reinterpret_cast<const uint4*>(
+                        qrow + sw128_offset(row, (uint32_t)(((c0 & 63) >> 3) + q4)));
+                    qv[4 * q4] = v4.x;
+                    qv[4 * q4 + 1] = v4.y;
+                    qv[4 * q4 + 2] = v4.z;
+                    qv[4 * q4 + 3] = v4.w;
+                }
+                ptx::tmem_st16(tmem + lane_addr + kColQ + (uint32_t)(c0 >> 1), qv);
+                ptx::tmem_wait_st();
+            }
+            ptx::tc_fence_before();
+            if (ok) ptx::mbar_arrive(&bars->q_tmem);
+        }
+
+        // Every warp walks all nt iterations and reaches every row barrier,
         // also after a failed wait (then it only skips its work), so that its
-        // partner can never be left waiting at a barrier.
+        // partners can never be left waiting at a barrier.
         for (int j = 0; j < nt; ++j) {
             const int sb = j & 1;
             if (ok && !warp_wait(&bars->s_full[sb], (j >> 1) & 1, p.limit_ns, abort_flag)) {
@@ -383,31 +415,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = false;
             }
             const uint32_t t_s = tmem + lane_addr + (uint32_t)(sb * kBlockN);
-            const int key_base = j * kBlockN + hf * 64;
-            const bool masked = key_base + 63 > row_lim;
-            uint32_t r[2][32];
+            const int key_base = j * kBlockN + part * 32;
+            const bool masked = key_base + 31 > row_lim;
+            uint32_t r[32];
             float pmax = -INFINITY;
             if (ok) {
                 ptx::tc_fence_after();
-                ptx::tmem_ld32(t_s + hf * 64, r[0]);
-                ptx::tmem_ld32(t_s + hf * 64 + 32, r[1]);
+                ptx::tmem_ld32(t_s + part * 32, r);
                 float mx8[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
-                ptx::tmem_wait_ld_dep(r[0]);
-                ptx::tmem_wait_ld_dep(r[1]);
+                ptx::tmem_wait_ld_dep(r);
                 if (masked)
-                    half_max<true>(r, key_base, row_lim, mx8);
+                    part_max<true>(r, key_base, row_lim, mx8);
                 else
-                    half_max<false>(r, key_base, row_lim, mx8);
+                    part_max<false>(r, key_base, row_lim, mx8);
                 pmax = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]),
                                  ptx::max3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
             }
-            // the row maximum over both halves, through shared memory
-            red_max[((j & 1) * 2 + hf) * 128 + row] = pmax;
-            ptx::named_barrier_sync(pair_bar, 64);
+            // the row maximum over the four parts, through shared memory
+            red_max[((j & 1) * 4 + part) * 128 + row] = pmax;
+            ptx::named_barrier_sync(row_bar, 128);
             if (!ok) continue;
-            const float mx = fmaxf(pmax, red_max[((j & 1) * 2 + (hf ^ 1)) * 128 + row]);
+            const float* rm = red_max + (j & 1) * 4 * 128 + row;
+            const float mx = fmaxf(ptx::max3(rm[0], rm[128], rm[256]), rm[384]);
             const float m_tile = mx * sl2;  // -inf stays -inf (sl2 > 0)
             float alpha = 1.f;
             bool rescale = false;
@@ -418,24 +449,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
             uint64_t acc2[4] = {0, 0, 0, 0};  // four pair accumulators of the row sum
-            uint32_t pk[32];
+            uint32_t pk[16];
             if (masked)
-                half_exp<true, BF16>(r, key_base, row_lim, ptx::f2_pack(sl2, sl2),
+                part_exp<true, BF16>(r, key_base, row_lim, ptx::f2_pack(sl2, sl2),
                                      ptx::f2_pack(-m_use, -m_use), acc2, pk);
             else
-                half_exp<false, BF16>(r, key_base, row_lim, ptx::f2_pack(sl2, sl2),
+                part_exp<false, BF16>(r, key_base, row_lim, ptx::f2_pack(sl2, sl2),
                                       ptx::f2_pack(-m_use, -m_use), acc2, pk);
-            // P of these 64 keys over columns [32 hf, 32 hf + 32) of S[sb]
-            ptx::tmem_st32(t_s + hf * 32, pk);
+            // P of these 32 keys over columns [16 part, 16 part + 16) of S[sb]
+            ptx::tmem_st16(t_s + part * 16, pk);
             float s0, s1, s2, s3, s4, s5, s6, s7;
             ptx::f2_unpack(acc2[0], s0, s1);
             ptx::f2_unpack(acc2[1], s2, s3);
             ptx::f2_unpack(acc2[2], s4, s5);
             ptx::f2_unpack(acc2[3], s6, s7);
-            l_half = l_half * alpha + (((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
+            l_part = l_part * alpha + (((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
             if (__any_sync(0xffffffffu, rescale)) {
-                // O must hold P_{j-1} V_{j-1} before it is rescaled (both
-                // halves of a row take the same decision).  S_j being done
+                // O must hold P_{j-1} V_{j-1} before it is rescaled (all four
+                // warps of a row take the same decision).  S_j being done
                 // implies P_{j-2} V_{j-2} is, so phase j-1 is the current or
                 // the previous phase of o_done and a parity wait is exact.
                 if (!warp_wait(&bars->o_done, (j - 1) & 1, p.limit_ns, abort_flag)) {
@@ -446,18 +477,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ptx::tc_fence_after();
                 const float sc = rescale ? alpha : 1.f;
-#pragma unroll 1
-                for (int c = 0; c < kHalfD / 32; ++c) {
+                if constexpr (kPartD == 32) {
                     uint32_t o[32];
-                    ptx::tmem_ld32(t_o + c * 32, o);
+                    ptx::tmem_ld32(t_o, o);
                     ptx::tmem_wait_ld_dep(o);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * sc);
-                    ptx::tmem_st32(t_o + c * 32, o);
+                    ptx::tmem_st32(t_o, o);
+                } else {
+                    uint32_t o[16];
+                    ptx::tmem_ld16(t_o, o);
+                    ptx::tmem_wait_ld_dep16(o);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * sc);
+                    ptx::tmem_st16(t_o, o);
                 }
             }
             ptx::tmem_wait_st();
-            const bool zero_v = p.seqlens_k != nullptr && j * kBlockN + kBlockN > Lk && hf == 0;
+            const bool zero_v = p.seqlens_k != nullptr && j * kBlockN + kBlockN > Lk && part == 0;
             if (zero_v) {
                 // keys behind the real length: zero their V rows so that a
                 // non-finite value stored there cannot reach O through 0 * NaN
@@ -483,11 +520,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 
         // ---- epilogue: O / l -> bf16/fp16 -> swizzled staging (the Q
-        // buffer, free once the last S MMA is done) -> TMA store
-        // o_done completes once per P·V.  When the last tile's softmax ends,
-        // P_{nt-2}·V may still be pending (S_{nt-1} was issued before it), and a
-        // parity wait only tells the current phase from the one before it:
-        // wait for phase nt-2, then for phase nt-1.
+        // buffer, free once Q is in tensor memory and the last MMA is done)
+        // -> TMA store.  o_done completes once per P·V.  When the last tile's
+        // softmax ends, P_{nt-2}·V may still be pending (S_{nt-1} was issued
+        // before it), and a parity wait only tells the current phase from the
+        // one before it: wait for phase nt-2, then for phase nt-1.
         if (ok && nt > 0) {
             if ((nt >= 2 && !warp_wait(&bars->o_done, (nt - 2) & 1, p.limit_ns, abort_flag)) ||
                 !warp_wait(&bars->o_done, (nt - 1) & 1, p.limit_ns, abort_flag)) {
@@ -496,50 +533,52 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ptx::tc_fence_after();
         }
-        // both halves' sums of the row
-        red_sum[hf * 128 + row] = l_half;
-        ptx::named_barrier_sync(pair_bar, 64);
-        const float l_sum = l_half + red_sum[(hf ^ 1) * 128 + row];
+        // the four parts' sums of the row
+        red_sum[part * 128 + row] = l_part;
+        ptx::named_barrier_sync(row_bar, 128);
+        const float l_sum = (red_sum[row] + red_sum[128 + row]) + (red_sum[256 + row] + red_sum[384 + row]);
         const bool have = ok && nt > 0 && l_sum > 0.f;
         const float inv_l = have ? 1.f / l_sum : 0.f;
         uint8_t* stage = smem + L::kQ;
         if (q0 < p.Nq) {
-#pragma unroll
-            for (int c = 0; c < kHalfD / 32; ++c) {
-                uint32_t o[32];
-                if (ok && nt > 0) {
-                    ptx::tmem_ld32(t_o + c * 32, o);
+            uint32_t o[kPartD];
+            if (ok && nt > 0) {
+                if constexpr (kPartD == 32) {
+                    ptx::tmem_ld32(t_o, o);
                     ptx::tmem_wait_ld_dep(o);
                 } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = 0u;
+                    ptx::tmem_ld16(t_o, o);
+                    ptx::tmem_wait_ld_dep16(o);
                 }
-                uint32_t o2[16];
+            } else {
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    o2[e] = ptx::pack2<BF16>(__uint_as_float(o[2 * e]) * inv_l,
-                                             __uint_as_float(o[2 * e + 1]) * inv_l);
-                // output columns hf * D/2 + 32 c .. +31: 128-byte block col / 64,
-                // 16-byte chunks (col % 64) / 8 .. +3
-                const int col = hf * kHalfD + c * 32;
+                for (int e = 0; e < kPartD; ++e) o[e] = 0u;
+            }
+            uint32_t o2[kPartD / 2];
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const uint32_t ch = (uint32_t)(((col & 63) >> 3) + q4);
-                    *reinterpret_cast<uint4*>(stage + (col >> 6) * kBlockBytes +
-                                              sw128_offset(row, ch)) =
-                        make_uint4(o2[q4 * 4], o2[q4 * 4 + 1], o2[q4 * 4 + 2], o2[q4 * 4 + 3]);
-                }
+            for (int e = 0; e < kPartD / 2; ++e)
+                o2[e] = ptx::pack2<BF16>(__uint_as_float(o[2 * e]) * inv_l,
+                                         __uint_as_float(o[2 * e + 1]) * inv_l);
+            // output columns part * D/4 .. +D/4: 128-byte block col / 64,
+            // 16-byte chunks (col % 64) / 8 ..
+            const int col = part * kPartD;
+#pragma unroll
+            for (int q4 = 0; q4 < kPartD / 8; ++q4) {
+                const uint32_t ch = (uint32_t)(((col & 63) >> 3) + q4);
+                *reinterpret_cast<uint4*>(stage + (col >> 6) * kBlockBytes +
+                                          sw128_offset(row, ch)) =
+                    make_uint4(o2[q4 * 4], o2[q4 * 4 + 1], o2[q4 * 4 + 2], o2[q4 * 4 + 3]);
             }
             ptx::fence_proxy_async_smem();
         }
-        ptx::named_barrier_sync(5, 256);
+        ptx::named_barrier_sync(5, 32 * kSoftmaxWarps);
         if (warp == 0 && lane == 0 && q0 < p.Nq) {
             for (int c = 0; c < kDBlocks; ++c)
                 ptx::tma_store_4d(&tm_o, stage + c * kBlockBytes, c * 64, h, q0, b);
             ptx::bulk_commit_group();
             ptx::bulk_wait_group_read0();
         }
-        if (hf == 0 && i < p.Nq) {
+        if (part == 0 && i < p.Nq) {
             const float lse = have ? (m_ref + ptx::lg2_approx(l_sum)) * 0.69314718055994531f
                                    : -INFINITY;
             p.lse[((size_t)b * p.Hq + h) * p.Nq + i] = lse;
@@ -548,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == kMmaWarp) {
         __syncwarp();
         ptx::tc_fence_after();
         ptx::tmem_dealloc<kTmemCols>(tmem);
