@@ -214,10 +214,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(&bars->s_full[s], 1);
-            ptx::mbar_init(&bars->p_full[s], 32 * kSoftmaxWarps);
+            ptx::mbar_init(&bars->p_full[s], kSoftmaxWarps);  // one arrival per warp
         }
         ptx::mbar_init(&bars->o_done, 1);
-        ptx::mbar_init(&bars->q_tmem, 32 * kSoftmaxWarps);
+        ptx::mbar_init(&bars->q_tmem, kSoftmaxWarps);
         ptx::mbar_init(&bars->drain, 1);
         bars->abort = 0;
         ptx::fence_barrier_init();
@@ -308,20 +308,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto issue_s = [&](int j) {
                 if (!wait_or_fail(&bars->k_full[j % KST], (j / KST) & 1, 4)) return;
                 ptx::tc_fence_after();
-                if (lane == 0) {
-                    const uint64_t kd = k_desc0 + (uint64_t)(j % KST) * kTileUnits;
-                    const uint32_t d_s = tmem + (uint32_t)((j & 1) * kBlockN);
+                const uint64_t kd = k_desc0 + (uint64_t)(j % KST) * kTileUnits;
+                const uint32_t d_s = tmem + (uint32_t)((j & 1) * kBlockN);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        // A = Q from tensor memory (8 columns per 16 values);
-                        // B = K, K-major: +32 B per 16 values, +16 KB per block
-                        const uint64_t off =
-                            (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
-                        ptx::umma_ts(d_s, tmem + kColQ + kk * 8, kd + off, kIdescS, kk > 0);
-                    }
-                    ptx::umma_commit(&bars->s_full[j & 1]);
-                    ptx::umma_commit(&bars->k_empty[j % KST]);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    // A = Q from tensor memory (8 columns per 16 values);
+                    // B = K, K-major: +32 B per 16 values, +16 KB per block
+                    const uint64_t off = (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
+                    ptx::umma_ts_elect(d_s, tmem + kColQ + kk * 8, kd + off, kIdescS, kk > 0);
                 }
+                ptx::umma_commit_elect(&bars->s_full[j & 1]);
+                ptx::umma_commit_elect(&bars->k_empty[j % KST]);
                 __syncwarp();
             };
             if (wait_or_fail(&bars->q_tmem, 0, 3)) {
@@ -336,19 +333,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_or_fail(&bars->p_full[j & 1], (j >> 1) & 1, 5)) break;
                 if (!wait_or_fail(&bars->v_full[j % VST], (j / VST) & 1, 6)) break;
                 ptx::tc_fence_after();
-                if (lane == 0) {
+                {
                     const uint64_t vd = v_desc0 + (uint64_t)(j % VST) * kTileUnits;
                     const uint32_t a_p = tmem + (uint32_t)((j & 1) * kBlockN);
                     const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
                     for (int kk = 0; kk < kBlockN / 16; ++kk) {
                         // MN-major V: +16 keys = +2 KB per step
-                        ptx::umma_ts(tmem + kColO, a_p + kk * 8,
-                                     vd + (uint64_t)((kk * 16 * 128) >> 4), kIdescO,
-                                     kk > 0 ? 1u : acc0);
+                        ptx::umma_ts_elect(tmem + kColO, a_p + kk * 8,
+                                           vd + (uint64_t)((kk * 16 * 128) >> 4), kIdescO,
+                                           kk > 0 ? 1u : acc0);
                     }
-                    ptx::umma_commit(&bars->o_done);
-                    ptx::umma_commit(&bars->v_empty[j % VST]);
+                    ptx::umma_commit_elect(&bars->o_done);
+                    ptx::umma_commit_elect(&bars->v_empty[j % VST]);
                 }
                 __syncwarp();
             }
@@ -356,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // make sure no MMA is still running before TMEM is freed
                 int zero = 0;
                 volatile int* no_abort = &zero;
-                if (lane == 0) ptx::umma_commit(&bars->drain);
+                ptx::umma_commit_elect(&bars->drain);
                 __syncwarp();
                 ptx::mbar_wait(&bars->drain, 0, p.limit_ns, no_abort);
             }
@@ -402,7 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tmem_wait_st();
             }
             ptx::tc_fence_before();
-            if (ok) ptx::mbar_arrive(&bars->q_tmem);
+            __syncwarp();
+            if (ok && lane == 0) ptx::mbar_arrive(&bars->q_tmem);
         }
 
         // Every warp walks all nt iterations and reaches every row barrier,
@@ -515,8 +513,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ptx::fence_proxy_async_smem();
             }
+            // each thread's P stores are complete (wait::st above); one
+            // arrival per warp after the warp has converged
             ptx::tc_fence_before();
-            ptx::mbar_arrive(&bars->p_full[sb]);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&bars->p_full[sb]);
         }
 
         // ---- epilogue: O / l -> bf16/fp16 -> swizzled staging (the Q
