@@ -1,34 +1,30 @@
 // attn_fwd_sm100a.cu -- exact attention forward on tcgen05 tensor cores.
 //
-// One CTA owns one 128-row tile of queries of one (batch, head) and streams
-// the key/value tiles of its head through shared memory (ai6s.net article on
-// the ops-transformer FlashAttention operator, section "FlashAttention 拆的不是
-// 算法，是数据流": split Q, K, V along the sequence into on-chip tiles, run
-// Q_tile·K_tileᵀ -> softmax -> ·V_tile on chip, write back only O; the
-// effectstory.com article "FlashAttention：IO 感知的精確注意力演算法..." states
-// the same single pass: Q, K, V loaded once, O written once).
+// One CTA owns two 128-row tiles of queries (Q0, Q1) of one (batch, head) and
+// streams the key/value tiles of its head through shared memory once for both
+// (ai6s.net article on the ops-transformer FlashAttention operator, section
+// "FlashAttention 拆的不是算法，是数据流": split Q, K, V along the sequence into
+// on-chip tiles, run Q_tile·K_tileᵀ -> softmax -> ·V_tile on chip, write back
+// only O; the effectstory.com article "FlashAttention：IO 感知的精確注意力演算
+// 法..." states the same single pass: Q, K, V loaded once, O written once).
 //
-// Warp roles (576 threads):
-//   warps 0-15  softmax: warp w owns query rows 32*(w%4) .. +31 (its TMEM lane
-//               quarter) and score columns 32*(w/4) .. +31 of every tile:
-//               four warps share each row, four softmax warps per SM
-//               sub-partition hide each other's latencies
-//   warp 16     TMA loader: Q once, then K_j / V_j into rings
-//   warp 17     tensor-memory owner and tcgen05.mma issuer (one lane)
-// Tensor memory (512 columns): score buffers S[0] = [0,128) and S[1] =
-// [128,256) (double-buffered: S_{j+1} is computed while the softmax of tile j
-// runs), O accumulator [256, 256+D), Q [384, 384+D/2) (two 16-bit values per
-// column).  The softmax warps copy Q from shared memory into tensor memory
-// once, so S = Q·Kᵀ reads only K from shared memory.  Each softmax thread
-// reads its 32 scores of S[j%2], agrees on the row maximum with the three
-// other warps of its rows through shared memory, keeps the running max m and
-// its share of the running sum l (the online softmax of the section above),
-// and writes P (bf16/fp16) back over the first 64 columns of S[j%2]; the P·V
-// MMA reads P from tensor memory as its A operand and V from shared memory.
+// Warp roles (320 threads):
+//   warps 0-3   softmax of Q0 (thread t owns query row t = TMEM lane t)
+//   warps 4-7   softmax of Q1
+//   warp 8      TMA loader: Q0, Q1 once, then K_j / V_j into rings
+//   warp 9      tensor-memory owner and single-thread tcgen05.mma issuer
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
+// O1 [256+D, 256+2D).  Each softmax thread reads its score row from S_a,
+// keeps the running max m and sum l (the online softmax of the section above),
+// and writes P (bf16/fp16) back over the first 64 columns of S_a; the P·V MMA
+// reads P straight from tensor memory as its A operand, V from shared memory.
 //
-// MMA issue order: S_0, then per tile j: S_{j+1}, P_j·V_j.  MMAs from one
-// thread execute in issue order, so S_{j+1} (into the buffer of P_{j-1}) never
-// overtakes P_{j-1}·V_{j-1}.
+// MMA issue order per key tile j:  S0_j, PV1_{j-1}, S1_j, PV0_j.  While the
+// softmax of Q0 works on S0_j the tensor core runs PV1_{j-1} and S1_j, and
+// while the softmax of Q1 works on S1_j it runs PV0_j and S0_{j+1}.  MMAs from
+// one thread execute in issue order, so when S_a_j is complete the previous
+// P_a·V has finished reading P_a and updating O_a: the softmax may rescale
+// O_a and overwrite P_a without another wait.
 //
 // Fused masks: the causal rule (adaptation point 2 of the ai6s.net article)
 // and the per-sequence key length (point 3) are index arithmetic on the score
@@ -46,35 +42,31 @@ namespace {
 
 constexpr int kBlockM = 128;  // rows per Q tile
 constexpr int kBlockN = 128;  // keys per K/V tile
-constexpr int kThreads = 576;
-constexpr int kSoftmaxWarps = 16;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 
 template <int D, int KST, int VST>
 struct FwdSmem {
     static constexpr uint32_t kTileBytes = kBlockM * D * 2;  // one 128 x D tile
-    static constexpr uint32_t kQ = 0;
-    static constexpr uint32_t kK = kQ + kTileBytes;
+    static constexpr uint32_t kQ = 0;                          // Q0, Q1
+    static constexpr uint32_t kK = kQ + 2 * kTileBytes;
     static constexpr uint32_t kV = kK + KST * kTileBytes;
-    static constexpr uint32_t kRedMax = kV + VST * kTileBytes;  // [2 slots][4 parts][128] fp32
-    static constexpr uint32_t kRedSum = kRedMax + 2 * 4 * 128 * 4;  // [4 parts][128] fp32
-    static constexpr uint32_t kBars = kRedSum + 4 * 128 * 4;
+    static constexpr uint32_t kBars = kV + VST * kTileBytes;
     static constexpr uint32_t kTotal = kBars + 512;
     static constexpr uint32_t kAlloc = kTotal + 1024;  // manual 1024-B alignment
 };
 
 template <int KST, int VST>
 struct FwdBars {
-    uint64_t q_full;
+    uint64_t q_full[2];
     uint64_t k_full[KST];
     uint64_t k_empty[KST];
     uint64_t v_full[VST];
     uint64_t v_empty[VST];
     uint64_t s_full[2];
     uint64_t p_full[2];
-    uint64_t o_done;
-    uint64_t q_tmem;  // Q copied into tensor memory
+    uint64_t o_done[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -113,37 +105,38 @@ __device__ __forceinline__ int tiles_for(int q_first, int Nq, int Lk, int causal
     return nt;
 }
 
-// Running maxima of 32 score columns (one 32-column TMEM load) into eight
-// independent chains.  kMask: the tile reaches past the row's last visible
-// key (key_base + c > row_lim is masked).
+// Running maxima of 64 score columns (two 32-column TMEM loads) into eight
+// independent chains of three-input maxima.  kMask: the tile reaches past
+// the row's last visible key (key_base + c > row_lim is masked).
 template <bool kMask>
-__device__ __forceinline__ void part_max(const uint32_t (&r)[32], int key_base, int row_lim,
+__device__ __forceinline__ void half_max(const uint32_t (&r)[2][32], int key_base, int row_lim,
                                          float (&mx8)[8]) {
 #pragma unroll
-    for (int c = 0; c < 32; c += 16) {
+    for (int c = 0; c < 64; c += 16) {
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            float v0 = __uint_as_float(r[c + u]);
-            float v1 = __uint_as_float(r[c + 8 + u]);
+            const int c0 = c + u, c1 = c + 8 + u;
+            float v0 = __uint_as_float(r[c0 >> 5][c0 & 31]);
+            float v1 = __uint_as_float(r[c1 >> 5][c1 & 31]);
             if (kMask) {
-                if (key_base + c + u > row_lim) v0 = -INFINITY;
-                if (key_base + c + 8 + u > row_lim) v1 = -INFINITY;
+                if (key_base + c0 > row_lim) v0 = -INFINITY;
+                if (key_base + c1 > row_lim) v1 = -INFINITY;
             }
             mx8[u] = ptx::max3(mx8[u], v0, v1);
         }
     }
 }
 
-// p = 2^(s * scale_log2 - m) for 32 score columns, accumulated into four
+// p = 2^(s * scale_log2 - m) for 64 score columns, accumulated into four
 // pair sums and packed two per 32-bit word (bf16 or fp16).
 template <bool kMask, bool BF16>
-__device__ __forceinline__ void part_exp(const uint32_t (&r)[32], int key_base, int row_lim,
+__device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_base, int row_lim,
                                          uint64_t sl2_2, uint64_t nm_2, uint64_t (&acc2)[4],
-                                         uint32_t (&pk)[16]) {
+                                         uint32_t (&pk)[32]) {
 #pragma unroll
-    for (int c = 0; c < 32; c += 2) {
-        float v0 = __uint_as_float(r[c]);
-        float v1 = __uint_as_float(r[c + 1]);
+    for (int c = 0; c < 64; c += 2) {
+        float v0 = __uint_as_float(r[c >> 5][c & 31]);
+        float v1 = __uint_as_float(r[c >> 5][(c & 31) + 1]);
         if (kMask) {
             if (key_base + c > row_lim) v0 = -INFINITY;
             if (key_base + c + 1 > row_lim) v1 = -INFINITY;
@@ -177,10 +170,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kBlockBytes = kBlockM * 128;
     constexpr uint32_t kIdescS = ptx::idesc_f16(kBlockM, kBlockN, BF16, false);
     constexpr uint32_t kIdescO = ptx::idesc_f16(kBlockM, D, BF16, true);
-    constexpr uint32_t kColO = 256;
-    constexpr uint32_t kColQ = 384;
-    constexpr int kPartD = D / 4;  // O columns per softmax warp
-    constexpr int kLoaderWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = ptx::smem_u32(smem_raw);
@@ -193,17 +182,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = tid >> 5;
     const int lane = tid & 31;
 
-    // ---- work unit: rows [q0, q0 + 128) of head h of batch b
-    const int qt = p.causal ? (p.n_qtiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+    // ---- work unit: rows [qbase, qbase + 256) of head h of batch b
+    const int n_ctiles = (p.Nq + 2 * kBlockM - 1) / (2 * kBlockM);
+    const int ct = p.causal ? (n_ctiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;
     const int h = blockIdx.y;
     const int b = blockIdx.z;
     const int g = h / p.G;
     const int Lk = p.seqlens_k ? p.seqlens_k[b] : p.Nk;
-    const int q0 = qt * kBlockM;
-    const int nt = tiles_for(q0, p.Nq, Lk, p.causal);
+    const int qbase = ct * 2 * kBlockM;
+    const int nt0 = tiles_for(qbase, p.Nq, Lk, p.causal);
+    const int nt1 = tiles_for(qbase + kBlockM, p.Nq, Lk, p.causal);
+    const int nt = max(nt0, nt1);
 
     if (tid == 0) {
-        ptx::mbar_init(&bars->q_full, 1);
+        for (int a = 0; a < 2; ++a) {
+            ptx::mbar_init(&bars->q_full[a], 1);
+            ptx::mbar_init(&bars->s_full[a], 1);
+            ptx::mbar_init(&bars->p_full[a], 128);
+            ptx::mbar_init(&bars->o_done[a], 1);
+        }
         for (int s = 0; s < KST; ++s) {
             ptx::mbar_init(&bars->k_full[s], 1);
             ptx::mbar_init(&bars->k_empty[s], 1);
@@ -212,23 +209,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&bars->v_full[s], 1);
             ptx::mbar_init(&bars->v_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            ptx::mbar_init(&bars->s_full[s], 1);
-            ptx::mbar_init(&bars->p_full[s], kSoftmaxWarps);  // one arrival per warp
-        }
-        ptx::mbar_init(&bars->o_done, 1);
-        ptx::mbar_init(&bars->q_tmem, kSoftmaxWarps);
         ptx::mbar_init(&bars->drain, 1);
         bars->abort = 0;
         ptx::fence_barrier_init();
     }
-    if (warp == kLoaderWarp && lane == 0) {
+    if (warp == 8 && lane == 0) {
         ptx::prefetch_tmap(&tm_q);
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_v);
         ptx::prefetch_tmap(&tm_o);
     }
-    if (warp == kMmaWarp) {
+    if (warp == 9) {
         ptx::tmem_alloc<kTmemCols>(&bars->tmem_base);
         ptx::tmem_relinquish();
     }
@@ -237,45 +228,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    // The loader and MMA loops run on all 32 lanes of their warp; one lane
-    // issues the copies and MMAs, and every wait's outcome is warp-uniform.
-    if (warp == kLoaderWarp) {
+    if (warp == 8) {
         // ================================================= TMA loader
-        if (nt > 0 && !p.inject) {
+        if (lane == 0 && nt > 0 && !p.inject) {
             int issued_k = 0, issued_v = 0;
-            if (lane == 0) {
-                ptx::mbar_arrive_expect_tx(&bars->q_full, kTileBytes);
+            bool issued_q[2] = {false, false};
+            for (int a = 0; a < 2; ++a) {
+                if ((a == 0 ? nt0 : nt1) == 0) continue;
+                ptx::mbar_arrive_expect_tx(&bars->q_full[a], kTileBytes);
                 for (int c = 0; c < kDBlocks; ++c)
-                    ptx::tma_load_4d(smem + L::kQ + c * kBlockBytes, &tm_q, &bars->q_full, c * 64,
-                                     h, q0, b);
+                    ptx::tma_load_4d(smem + L::kQ + a * kTileBytes + c * kBlockBytes, &tm_q,
+                                     &bars->q_full[a], c * 64, h, qbase + a * kBlockM, b);
+                issued_q[a] = true;
             }
-            __syncwarp();
             for (int j = 0; j < nt; ++j) {
                 const int sk = j % KST;
-                if (!warp_wait(&bars->k_empty[sk], ((j / KST) & 1) ^ 1, p.limit_ns, abort_flag)) {
+                if (!ptx::mbar_wait(&bars->k_empty[sk], ((j / KST) & 1) ^ 1, p.limit_ns,
+                                    abort_flag)) {
                     record_error(p.err, kErrFwdBase + 1, &bars->abort);
                     break;
                 }
-                if (lane == 0) {
-                    ptx::mbar_arrive_expect_tx(&bars->k_full[sk], kTileBytes);
-                    for (int c = 0; c < kDBlocks; ++c)
-                        ptx::tma_load_4d(smem + L::kK + sk * kTileBytes + c * kBlockBytes, &tm_k,
-                                         &bars->k_full[sk], c * 64, g, j * kBlockN, b);
-                }
-                __syncwarp();
+                ptx::mbar_arrive_expect_tx(&bars->k_full[sk], kTileBytes);
+                for (int c = 0; c < kDBlocks; ++c)
+                    ptx::tma_load_4d(smem + L::kK + sk * kTileBytes + c * kBlockBytes, &tm_k,
+                                     &bars->k_full[sk], c * 64, g, j * kBlockN, b);
                 ++issued_k;
                 const int sv = j % VST;
-                if (!warp_wait(&bars->v_empty[sv], ((j / VST) & 1) ^ 1, p.limit_ns, abort_flag)) {
+                if (!ptx::mbar_wait(&bars->v_empty[sv], ((j / VST) & 1) ^ 1, p.limit_ns,
+                                    abort_flag)) {
                     record_error(p.err, kErrFwdBase + 2, &bars->abort);
                     break;
                 }
-                if (lane == 0) {
-                    ptx::mbar_arrive_expect_tx(&bars->v_full[sv], kTileBytes);
-                    for (int c = 0; c < kDBlocks; ++c)
-                        ptx::tma_load_4d(smem + L::kV + sv * kTileBytes + c * kBlockBytes, &tm_v,
-                                         &bars->v_full[sv], c * 64, g, j * kBlockN, b);
-                }
-                __syncwarp();
+                ptx::mbar_arrive_expect_tx(&bars->v_full[sv], kTileBytes);
+                for (int c = 0; c < kDBlocks; ++c)
+                    ptx::tma_load_4d(smem + L::kV + sv * kTileBytes + c * kBlockBytes, &tm_v,
+                                     &bars->v_full[sv], c * 64, g, j * kBlockN, b);
                 ++issued_v;
             }
             // Never leave the CTA with a copy in flight: wait (bounded, and
@@ -283,160 +270,138 @@ __global__ void __launch_bounds__(kThreads, 1)
             // barrier that received a copy.
             int zero = 0;
             volatile int* no_abort = &zero;
-            ptx::mbar_wait(&bars->q_full, 0, p.limit_ns, no_abort);
+            for (int a = 0; a < 2; ++a)
+                if (issued_q[a]) ptx::mbar_wait(&bars->q_full[a], 0, p.limit_ns, no_abort);
             for (int j = max(0, issued_k - KST); j < issued_k; ++j)
                 ptx::mbar_wait(&bars->k_full[j % KST], (j / KST) & 1, p.limit_ns, no_abort);
             for (int j = max(0, issued_v - VST); j < issued_v; ++j)
                 ptx::mbar_wait(&bars->v_full[j % VST], (j / VST) & 1, p.limit_ns, no_abort);
         }
-    } else if (warp == kMmaWarp) {
+    } else if (warp == 9) {
         // ================================================= MMA issuer
-        if (nt > 0) {
+        if (lane == 0 && nt > 0) {
             bool ok = true;
+            bool q_ready[2] = {false, false};
+            const uint32_t col_s[2] = {0u, 128u};
+            const uint32_t col_o[2] = {256u, 256u + D};
+            const uint32_t q_addr[2] = {sbase + L::kQ, sbase + L::kQ + kTileBytes};
             auto wait_or_fail = [&](uint64_t* bar, uint32_t parity, unsigned site) {
-                if (!warp_wait(bar, parity, p.limit_ns, abort_flag)) {
+                if (!ptx::mbar_wait(bar, parity, p.limit_ns, abort_flag)) {
                     record_error(p.err, kErrFwdBase + site, &bars->abort);
                     ok = false;
                 }
                 return ok;
             };
-            // Descriptors are built once; each MMA adds a compile-time offset
-            // (in 16-byte units) to a base descriptor.
-            const uint64_t k_desc0 = ptx::sdesc_sw128(sbase + L::kK, 16, 1024);
-            const uint64_t v_desc0 = ptx::sdesc_sw128(sbase + L::kV, kBlockBytes, 1024);
-            constexpr uint64_t kTileUnits = kTileBytes >> 4;
-            auto issue_s = [&](int j) {
-                if (!wait_or_fail(&bars->k_full[j % KST], (j / KST) & 1, 4)) return;
-                ptx::tc_fence_after();
-                const uint64_t kd = k_desc0 + (uint64_t)(j % KST) * kTileUnits;
-                const uint32_t d_s = tmem + (uint32_t)((j & 1) * kBlockN);
+            auto issue_s = [&](int a, int j) {
+                if (!q_ready[a]) {
+                    if (!wait_or_fail(&bars->q_full[a], 0, 3)) return;
+                    ptx::tc_fence_after();
+                    q_ready[a] = true;
+                }
+                const uint32_t k_addr = sbase + L::kK + (j % KST) * kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    // A = Q from tensor memory (8 columns per 16 values);
-                    // B = K, K-major: +32 B per 16 values, +16 KB per block
-                    const uint64_t off = (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
-                    ptx::umma_ts_elect(d_s, tmem + kColQ + kk * 8, kd + off, kIdescS, kk > 0);
+                    const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
+                    ptx::umma_ss(tmem + col_s[a], ptx::sdesc_sw128(q_addr[a] + off, 16, 1024),
+                                 ptx::sdesc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0);
                 }
-                ptx::umma_commit_elect(&bars->s_full[j & 1]);
-                ptx::umma_commit_elect(&bars->k_empty[j % KST]);
-                __syncwarp();
+                ptx::umma_commit(&bars->s_full[a]);
             };
-            if (wait_or_fail(&bars->q_tmem, 0, 3)) {
+            auto issue_pv = [&](int a, int j) {
+                if (!wait_or_fail(&bars->p_full[a], j & 1, 5)) return;
+                if (!wait_or_fail(&bars->v_full[j % VST], (j / VST) & 1, 6)) return;
                 ptx::tc_fence_after();
-                issue_s(0);
-            }
-            for (int j = 0; ok && j < nt; ++j) {
-                if (j + 1 < nt) {
-                    issue_s(j + 1);
+                const uint32_t v_addr = sbase + L::kV + (j % VST) * kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                    ptx::umma_ts(tmem + col_o[a], tmem + col_s[a] + kk * 8,
+                                 ptx::sdesc_sw128(v_addr + kk * 16 * 128, kBlockBytes, 1024),
+                                 kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (j == (a == 0 ? nt0 : nt1) - 1) ptx::umma_commit(&bars->o_done[a]);
+            };
+            for (int j = 0; ok && j <= nt; ++j) {
+                if (j < nt) {
+                    if (!wait_or_fail(&bars->k_full[j % KST], (j / KST) & 1, 4)) break;
+                    ptx::tc_fence_after();
+                    if (j < nt0) issue_s(0, j);
                     if (!ok) break;
                 }
-                if (!wait_or_fail(&bars->p_full[j & 1], (j >> 1) & 1, 5)) break;
-                if (!wait_or_fail(&bars->v_full[j % VST], (j / VST) & 1, 6)) break;
-                ptx::tc_fence_after();
-                {
-                    const uint64_t vd = v_desc0 + (uint64_t)(j % VST) * kTileUnits;
-                    const uint32_t a_p = tmem + (uint32_t)((j & 1) * kBlockN);
-                    const uint32_t acc0 = j > 0 ? 1u : 0u;
-#pragma unroll
-                    for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                        // MN-major V: +16 keys = +2 KB per step
-                        ptx::umma_ts_elect(tmem + kColO, a_p + kk * 8,
-                                           vd + (uint64_t)((kk * 16 * 128) >> 4), kIdescO,
-                                           kk > 0 ? 1u : acc0);
-                    }
-                    ptx::umma_commit_elect(&bars->o_done);
-                    ptx::umma_commit_elect(&bars->v_empty[j % VST]);
+                if (j >= 1 && j - 1 < nt1) {
+                    issue_pv(1, j - 1);
+                    if (!ok) break;
+                    ptx::umma_commit(&bars->v_empty[(j - 1) % VST]);
                 }
-                __syncwarp();
+                if (j < nt) {
+                    if (j < nt1) issue_s(1, j);
+                    if (!ok) break;
+                    ptx::umma_commit(&bars->k_empty[j % KST]);
+                    if (j < nt0) {
+                        issue_pv(0, j);
+                        if (!ok) break;
+                        if (j >= nt1) ptx::umma_commit(&bars->v_empty[j % VST]);
+                    }
+                }
             }
             if (!ok) {
                 // make sure no MMA is still running before TMEM is freed
                 int zero = 0;
                 volatile int* no_abort = &zero;
-                ptx::umma_commit_elect(&bars->drain);
-                __syncwarp();
+                ptx::umma_commit(&bars->drain);
                 ptx::mbar_wait(&bars->drain, 0, p.limit_ns, no_abort);
             }
         }
     } else {
-        // ================================================= softmax warps
+        // ================================================= softmax warpgroups
+        const int a = warp >> 2;  // which Q tile
+        const int nta = a == 0 ? nt0 : nt1;
         const uint32_t quarter = (uint32_t)(warp & 3);
-        const int part = warp >> 2;  // which 32 score columns / D/4 output columns
         const uint32_t row = quarter * 32u + (uint32_t)lane;
         const uint32_t lane_addr = (quarter * 32u) << 16;
-        const int i = q0 + (int)row;
+        const int qa = qbase + a * kBlockM;
+        const int i = qa + (int)row;
         int row_lim = Lk - 1;  // last visible key of this row
         if (p.causal) row_lim = min(row_lim, i + Lk - p.Nq);
         const float sl2 = p.scale_log2;
         float m_ref = -INFINITY;  // running reference max, scale*log2 units
-        float l_part = 0.f;       // this warp's share of the running sum
+        float l_sum = 0.f;        // running sum of exp2(s*sl2 - m_ref)
         bool ok = true;
-        float* red_max = reinterpret_cast<float*>(smem + L::kRedMax);
-        float* red_sum = reinterpret_cast<float*>(smem + L::kRedSum);
-        const uint32_t row_bar = 1 + quarter;  // the four warps of these rows
-        const uint32_t t_o = tmem + lane_addr + kColO + (uint32_t)(part * kPartD);
+        const uint32_t t_s = tmem + lane_addr + (a == 0 ? 0u : 128u);
+        const uint32_t t_o = tmem + lane_addr + (a == 0 ? 256u : 256u + D);
 
-        // ---- Q -> tensor memory (A operand of S = Q Kᵀ): this warp copies
-        // d values [32 part, 32 part + 32) of its rows, two per column
-        if (nt > 0) {
-            if (!warp_wait(&bars->q_full, 0, p.limit_ns, abort_flag)) {
-                record_error(p.err, kErrFwdBase + 11, &bars->abort);
-                ok = false;
-            } else if (part * 32 < D) {
-                const int c0 = part * 32;  // first d value
-                const uint8_t* qrow = smem + L::kQ + (c0 >> 6) * kBlockBytes;
-                uint32_t qv[16];
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const uint4 v4 = *reinterpret_cast<const uint4*>(
-                        qrow + sw128_offset(row, (uint32_t)(((c0 & 63) >> 3) + q4)));
-                    qv[4 * q4] = v4.x;
-                    qv[4 * q4 + 1] = v4.y;
-                    qv[4 * q4 + 2] = v4.z;
-                    qv[4 * q4 + 3] = v4.w;
-                }
-                ptx::tmem_st16(tmem + lane_addr + kColQ + (uint32_t)(c0 >> 1), qv);
-                ptx::tmem_wait_st();
-            }
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (ok && lane == 0) ptx::mbar_arrive(&bars->q_tmem);
-        }
-
-        // Every warp walks all nt iterations and reaches every row barrier,
-        // also after a failed wait (then it only skips its work), so that its
-        // partners can never be left waiting at a barrier.
-        for (int j = 0; j < nt; ++j) {
-            const int sb = j & 1;
-            if (ok && !warp_wait(&bars->s_full[sb], (j >> 1) & 1, p.limit_ns, abort_flag)) {
+        for (int j = 0; j < nta; ++j) {
+            if (!warp_wait(&bars->s_full[a], j & 1, p.limit_ns, abort_flag)) {
                 record_error(p.err, kErrFwdBase + 7, &bars->abort);
                 ok = false;
+                break;
             }
-            const uint32_t t_s = tmem + lane_addr + (uint32_t)(sb * kBlockN);
-            const int key_base = j * kBlockN + part * 32;
-            const bool masked = key_base + 31 > row_lim;
-            uint32_t r[32];
-            float pmax = -INFINITY;
-            if (ok) {
-                ptx::tc_fence_after();
-                ptx::tmem_ld32(t_s + part * 32, r);
-                float mx8[8];
+            ptx::tc_fence_after();
+            const int key0 = j * kBlockN;
+            const bool masked = key0 + kBlockN - 1 > row_lim;
+            // pass 1: row maximum, two halves of 64 columns, eight independent
+            // chains of three-input maxima
+            float mx8[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
-                ptx::tmem_wait_ld_dep(r);
-                if (masked)
-                    part_max<true>(r, key_base, row_lim, mx8);
-                else
-                    part_max<false>(r, key_base, row_lim, mx8);
-                pmax = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]),
-                                 ptx::max3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+            for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
+            {
+                uint32_t r[2][2][32];
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    ptx::tmem_ld32(t_s + hf * 64, r[hf][0]);
+                    ptx::tmem_ld32(t_s + hf * 64 + 32, r[hf][1]);
+                }
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    ptx::tmem_wait_ld_dep(r[hf][0]);
+                    ptx::tmem_wait_ld_dep(r[hf][1]);
+                    if (masked)
+                        half_max<true>(r[hf], key0 + hf * 64, row_lim, mx8);
+                    else
+                        half_max<false>(r[hf], key0 + hf * 64, row_lim, mx8);
+                }
             }
-            // the row maximum over the four parts, through shared memory
-            red_max[((j & 1) * 4 + part) * 128 + row] = pmax;
-            ptx::named_barrier_sync(row_bar, 128);
-            if (!ok) continue;
-            const float* rm = red_max + (j & 1) * 4 * 128 + row;
-            const float mx = fmaxf(ptx::max3(rm[0], rm[128], rm[256]), rm[384]);
+            const float mx = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]),
+                                       ptx::max3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
             const float m_tile = mx * sl2;  // -inf stays -inf (sl2 > 0)
             float alpha = 1.f;
             bool rescale = false;
@@ -446,53 +411,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_ref = m_tile;
             }
             const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+            const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
+            const uint64_t nm_2 = ptx::f2_pack(-m_use, -m_use);
             uint64_t acc2[4] = {0, 0, 0, 0};  // four pair accumulators of the row sum
-            uint32_t pk[16];
-            if (masked)
-                part_exp<true, BF16>(r, key_base, row_lim, ptx::f2_pack(sl2, sl2),
-                                     ptx::f2_pack(-m_use, -m_use), acc2, pk);
-            else
-                part_exp<false, BF16>(r, key_base, row_lim, ptx::f2_pack(sl2, sl2),
-                                      ptx::f2_pack(-m_use, -m_use), acc2, pk);
-            // P of these 32 keys over columns [16 part, 16 part + 16) of S[sb]
-            ptx::tmem_st16(t_s + part * 16, pk);
+            // pass 2: exponentials per half; P of half hf goes to columns
+            // [32 hf, 32 hf + 32) of S_a, which pass 2 has already consumed
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t r[2][32];
+                ptx::tmem_ld32(t_s + hf * 64, r[0]);
+                ptx::tmem_ld32(t_s + hf * 64 + 32, r[1]);
+                ptx::tmem_wait_ld_dep(r[0]);
+                ptx::tmem_wait_ld_dep(r[1]);
+                uint32_t pk[32];
+                if (masked)
+                    half_exp<true, BF16>(r, key0 + hf * 64, row_lim, sl2_2, nm_2, acc2, pk);
+                else
+                    half_exp<false, BF16>(r, key0 + hf * 64, row_lim, sl2_2, nm_2, acc2, pk);
+                ptx::tmem_st32(t_s + hf * 32, pk);
+            }
             float s0, s1, s2, s3, s4, s5, s6, s7;
             ptx::f2_unpack(acc2[0], s0, s1);
             ptx::f2_unpack(acc2[1], s2, s3);
             ptx::f2_unpack(acc2[2], s4, s5);
             ptx::f2_unpack(acc2[3], s6, s7);
-            l_part = l_part * alpha + (((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7)));
+            const float rowsum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+            l_sum = l_sum * alpha + rowsum;
             if (__any_sync(0xffffffffu, rescale)) {
-                // O must hold P_{j-1} V_{j-1} before it is rescaled (all four
-                // warps of a row take the same decision).  S_j being done
-                // implies P_{j-2} V_{j-2} is, so phase j-1 is the current or
-                // the previous phase of o_done and a parity wait is exact.
-                if (!warp_wait(&bars->o_done, (j - 1) & 1, p.limit_ns, abort_flag)) {
-                    record_error(p.err, kErrFwdBase + 10, &bars->abort);
-                    ok = false;
-                    ptx::tmem_wait_st();
-                    continue;
-                }
-                ptx::tc_fence_after();
-                const float sc = rescale ? alpha : 1.f;
-                if constexpr (kPartD == 32) {
-                    uint32_t o[32];
-                    ptx::tmem_ld32(t_o, o);
-                    ptx::tmem_wait_ld_dep(o);
+                // the previous P_a V has completed (it precedes S_a_j); done
+                // after the exponentials so that the score registers are free
+                const float s = rescale ? alpha : 1.f;
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    ptx::tmem_ld32(t_o + c * 32, r);
+                    ptx::tmem_wait_ld_dep(r);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * sc);
-                    ptx::tmem_st32(t_o, o);
-                } else {
-                    uint32_t o[16];
-                    ptx::tmem_ld16(t_o, o);
-                    ptx::tmem_wait_ld_dep16(o);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * sc);
-                    ptx::tmem_st16(t_o, o);
+                    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * s);
+                    ptx::tmem_st32(t_o + c * 32, r);
                 }
+                ptx::tmem_wait_st();
             }
             ptx::tmem_wait_st();
-            const bool zero_v = p.seqlens_k != nullptr && j * kBlockN + kBlockN > Lk && part == 0;
+            const bool zero_v = p.seqlens_k != nullptr && key0 + kBlockN > Lk &&
+                                (a == 0 ? true : j >= nt0);
             if (zero_v) {
                 // keys behind the real length: zero their V rows so that a
                 // non-finite value stored there cannot reach O through 0 * NaN
@@ -500,9 +462,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!warp_wait(&bars->v_full[sv], (j / VST) & 1, p.limit_ns, abort_flag)) {
                     record_error(p.err, kErrFwdBase + 8, &bars->abort);
                     ok = false;
-                    continue;
+                    break;
                 }
-                if (j * kBlockN + (int)row >= Lk) {
+                if (key0 + (int)row >= Lk) {
                     uint8_t* vt = smem + L::kV + sv * kTileBytes;
 #pragma unroll
                     for (int c = 0; c < kDBlocks; ++c)
@@ -513,73 +475,57 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ptx::fence_proxy_async_smem();
             }
-            // each thread's P stores are complete (wait::st above); one
-            // arrival per warp after the warp has converged
             ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&bars->p_full[sb]);
+            ptx::mbar_arrive(&bars->p_full[a]);
         }
 
-        // ---- epilogue: O / l -> bf16/fp16 -> swizzled staging (the Q
-        // buffer, free once Q is in tensor memory and the last MMA is done)
-        // -> TMA store.  o_done completes once per P·V.  When the last tile's
-        // softmax ends, P_{nt-2}·V may still be pending (S_{nt-1} was issued
-        // before it), and a parity wait only tells the current phase from the
-        // one before it: wait for phase nt-2, then for phase nt-1.
-        if (ok && nt > 0) {
-            if ((nt >= 2 && !warp_wait(&bars->o_done, (nt - 2) & 1, p.limit_ns, abort_flag)) ||
-                !warp_wait(&bars->o_done, (nt - 1) & 1, p.limit_ns, abort_flag)) {
+        // ---- epilogue: O / l -> bf16/fp16 -> swizzled staging (the Q_a
+        // buffer, free once the last S_a MMA is done) -> TMA store
+        if (ok && nta > 0) {
+            if (!warp_wait(&bars->o_done[a], 0, p.limit_ns, abort_flag)) {
                 record_error(p.err, kErrFwdBase + 9, &bars->abort);
                 ok = false;
             }
             ptx::tc_fence_after();
         }
-        // the four parts' sums of the row
-        red_sum[part * 128 + row] = l_part;
-        ptx::named_barrier_sync(row_bar, 128);
-        const float l_sum = (red_sum[row] + red_sum[128 + row]) + (red_sum[256 + row] + red_sum[384 + row]);
-        const bool have = ok && nt > 0 && l_sum > 0.f;
+        const bool have = ok && nta > 0 && l_sum > 0.f;
         const float inv_l = have ? 1.f / l_sum : 0.f;
-        uint8_t* stage = smem + L::kQ;
-        if (q0 < p.Nq) {
-            uint32_t o[kPartD];
-            if (ok && nt > 0) {
-                if constexpr (kPartD == 32) {
-                    ptx::tmem_ld32(t_o, o);
-                    ptx::tmem_wait_ld_dep(o);
+        uint8_t* stage = smem + L::kQ + a * kTileBytes;
+        if (qa < p.Nq) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                if (ok && nta > 0) {
+                    ptx::tmem_ld32(t_o + c * 32, r);
+                    ptx::tmem_wait_ld_dep(r);
                 } else {
-                    ptx::tmem_ld16(t_o, o);
-                    ptx::tmem_wait_ld_dep16(o);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) r[e] = 0u;
                 }
-            } else {
+                uint32_t o2[16];
 #pragma unroll
-                for (int e = 0; e < kPartD; ++e) o[e] = 0u;
-            }
-            uint32_t o2[kPartD / 2];
+                for (int e = 0; e < 16; ++e)
+                    o2[e] = ptx::pack2<BF16>(__uint_as_float(r[2 * e]) * inv_l,
+                                             __uint_as_float(r[2 * e + 1]) * inv_l);
+                // 32 columns = 4 chunks of 16 bytes in block c/2, chunks (c%2)*4..+3
 #pragma unroll
-            for (int e = 0; e < kPartD / 2; ++e)
-                o2[e] = ptx::pack2<BF16>(__uint_as_float(o[2 * e]) * inv_l,
-                                         __uint_as_float(o[2 * e + 1]) * inv_l);
-            // output columns part * D/4 .. +D/4: 128-byte block col / 64,
-            // 16-byte chunks (col % 64) / 8 ..
-            const int col = part * kPartD;
-#pragma unroll
-            for (int q4 = 0; q4 < kPartD / 8; ++q4) {
-                const uint32_t ch = (uint32_t)(((col & 63) >> 3) + q4);
-                *reinterpret_cast<uint4*>(stage + (col >> 6) * kBlockBytes +
-                                          sw128_offset(row, ch)) =
-                    make_uint4(o2[q4 * 4], o2[q4 * 4 + 1], o2[q4 * 4 + 2], o2[q4 * 4 + 3]);
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const uint32_t ch = (uint32_t)((c & 1) * 4 + q4);
+                    *reinterpret_cast<uint4*>(stage + (c >> 1) * kBlockBytes +
+                                              sw128_offset(row, ch)) =
+                        make_uint4(o2[q4 * 4], o2[q4 * 4 + 1], o2[q4 * 4 + 2], o2[q4 * 4 + 3]);
+                }
             }
             ptx::fence_proxy_async_smem();
         }
-        ptx::named_barrier_sync(5, 32 * kSoftmaxWarps);
-        if (warp == 0 && lane == 0 && q0 < p.Nq) {
+        ptx::named_barrier_sync(1 + a, 128);
+        if (quarter == 0 && lane == 0 && qa < p.Nq) {
             for (int c = 0; c < kDBlocks; ++c)
-                ptx::tma_store_4d(&tm_o, stage + c * kBlockBytes, c * 64, h, q0, b);
+                ptx::tma_store_4d(&tm_o, stage + c * kBlockBytes, c * 64, h, qa, b);
             ptx::bulk_commit_group();
             ptx::bulk_wait_group_read0();
         }
-        if (part == 0 && i < p.Nq) {
+        if (i < p.Nq) {
             const float lse = have ? (m_ref + ptx::lg2_approx(l_sum)) * 0.69314718055994531f
                                    : -INFINITY;
             p.lse[((size_t)b * p.Hq + h) * p.Nq + i] = lse;
@@ -588,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == kMmaWarp) {
+    if (warp == 9) {
         __syncwarp();
         ptx::tc_fence_after();
         ptx::tmem_dealloc<kTmemCols>(tmem);
@@ -603,7 +549,7 @@ cudaError_t launch_fwd_t(const FwdMaps& maps, const FwdParams& p, cudaStream_t s
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.n_qtiles, p.Hq, p.B);
+    dim3 grid((p.Nq + 2 * kBlockM - 1) / (2 * kBlockM), p.Hq, p.B);
     kern<<<grid, kThreads, L::kAlloc, stream>>>(maps.q, maps.k, maps.v, maps.o, p);
     return cudaGetLastError();
 }
@@ -613,8 +559,8 @@ cudaError_t launch_fwd_t(const FwdMaps& maps, const FwdParams& p, cudaStream_t s
 cudaError_t launch_fwd(const FwdMaps& maps, const FwdParams& p, int d, bool bf16,
                        cudaStream_t stream) {
     if (d == 64) {
-        return bf16 ? launch_fwd_t<64, true, 4, 4>(maps, p, stream)
-                    : launch_fwd_t<64, false, 4, 4>(maps, p, stream);
+        return bf16 ? launch_fwd_t<64, true, 3, 4>(maps, p, stream)
+                    : launch_fwd_t<64, false, 3, 4>(maps, p, stream);
     }
     return bf16 ? launch_fwd_t<128, true, 2, 3>(maps, p, stream)
                 : launch_fwd_t<128, false, 2, 3>(maps, p, stream);
