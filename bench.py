@@ -443,7 +443,8 @@ def run_reference(args, rank, world):
 def run_profile_case(kernel: str, launches: int):
     """Small, self-contained launches for ncu captures: the forward of the
     bench workload (268 MB of inputs), or a decode of the Llama2-70B shape with
-    lengths up to 8192 (about 0.5 GB of cache); both larger than L2."""
+    lengths up to 8192 (about 0.5 GB of cache; one new token, or a causal
+    chunk of 16); all larger than L2."""
     from io_aware_exact_29_b200 import attn
     from io_aware_exact_29_b200.workloads import DecodeCase
 
@@ -454,7 +455,8 @@ def run_profile_case(kernel: str, launches: int):
         for _ in range(2 + launches):
             attn.attn_fwd(fin["q"], fin["k"], fin["v"], scale=fc.scale, causal=fc.causal)
     else:
-        dc = DecodeCase("profile", 32, 64, 8, 1, 128, (1, 8192), False)
+        nq = 16 if kernel == "decode_chunk16" else 1
+        dc = DecodeCase("profile", 32, 64, 8, nq, 128, (nq, 8192), nq > 1)
         din = kvcache_inputs(dc, seed=0, device="cuda")
         ml = int(din["seqlens_k"].max().item())
         ws = torch.empty(attn.decode_workspace_bytes(dc.B, dc.Hq, dc.Hkv, dc.Nq, dc.d, ml),
@@ -462,7 +464,7 @@ def run_profile_case(kernel: str, launches: int):
         for _ in range(2 + launches):
             attn.attn_fwd_varlen_kvcache(din["q"], din["k_cache"], din["v_cache"],
                                          din["cu_seqlens_k"], din["seqlens_k"], ml,
-                                         scale=dc.scale, workspace=ws)
+                                         scale=dc.scale, causal=dc.causal, workspace=ws)
         lens = din["seqlens_k"].tolist()
         print("decode profile case: sum_len", sum(lens), "algorithmic bytes per launch",
               accounting.decode_bytes(lens, dc.B, dc.Hq, dc.Hkv, dc.Nq, dc.d))
@@ -540,7 +542,7 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=32)
-    ap.add_argument("--profile", choices=["fwd", "decode"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "decode", "decode_chunk16"], default=None,
                     help="run a small case of one kernel for an ncu capture and exit")
     ap.add_argument("--profile-launches", type=int, default=3)
     ap.add_argument("--sweep", action="store_true",

@@ -227,13 +227,26 @@ int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_ca
         (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return ATTN_ERR_WORKSPACE;
 
-    CUtensorMap kmap, vmap;
+    const int G = Hq / Hkv;
+    CUtensorMap kmap, vmap, qmap, omap;
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)Hkv, (uint64_t)cache_slots};
     const uint64_t strides[2] = {(uint64_t)d * 2, (uint64_t)Hkv * d * 2};
-    const uint32_t box[3] = {64, 1, 64};
+    const uint32_t box[3] = {64, 1, lay.tc ? 128u : 64u};
     if (!encode_map(&kmap, dtype, k_cache, 3, dims, strides, box) ||
         !encode_map(&vmap, dtype, v_cache, 3, dims, strides, box))
         return ATTN_ERR_INVALID_ARG;
+    if (lay.tc) {
+        // Q and O [B, Nq, Hq, d] seen as {d, G, Hkv, Nq, B}: one box gathers
+        // the 128 / G tokens x G heads that share kv head g (row t * G + hh)
+        const uint64_t qdims[5] = {(uint64_t)d, (uint64_t)G, (uint64_t)Hkv, (uint64_t)Nq,
+                                   (uint64_t)B};
+        const uint64_t qstrides[4] = {(uint64_t)d * 2, (uint64_t)G * d * 2, (uint64_t)Hq * d * 2,
+                                      (uint64_t)Nq * Hq * d * 2};
+        const uint32_t qbox[5] = {64, (uint32_t)G, 1, (uint32_t)(128 / G), 1};
+        if (!encode_map(&qmap, dtype, q, 5, qdims, qstrides, qbox) ||
+            !encode_map(&omap, dtype, o, 5, qdims, qstrides, qbox))
+            return ATTN_ERR_INVALID_ARG;
+    }
 
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     DecodeParams p{};
@@ -249,7 +262,7 @@ int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_ca
     p.Hq = Hq;
     p.Hkv = Hkv;
     p.Nq = Nq;
-    p.G = Hq / Hkv;
+    p.G = G;
     p.rows = Nq * p.G;
     p.n_mgroups = lay.n_mgroups;
     p.split_keys = lay.split_keys;
@@ -262,7 +275,8 @@ int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_ca
     if (cudaMemsetAsync(p.counters, 0, (size_t)B * Hkv * lay.n_mgroups * sizeof(unsigned), s) !=
         cudaSuccess)
         return ATTN_ERR_CUDA;
-    cudaError_t e = launch_decode(kmap, vmap, p, d, dtype == ATTN_BF16, s);
+    cudaError_t e = lay.tc ? launch_decode_tc(qmap, kmap, vmap, omap, p, d, dtype == ATTN_BF16, s)
+                           : launch_decode(kmap, vmap, p, d, dtype == ATTN_BF16, s);
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

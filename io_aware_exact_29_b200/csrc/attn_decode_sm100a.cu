@@ -458,22 +458,31 @@ DecodeLayout decode_layout(int B, int Hq, int Hkv, int Nq, int d, int max_seqlen
     DecodeLayout l{};
     const int G = Hq / Hkv;
     const int rows = Nq * G;
-    l.n_mgroups = (rows + 15) / 16;
+    l.tc = decode_use_tc(G, Nq, split_keys) ? 1 : 0;
+    l.n_mgroups = l.tc ? 1 : (rows + 15) / 16;
+    const int unit_rows = l.tc ? 128 : 16;
     int split = split_keys;
-    if (split <= 0) {
+    const long units = (long)B * Hkv * l.n_mgroups;
+    auto n_work = [&](int s) { return units * ((max_seqlen_k + s - 1) / s); };
+    if (split <= 0 && l.tc) {
+        // one CTA per SM: long splits (each CTA pays a pipeline fill and a
+        // partial-result write), but about four CTAs per SM over the longest
+        // sequence, in splits of at least 512 keys
+        split = 16384;
+        while (split > 512 && n_work(split) < 148L * 4) split /= 2;
+    } else if (split <= 0) {
         // enough work units to fill the GPU several times over, but splits of
         // at least 256 keys so that each unit amortises its set-up
-        const long units = (long)B * Hkv * l.n_mgroups;
         split = 1024;
-        while (split > 256 && units * ((max_seqlen_k + split - 1) / split) < 148L * 2 * 8) split /= 2;
+        while (split > 256 && n_work(split) < 148L * 2 * 8) split /= 2;
     }
     l.split_keys = split;
     l.max_splits = max_seqlen_k > 0 ? (max_seqlen_k + split - 1) / split : 1;
-    const size_t n_units = (size_t)B * Hkv * l.n_mgroups;
+    const size_t n_units = (size_t)units;
     auto align = [](size_t x) { return (x + 255) & ~(size_t)255; };
     l.part_o_off = 0;
-    l.part_lse_off = align(n_units * l.max_splits * 16 * (size_t)d * 4);
-    l.counters_off = l.part_lse_off + align(n_units * l.max_splits * 16 * 4);
+    l.part_lse_off = align(n_units * l.max_splits * unit_rows * (size_t)d * 4);
+    l.counters_off = l.part_lse_off + align(n_units * l.max_splits * unit_rows * 4);
     l.total = l.counters_off + align(n_units * 4);
     return l;
 }

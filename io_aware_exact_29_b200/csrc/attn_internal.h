@@ -41,8 +41,8 @@ struct DecodeParams {
     float* lse;            // [B, Hq, Nq]
     const int* cu_seqlens_k;
     const int* seqlens_k;
-    float* part_o;         // [B, Hkv, n_mgroups, max_splits, 16, d] fp32
-    float* part_lse;       // [B, Hkv, n_mgroups, max_splits, 16]
+    float* part_o;         // [B, Hkv, n_mgroups, max_splits, R, d] fp32 (R = 16, or 128 for tc)
+    float* part_lse;       // [B, Hkv, n_mgroups, max_splits, R]
     unsigned* counters;    // [B, Hkv, n_mgroups]
     int B, Hq, Hkv, Nq, G;
     int rows;              // Nq * G query rows per (sequence, kv head)
@@ -56,15 +56,29 @@ struct DecodeParams {
 };
 
 struct DecodeLayout {
+    int tc;  // 1: tensor-core kernel (one 128-row tile per unit), 0: mma.sync kernel
     int split_keys, max_splits, n_mgroups;
     size_t part_o_off, part_lse_off, counters_off, total;
 };
+
+// The tensor-core decode takes the shapes whose Nq * G query rows per kv
+// head fill 64..128 rows of one tile, with whole 128-key tiles per split.
+inline bool decode_use_tc(int G, int Nq, int split_keys) {
+    const int rows = Nq * G;
+    return G <= 128 && 128 % G == 0 && rows >= 64 && rows <= 128 && split_keys % 128 == 0;
+}
 
 DecodeLayout decode_layout(int B, int Hq, int Hkv, int Nq, int d, int max_seqlen_k,
                            int split_keys);
 
 cudaError_t launch_decode(const CUtensorMap& kmap, const CUtensorMap& vmap,
                           const DecodeParams& p, int d, bool bf16, cudaStream_t stream);
+
+// Tensor-core decode: qmap/omap are the 5-D maps {d, G, Hkv, Nq, B} with box
+// {64, G, 1, 128 / G, 1}; kmap/vmap the packed-cache maps with 128-row boxes.
+cudaError_t launch_decode_tc(const CUtensorMap& qmap, const CUtensorMap& kmap,
+                             const CUtensorMap& vmap, const CUtensorMap& omap,
+                             const DecodeParams& p, int d, bool bf16, cudaStream_t stream);
 
 // Address of the device error word on the current device.
 unsigned* device_error_word();

@@ -82,6 +82,52 @@ def test_chunk_causal_bottom_right(nq):
         assert torch.all(torch.isneginf(lse[4, :, : nq - 3]))
 
 
+# Shapes whose Nq * G query rows per kv head fill 64..128 rows run on the
+# tensor-core decode kernel (one 128-row tile per CTA, 128-key tiles); the
+# rest, and split sizes that are not a multiple of 128, on the mma.sync one.
+TC_LENS = [0, 1, 15, 16, 17, 127, 128, 129, 511, 512, 513, 2047, 2048, 2049, 5000]
+
+
+@pytest.mark.parametrize("hq,hkv,nq", [(16, 2, 16), (16, 2, 8), (32, 2, 8), (8, 2, 16),
+                                       (64, 2, 4), (128, 1, 1)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_tensor_core_chunk_shapes(hq, hkv, nq, causal):
+    c = DecodeCase("tc", len(TC_LENS), hq, hkv, nq, 128, (0, 5000), causal, slack=5)
+    inp = kvcache_inputs(c, seed=20 + nq, seqlens=TC_LENS)
+    _check(inp, c, split_keys=0, what=f"tc {hq}/{hkv} nq {nq} causal {causal}")
+
+
+@pytest.mark.parametrize("split", [128, 384, 1024, 8192])
+def test_tensor_core_split_sizes(split):
+    c = DecodeCase("tcs", len(TC_LENS), 16, 2, 16, 128, (0, 5000), True, slack=3)
+    inp = kvcache_inputs(c, seed=31, seqlens=TC_LENS)
+    _check(inp, c, split_keys=split, what=f"tc split {split}")
+
+
+@pytest.mark.parametrize("d,dtype", [(64, "bf16"), (64, "fp16"), (128, "fp16")])
+def test_tensor_core_head_dims_and_fp16(d, dtype):
+    c = DecodeCase("tch", 7, 32, 4, 16, d, (1, 3000), True, dtype=dtype)
+    _check(kvcache_inputs(c, seed=32), c, split_keys=512, what=f"tc d{d} {dtype}")
+
+
+def test_tensor_core_unfilled_slots_hold_nan():
+    c = DecodeCase("tcn", 6, 16, 2, 16, 128, (1, 700), True, slack=40)
+    clean = kvcache_inputs(c, seed=33)
+    dirty = kvcache_inputs(c, seed=33, slack_fill=float("nan"))
+    (_, o1, l1) = _check(clean, c, split_keys=256, what="tc clean")
+    (_, o2, l2) = _check(dirty, c, split_keys=256, what="tc NaN in unfilled slots")
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_tensor_core_and_mma_sync_paths_agree():
+    c = DecodeCase("tca", 5, 16, 2, 16, 128, (1, 4000), True)
+    inp = kvcache_inputs(c, seed=34)
+    (_, o1, l1) = _check(inp, c, split_keys=64, what="mma.sync path")   # 64: not a 128 multiple
+    (_, o2, l2) = _check(inp, c, split_keys=1024, what="tensor-core path")
+    assert (o1.float() - o2.float()).abs().max().item() <= 1.6e-2
+    assert (l1 - l2).abs().max().item() <= 1e-4
+
+
 @pytest.mark.parametrize("name", ["llama70b_decode", "llama70b_chunk16"])
 def test_llama70b_shape_sampled_sequences(name):
     # full-size launch (B=32, Hq=64, Hkv=8, d=128, lengths up to 32768);
