@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -34,6 +35,7 @@ std::mutex g_mu;
 EncodeTiledFn g_encode = nullptr;
 int g_dev_state[kMaxDevices] = {0};  // 0 unknown, 1 supported, -1 unsupported
 unsigned* g_err_addr[kMaxDevices] = {nullptr};
+int g_sm_count[kMaxDevices] = {0};
 
 EncodeTiledFn encode_fn() {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -68,6 +70,12 @@ int check_device(int* dev_out) {
                 return 0;
             }
             g_err_addr[dev] = static_cast<unsigned*>(addr);
+            if (cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev) !=
+                    cudaSuccess ||
+                g_sm_count[dev] <= 0) {
+                g_dev_state[dev] = 0;
+                return 0;
+            }
         }
     }
     return g_dev_state[dev];
@@ -228,7 +236,7 @@ int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_ca
         return ATTN_ERR_WORKSPACE;
 
     const int G = Hq / Hkv;
-    CUtensorMap kmap, vmap, qmap, omap;
+    CUtensorMap kmap, vmap, qmap;
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)Hkv, (uint64_t)cache_slots};
     const uint64_t strides[2] = {(uint64_t)d * 2, (uint64_t)Hkv * d * 2};
     const uint32_t box[3] = {64, 1, lay.tc ? 128u : 64u};
@@ -243,9 +251,7 @@ int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_ca
         const uint64_t qstrides[4] = {(uint64_t)d * 2, (uint64_t)G * d * 2, (uint64_t)Hq * d * 2,
                                       (uint64_t)Nq * Hq * d * 2};
         const uint32_t qbox[5] = {64, (uint32_t)G, 1, (uint32_t)(128 / G), 1};
-        if (!encode_map(&qmap, dtype, q, 5, qdims, qstrides, qbox) ||
-            !encode_map(&omap, dtype, o, 5, qdims, qstrides, qbox))
-            return ATTN_ERR_INVALID_ARG;
+        if (!encode_map(&qmap, dtype, q, 5, qdims, qstrides, qbox)) return ATTN_ERR_INVALID_ARG;
     }
 
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -258,6 +264,8 @@ int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_ca
     p.part_o = reinterpret_cast<float*>(ws + lay.part_o_off);
     p.part_lse = reinterpret_cast<float*>(ws + lay.part_lse_off);
     p.counters = reinterpret_cast<unsigned*>(ws + lay.counters_off);
+    p.items = reinterpret_cast<int4*>(ws + lay.items_off);
+    p.work_meta = reinterpret_cast<int*>(ws + lay.meta_off);
     p.B = B;
     p.Hq = Hq;
     p.Hkv = Hkv;
@@ -272,11 +280,18 @@ int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_ca
     p.limit_ns = kDefaultLimitNs;
     p.err = g_err_addr[dev];
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(p.counters, 0, (size_t)B * Hkv * lay.n_mgroups * sizeof(unsigned), s) !=
-        cudaSuccess)
-        return ATTN_ERR_CUDA;
-    cudaError_t e = lay.tc ? launch_decode_tc(qmap, kmap, vmap, omap, p, d, dtype == ATTN_BF16, s)
-                           : launch_decode(kmap, vmap, p, d, dtype == ATTN_BF16, s);
+    cudaError_t e;
+    if (lay.tc) {
+        // the plan kernel clears the counters; one persistent CTA per SM
+        const long items_max = (long)B * Hkv * lay.max_splits;
+        const int n_ctas = (int)std::min<long>(g_sm_count[dev], items_max);
+        e = launch_decode_tc(qmap, kmap, vmap, p, d, dtype == ATTN_BF16, n_ctas, s);
+    } else {
+        if (cudaMemsetAsync(p.counters, 0, (size_t)B * Hkv * lay.n_mgroups * sizeof(unsigned),
+                            s) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        e = launch_decode(kmap, vmap, p, d, dtype == ATTN_BF16, s);
+    }
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

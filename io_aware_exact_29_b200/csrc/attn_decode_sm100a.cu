@@ -483,7 +483,9 @@ DecodeLayout decode_layout(int B, int Hq, int Hkv, int Nq, int d, int max_seqlen
     l.part_o_off = 0;
     l.part_lse_off = align(n_units * l.max_splits * unit_rows * (size_t)d * 4);
     l.counters_off = l.part_lse_off + align(n_units * l.max_splits * unit_rows * 4);
-    l.total = l.counters_off + align(n_units * 4);
+    l.items_off = l.counters_off + align(n_units * 4);
+    l.meta_off = l.items_off + (l.tc ? align(n_units * l.max_splits * 16) : 0);
+    l.total = l.meta_off + (l.tc ? 256 : 0);
     return l;
 }
 

@@ -44,6 +44,8 @@ struct DecodeParams {
     float* part_o;         // [B, Hkv, n_mgroups, max_splits, R, d] fp32 (R = 16, or 128 for tc)
     float* part_lse;       // [B, Hkv, n_mgroups, max_splits, R]
     unsigned* counters;    // [B, Hkv, n_mgroups]
+    int4* items;           // tc: work list {b, g, split, nsplit}, longest first
+    int* work_meta;        // tc: [0] number of items, [1] next item to take
     int B, Hq, Hkv, Nq, G;
     int rows;              // Nq * G query rows per (sequence, kv head)
     int n_mgroups;         // ceil(rows / 16)
@@ -58,7 +60,7 @@ struct DecodeParams {
 struct DecodeLayout {
     int tc;  // 1: tensor-core kernel (one 128-row tile per unit), 0: mma.sync kernel
     int split_keys, max_splits, n_mgroups;
-    size_t part_o_off, part_lse_off, counters_off, total;
+    size_t part_o_off, part_lse_off, counters_off, items_off, meta_off, total;
 };
 
 // The tensor-core decode takes the shapes whose Nq * G query rows per kv
@@ -74,11 +76,12 @@ DecodeLayout decode_layout(int B, int Hq, int Hkv, int Nq, int d, int max_seqlen
 cudaError_t launch_decode(const CUtensorMap& kmap, const CUtensorMap& vmap,
                           const DecodeParams& p, int d, bool bf16, cudaStream_t stream);
 
-// Tensor-core decode: qmap/omap are the 5-D maps {d, G, Hkv, Nq, B} with box
+// Tensor-core decode (a plan kernel, then a persistent kernel of n_ctas
+// CTAs): qmap is the 5-D map {d, G, Hkv, Nq, B} of Q with box
 // {64, G, 1, 128 / G, 1}; kmap/vmap the packed-cache maps with 128-row boxes.
 cudaError_t launch_decode_tc(const CUtensorMap& qmap, const CUtensorMap& kmap,
-                             const CUtensorMap& vmap, const CUtensorMap& omap,
-                             const DecodeParams& p, int d, bool bf16, cudaStream_t stream);
+                             const CUtensorMap& vmap, const DecodeParams& p, int d, bool bf16,
+                             int n_ctas, cudaStream_t stream);
 
 // Address of the device error word on the current device.
 unsigned* device_error_word();

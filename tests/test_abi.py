@@ -101,11 +101,13 @@ def test_decode_workspace_accounting():
 def test_decode_workspace_accounting_tensor_core_layout():
     # 16 new tokens x 8 query heads per kv head = 128 rows: one 128-row tile
     # per (sequence, kv head); automatic split 8192 keys (256 units x 4
-    # splits >= 148 x 4 work items), 128 rows x (128 + 1) floats per split
+    # splits >= 148 x 4 work items), 128 rows x (128 + 1) floats per split,
+    # a counter per unit, the 16-byte work-list entries and the list's header
     n = attn.decode_workspace_bytes(32, 64, 8, 16, 128, 32768)
     units, splits = 32 * 8, 4
-    expect = units * splits * 128 * 128 * 4 + units * splits * 128 * 4 + units * 4
-    assert expect <= n <= expect + 3 * 256
+    expect = (units * splits * 128 * 128 * 4 + units * splits * 128 * 4 + units * 4
+              + units * splits * 16 + 8)
+    assert expect <= n <= expect + 4 * 256
     # a split that is not a multiple of 128 keeps the 16-row layout
     n64 = attn.decode_workspace_bytes(32, 64, 8, 16, 128, 32768, split_keys=64)
     expect64 = 32 * 8 * 8 * 512 * 16 * 128 * 4 + 32 * 8 * 8 * 512 * 16 * 4 + 32 * 8 * 8 * 4

@@ -157,3 +157,15 @@ def test_max_seqlen_too_small_is_reported():
                                  dev["seqlens_k"], 1000, scale=c.scale, split_keys=256)
     torch.cuda.synchronize()
     assert attn.get_device_error() == attn.ERR_DECODE_BASE + 1
+
+
+def test_tensor_core_max_seqlen_too_small_is_reported():
+    c = DecodeCase("tce", 2, 16, 2, 16, 128, (16, 3000), True)
+    inp = kvcache_inputs(c, seed=35, seqlens=[3000, 20])
+    attn.get_device_error()
+    dev = {k: v.cuda() for k, v in inp.items()}
+    attn.attn_fwd_varlen_kvcache(dev["q"], dev["k_cache"], dev["v_cache"], dev["cu_seqlens_k"],
+                                 dev["seqlens_k"], 1000, scale=c.scale, causal=True,
+                                 split_keys=256)
+    torch.cuda.synchronize()
+    assert attn.get_device_error() == attn.ERR_DECODE_BASE + 1
