@@ -264,8 +264,11 @@ int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_ca
     p.part_o = reinterpret_cast<float*>(ws + lay.part_o_off);
     p.part_lse = reinterpret_cast<float*>(ws + lay.part_lse_off);
     p.counters = reinterpret_cast<unsigned*>(ws + lay.counters_off);
-    p.items = reinterpret_cast<int4*>(ws + lay.items_off);
-    p.work_meta = reinterpret_cast<int*>(ws + lay.meta_off);
+    p.plan = reinterpret_cast<DecodePlan*>(ws + lay.plan_off);
+    p.seq_prefix = reinterpret_cast<long long*>(ws + lay.prefix_off);
+    p.range_units = reinterpret_cast<int2*>(ws + lay.ranges_off);
+    p.max_seqlen_k = max_seqlen_k;
+    p.max_ranges = lay.max_ranges;
     p.B = B;
     p.Hq = Hq;
     p.Hkv = Hkv;
@@ -283,8 +286,7 @@ int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_ca
     cudaError_t e;
     if (lay.tc) {
         // the plan kernel clears the counters; one persistent CTA per SM
-        const long items_max = (long)B * Hkv * lay.max_splits;
-        const int n_ctas = (int)std::min<long>(g_sm_count[dev], items_max);
+        const int n_ctas = std::min(g_sm_count[dev], lay.max_ranges);
         e = launch_decode_tc(qmap, kmap, vmap, p, d, dtype == ATTN_BF16, n_ctas, s);
     } else {
         if (cudaMemsetAsync(p.counters, 0, (size_t)B * Hkv * lay.n_mgroups * sizeof(unsigned),

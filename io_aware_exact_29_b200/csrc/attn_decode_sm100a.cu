@@ -23,6 +23,8 @@
 // partial O and LSE to the workspace and the last CTA of the (b, g, row
 // group) -- found with an atomic counter, no spinning -- merges all splits in
 // split order:  LSE = log sum_s exp(LSE_s),  O = sum_s exp(LSE_s - LSE) O_s.
+#include <algorithm>
+
 #include "attn_internal.h"
 #include "ptx.cuh"
 
@@ -458,34 +460,49 @@ DecodeLayout decode_layout(int B, int Hq, int Hkv, int Nq, int d, int max_seqlen
     DecodeLayout l{};
     const int G = Hq / Hkv;
     const int rows = Nq * G;
+    auto align = [](size_t x) { return (x + 255) & ~(size_t)255; };
     l.tc = decode_use_tc(G, Nq, split_keys) ? 1 : 0;
-    l.n_mgroups = l.tc ? 1 : (rows + 15) / 16;
-    const int unit_rows = l.tc ? 128 : 16;
+    if (l.tc) {
+        // stream-K ranges: at most kDecodeMaxRangesAuto in automatic mode,
+        // else ranges of split_keys / 128 tiles of weight
+        const long units = (long)B * Hkv;
+        const long w_max = units * ((max_seqlen_k + 127) / 128 + kDecodeSegCost);
+        long ranges;
+        if (split_keys <= 0)
+            ranges = std::min<long>(kDecodeMaxRangesAuto,
+                                    (w_max + kDecodeMinRangeWeight - 1) / kDecodeMinRangeWeight);
+        else
+            ranges = (w_max + split_keys / 128 - 1) / (split_keys / 128);
+        l.max_ranges = (int)std::min<long>(ranges, 1L << 24);
+        l.split_keys = split_keys;
+        l.max_splits = 1;
+        l.n_mgroups = 1;
+        const size_t slots = 2 * (size_t)l.max_ranges;
+        l.part_o_off = 0;
+        l.part_lse_off = align(slots * 128 * (size_t)d * 4);
+        l.counters_off = l.prefix_off = l.part_lse_off + align(slots * 128 * 4);
+        l.ranges_off = l.prefix_off + align(((size_t)B + 1) * 8);
+        l.plan_off = l.ranges_off + align((size_t)l.max_ranges * 8);
+        l.total = l.plan_off + align(sizeof(DecodePlan));
+        return l;
+    }
+    l.n_mgroups = (rows + 15) / 16;
     int split = split_keys;
     const long units = (long)B * Hkv * l.n_mgroups;
-    auto n_work = [&](int s) { return units * ((max_seqlen_k + s - 1) / s); };
-    if (split <= 0 && l.tc) {
-        // one CTA per SM: long splits (each CTA pays a pipeline fill and a
-        // partial-result write), but about four CTAs per SM over the longest
-        // sequence, in splits of at least 512 keys
-        split = 16384;
-        while (split > 512 && n_work(split) < 148L * 4) split /= 2;
-    } else if (split <= 0) {
+    if (split <= 0) {
         // enough work units to fill the GPU several times over, but splits of
         // at least 256 keys so that each unit amortises its set-up
         split = 1024;
-        while (split > 256 && n_work(split) < 148L * 2 * 8) split /= 2;
+        while (split > 256 && units * ((max_seqlen_k + split - 1) / split) < 148L * 2 * 8) split /= 2;
     }
     l.split_keys = split;
     l.max_splits = max_seqlen_k > 0 ? (max_seqlen_k + split - 1) / split : 1;
     const size_t n_units = (size_t)units;
-    auto align = [](size_t x) { return (x + 255) & ~(size_t)255; };
     l.part_o_off = 0;
-    l.part_lse_off = align(n_units * l.max_splits * unit_rows * (size_t)d * 4);
-    l.counters_off = l.part_lse_off + align(n_units * l.max_splits * unit_rows * 4);
-    l.items_off = l.counters_off + align(n_units * 4);
-    l.meta_off = l.items_off + (l.tc ? align(n_units * l.max_splits * 16) : 0);
-    l.total = l.meta_off + (l.tc ? 256 : 0);
+    l.part_lse_off = align(n_units * l.max_splits * 16 * (size_t)d * 4);
+    l.counters_off = l.part_lse_off + align(n_units * l.max_splits * 16 * 4);
+    l.prefix_off = l.ranges_off = l.plan_off = l.counters_off + align(n_units * 4);
+    l.total = l.plan_off;
     return l;
 }
 

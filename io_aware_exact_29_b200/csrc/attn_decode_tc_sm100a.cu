@@ -11,14 +11,17 @@
 // split the keys are processed tile by tile with a running max and sum
 // (section "FlashAttention 拆的不是算法，是数据流").
 //
-// Scheduling.  A work item is (sequence b, kv head g, key split s).  A
-// one-CTA plan kernel lists the items longest first (all full splits, then
-// the last, shorter split of each sequence in decreasing length) and clears
-// the counters; the decode kernel is persistent -- one CTA per SM -- and
-// its loader warp takes items from the list with an atomic counter, so
-// short items fill the end of the run and each CTA pays its set-up once.
-// The loader moves on to the next item's Q and K/V tiles while the current
-// one finishes, so the memory pipe stays busy across item boundaries.
+// Scheduling (stream-K style).  Unit (b, g) -- sequence b, kv head g --
+// weighs its 128-key tiles plus a fixed set-up weight; the units are laid
+// end to end and the total weight is cut into equal ranges, one per CTA of
+// a persistent grid (one CTA per SM).  A CTA walks its range unit by unit;
+// a unit is split only where a range boundary falls inside it, so every CTA
+// gets the same work whatever the length mix, and only the (at most two)
+// units at the ends of a range need a merge.  A one-CTA plan kernel computes
+// the weight prefix over sequences and each range's first and last unit.
+// The loader warp moves on to the next unit's Q and K/V tiles while the
+// current one finishes, so the memory pipe stays busy across unit
+// boundaries.
 //
 // Query row r = t * G + hh is token t, query head g * G + hh; a 5-D TMA box
 // gathers the 128 rows (tokens past Nq read as zeros).
@@ -32,11 +35,15 @@
 // (bf16/fp16) overwrites the first 64 columns of its S buffer and is the A
 // operand of P·V.
 //
-// With one split an item's O and LSE go straight to the output; otherwise
-// the item writes its normalised partial O (fp32) and LSE to the workspace
-// and the CTA that finishes the last split of a (sequence, kv head) -- found
-// with an atomic counter, no spinning -- merges all splits in split order:
-// LSE = log sum_s exp(LSE_s), O = sum_s exp(LSE_s - LSE) O_s.
+// A unit done in one piece writes O and LSE straight to the output; a
+// split unit writes each piece's normalised partial O (fp32) and LSE to the
+// slot its range owns (range r: slot 2r for a unit continuing from range
+// r-1, slot 2r+1 for a unit continuing into range r+1), and a small merge
+// kernel that runs after the decode combines the pieces in key order:
+// LSE = log sum_s exp(LSE_s), O = sum_s exp(LSE_s - LSE) O_s.  (Merging in
+// the decode kernel, by whichever CTA finishes a unit's last piece, put a
+// fence, an atomic and dependent cache misses under full memory load at the
+// end of the run.)
 //
 // Every wait is a bounded mbarrier wait (named barriers cannot time out, and
 // a persistent loop must be able to leave on an error at any point).
@@ -55,7 +62,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.69314718055994531f;
 constexpr int kPlanThreads = 1024;
-constexpr int kPlanBuckets = 256;
 
 template <int D, int KST, int VST>
 struct TcSmem {
@@ -64,15 +70,15 @@ struct TcSmem {
     static constexpr uint32_t kK = kQ + kTileBytes;
     static constexpr uint32_t kV = kK + KST * kTileBytes;
     static constexpr uint32_t kRed = kV + VST * kTileBytes;    // [2 slots][4 parts][128] fp32
-    static constexpr uint32_t kRowLse = kRed + 2 * 4 * 128 * 4;  // [128] fp32
-    static constexpr uint32_t kBars = kRowLse + 128 * 4;
+    static constexpr uint32_t kBars = kRed + 2 * 4 * 128 * 4;
     static constexpr uint32_t kTotal = kBars + 1024;
     static constexpr uint32_t kAlloc = kTotal + 1024;
 };
 
-// One pushed work item: b < 0 ends the work.
+// One pushed piece of work: keys [key_begin, key_end) of unit (b, g), piece
+// seg of nseg, inside range `range`; b < 0 ends the work.
 struct TcItem {
-    int b, g, split, nsplit, Lk, slot0, pad0, pad1;
+    int b, g, key_begin, key_end, nseg, seg, range, Lk, slot0, pad0, pad1, pad2;
 };
 
 template <int KST, int VST>
@@ -90,11 +96,9 @@ struct TcBars {
     uint64_t o_final;  // one phase per item: every MMA of the item is complete
     uint64_t o_free;   // one phase per item: the softmax warps have read O
     uint64_t row_sync[4];
-    uint64_t ep_sync;
     uint64_t drain;
     TcItem item[kItemRing];
     uint32_t tmem_base;
-    int is_last;
     int abort;
 };
 
@@ -185,54 +189,164 @@ __device__ __forceinline__ void store_row_part(void* o, size_t elem, const float
 }
 
 // ------------------------------------------------------------------ plan
-// One CTA: lists the work items longest first and clears the counters.
-// Items of a bucket (same number of key tiles, capped at 255) keep the
-// order the atomics give; results do not depend on it, because every
-// partial lands in its own (unit, split) slot and the merge sums in split
-// order.
+// Key length of sequence b as the schedule sees it; a length outside
+// [0, max_seqlen_k] is reported (by the plan) and treated as empty.
+__device__ __forceinline__ int checked_len(const DecodeParams& p, int b) {
+    const int L = p.seqlens_k[b];
+    return (L < 0 || L > p.max_seqlen_k) ? 0 : L;
+}
+
+// One CTA: the exclusive prefix of sequence weights Hkv * (tiles_b + set-up),
+// the ranges, and each range's first and last unit (binary search over the
+// prefix).
 __global__ void __launch_bounds__(kPlanThreads)
-    attn_decode_plan_kernel(const __grid_constant__ DecodeParams p) {
-    __shared__ int hist[kPlanBuckets];
-    __shared__ int offs[kPlanBuckets];
+    attn_decode_plan_kernel(const __grid_constant__ DecodeParams p, int n_ctas) {
+    __shared__ long long warp_incl[kPlanThreads / 32];
+    __shared__ long long carry;
     const int tid = threadIdx.x;
-    for (int k = tid; k < kPlanBuckets; k += kPlanThreads) hist[k] = 0;
-    const int units = p.B * p.Hkv;
-    for (int u = tid; u < units; u += kPlanThreads) p.counters[u] = 0u;
+    const int lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) carry = 0;
     __syncthreads();
-    const int full_tiles = (p.split_keys + kBlockN - 1) / kBlockN;
-    const int full_bucket = min(full_tiles, kPlanBuckets - 1);
-    for (int b = tid; b < p.B; b += kPlanThreads) {
-        const int L = p.seqlens_k[b];
-        const int ns = L > 0 ? (L + p.split_keys - 1) / p.split_keys : 1;
-        if (ns > p.max_splits || L < 0) {
-            atomicCAS(p.err, 0u, kErrDecodeBase + 1);  // max_seqlen_k was too small
-            continue;
+    for (int base = 0; base < p.B; base += kPlanThreads) {
+        const int b = base + tid;
+        long long w = 0;
+        if (b < p.B) {
+            const int L = p.seqlens_k[b];
+            if (L < 0 || L > p.max_seqlen_k) atomicCAS(p.err, 0u, kErrDecodeBase + 1);
+            w = (long long)p.Hkv * ((checked_len(p, b) + kBlockN - 1) / kBlockN + kDecodeSegCost);
         }
-        const int last_tiles = (L - (ns - 1) * p.split_keys + kBlockN - 1) / kBlockN;
-        if (ns > 1) atomicAdd(&hist[full_bucket], (ns - 1) * p.Hkv);
-        atomicAdd(&hist[min(last_tiles, kPlanBuckets - 1)], p.Hkv);
+        long long x = w;  // inclusive scan within the warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_incl[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            long long t = warp_incl[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const long long y = __shfl_up_sync(0xffffffffu, t, o);
+                if (lane >= o) t += y;
+            }
+            warp_incl[lane] = t;
+        }
+        __syncthreads();
+        const long long before = carry + (warp > 0 ? warp_incl[warp - 1] : 0) + (x - w);
+        if (b < p.B) p.seq_prefix[b] = before;
+        __syncthreads();
+        if (tid == kPlanThreads - 1) carry = before + w;
+        __syncthreads();
     }
-    __syncthreads();
+    const long long total = carry;
+    long long rw = 0, n_ranges;
+    if (p.split_keys > 0) {
+        rw = p.split_keys / kBlockN;
+        n_ranges = (total + rw - 1) / rw;
+    } else {
+        // balanced: range r starts at floor(r * total / n_ranges)
+        n_ranges = (total + kDecodeMinRangeWeight - 1) / kDecodeMinRangeWeight;
+        n_ranges = max(1ll, min(n_ranges, (long long)n_ctas));
+    }
+    if (n_ranges > p.max_ranges) {  // cannot happen for lengths <= max_seqlen_k
+        if (tid == 0) atomicCAS(p.err, 0u, kErrDecodeBase + 2);
+        n_ranges = 0;
+    }
     if (tid == 0) {
-        int off = 0;
-        for (int k = kPlanBuckets - 1; k >= 0; --k) {
-            offs[k] = off;
-            off += hist[k];
-        }
-        p.work_meta[0] = off;  // number of items
-        p.work_meta[1] = 0;    // next item to take
+        p.seq_prefix[p.B] = total;
+        p.plan->range_weight = rw;
+        p.plan->total_weight = total;
+        p.plan->n_ranges = (int)n_ranges;
     }
-    __syncthreads();
-    for (int b = tid; b < p.B; b += kPlanThreads) {
-        const int L = p.seqlens_k[b];
-        const int ns = L > 0 ? (L + p.split_keys - 1) / p.split_keys : 1;
-        if (ns > p.max_splits || L < 0) continue;
-        for (int s = 0; s < ns; ++s) {
-            const int keys = min(L, (s + 1) * p.split_keys) - s * p.split_keys;
-            const int bucket = min((keys + kBlockN - 1) / kBlockN, kPlanBuckets - 1);
-            const int pos = atomicAdd(&offs[bucket], p.Hkv);
-            for (int g = 0; g < p.Hkv; ++g) p.items[pos + g] = make_int4(b, g, s, ns);
+    // the unit holding weight position x: last sequence whose prefix is <= x,
+    // then the kv head within it
+    auto unit_at = [&](long long x) {
+        int lo = 0, hi = p.B - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.seq_prefix[mid] <= x) lo = mid;
+            else hi = mid - 1;
         }
+        const long long wu = (checked_len(p, lo) + kBlockN - 1) / kBlockN + kDecodeSegCost;
+        return lo * p.Hkv + (int)min((long long)(p.Hkv - 1), (x - p.seq_prefix[lo]) / wu);
+    };
+    for (long long r = tid; r < n_ranges; r += kPlanThreads) {
+        const long long a = plan_range_begin(rw, total, n_ranges, r);
+        const long long e = min(total, plan_range_begin(rw, total, n_ranges, r + 1));
+        p.range_units[r] = make_int2(unit_at(a), unit_at(e - 1));
+    }
+}
+
+// Partial slot of piece `seg` of a unit whose piece lies in range r: the
+// unit's first piece takes its range's slot 2r + 1 (a unit continuing into
+// the next range), every later piece its range's slot 2r (a unit continuing
+// from the previous range).  A range holds at most one of each.
+__device__ __forceinline__ int piece_slot(int r, int seg) { return seg == 0 ? 2 * r + 1 : 2 * r; }
+
+// ------------------------------------------------------------------ merge
+// One CTA per range (looping when there are more ranges than CTAs): if the
+// last unit of range r has its first piece in r and continues into later
+// ranges, combine its pieces in key order,
+//   LSE = log sum_s exp(LSE_s),  O = sum_s exp(LSE_s - LSE) O_s,
+// one thread per (row, quarter of the head dimension).
+template <int D, bool BF16>
+__global__ void __launch_bounds__(4 * kBlockM, 1)
+    attn_decode_merge_kernel(const __grid_constant__ DecodeParams p) {
+    constexpr int kPartD = D / 4;
+    const volatile DecodePlan* plan = p.plan;
+    const long long rw = plan->range_weight;
+    const long long total = plan->total_weight;
+    const int n_ranges = plan->n_ranges;
+    const int row = threadIdx.x % kBlockM;
+    const int part = threadIdx.x / kBlockM;
+    if (row >= p.rows) return;
+    const int tok = row / p.G;
+    const int head_in_group = row % p.G;
+    for (int r = blockIdx.x; r < n_ranges; r += gridDim.x) {
+        const int u = p.range_units[r].y;
+        const int b = u / p.Hkv, g = u - b * p.Hkv;
+        const int tiles = (checked_len(p, b) + kBlockN - 1) / kBlockN;
+        if (tiles == 0) continue;
+        const long long k0 = p.seq_prefix[b] + (long long)g * (tiles + kDecodeSegCost) +
+                             kDecodeSegCost;
+        if (plan_range_of(rw, total, n_ranges, k0) != r) continue;
+        const int nseg = (int)plan_range_of(rw, total, n_ranges, k0 + tiles - 1) - r + 1;
+        if (nseg == 1) continue;
+        float M = -INFINITY;
+        for (int s = 0; s < nseg; ++s)
+            M = fmaxf(M, p.part_lse[(size_t)piece_slot(r + s, s) * kBlockM + row]);
+        float tot = -INFINITY;
+        float acc[kPartD];
+#pragma unroll
+        for (int e = 0; e < kPartD; ++e) acc[e] = 0.f;
+        if (M != -INFINITY) {
+            float sum = 0.f;
+            for (int s = 0; s < nseg; ++s) {
+                const size_t sb = (size_t)piece_slot(r + s, s) * kBlockM + row;
+                const float ls = p.part_lse[sb];
+                const float w = ls == -INFINITY ? 0.f : __expf(ls - M);
+                sum += w;
+                const float4* src = reinterpret_cast<const float4*>(p.part_o + sb * D +
+                                                                     part * kPartD);
+#pragma unroll
+                for (int e = 0; e < kPartD / 4; ++e) {
+                    const float4 v4 = src[e];
+                    acc[4 * e] += w * v4.x;
+                    acc[4 * e + 1] += w * v4.y;
+                    acc[4 * e + 2] += w * v4.z;
+                    acc[4 * e + 3] += w * v4.w;
+                }
+            }
+            tot = M + __logf(sum);
+            const float inv = 1.f / sum;
+#pragma unroll
+            for (int e = 0; e < kPartD; ++e) acc[e] *= inv;
+        }
+        const int head = g * p.G + head_in_group;
+        store_row_part<kPartD, BF16>(
+            p.o, (((size_t)b * p.Nq + tok) * p.Hq + head) * D + part * kPartD, acc, 1.f);
+        if (part == 0) p.lse[((size_t)b * p.Hq + head) * p.Nq + tok] = tot;
     }
 }
 
@@ -290,10 +404,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_init(&bars->o_final, 1);
         ptx::mbar_init(&bars->o_free, kSoftmaxWarps);
         for (int s = 0; s < 4; ++s) ptx::mbar_init(&bars->row_sync[s], 4);
-        ptx::mbar_init(&bars->ep_sync, kSoftmaxWarps);
         ptx::mbar_init(&bars->drain, 1);
         bars->abort = 0;
-        bars->is_last = 0;
         ptx::fence_barrier_init();
     }
     if (warp == kLoaderWarp && lane == 0) {
@@ -311,38 +423,72 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = bars->tmem_base;
 
     auto item_tiles = [&](const TcItem& it, int& key_begin, int& key_end) {
-        key_begin = it.split * p.split_keys;
-        key_end = min(it.Lk, key_begin + p.split_keys);
+        key_begin = it.key_begin;
+        key_end = it.key_end;
         return (key_end - key_begin + kBlockN - 1) / kBlockN;  // 0 only for an empty sequence
     };
 
     if (warp == kLoaderWarp) {
         // ================================================= loader
-        const int n_items = *reinterpret_cast<volatile int*>(p.work_meta);
-        int n = 0;       // items pushed
-        int it = 0;      // items with keys (Q loads)
-        int tg = 0;      // K/V tile pairs issued
-        int k_extra = 0;  // a K tile issued without its V tile (error exit)
-        int w = 0;
-        if (lane == 0) w = atomicAdd(p.work_meta + 1, 1);
-        w = __shfl_sync(0xffffffffu, w, 0);
-        while (true) {
-            TcItem item{-1, 0, 0, 1, 0, 0, 0, 0};
-            int w_next = 0;
-            if (w < n_items) {
-                const int4 e = p.items[w];
-                item.b = e.x;
-                item.g = e.y;
-                item.split = e.z;
-                item.nsplit = e.w;
-                item.Lk = p.seqlens_k[e.x];
-                item.slot0 = p.cu_seqlens_k[e.x];
-                if (lane == 0) w_next = atomicAdd(p.work_meta + 1, 1);  // resolves later
+        const volatile DecodePlan* plan = p.plan;
+        const long long rw = plan->range_weight;
+        const long long total = plan->total_weight;
+        const int n_ranges = plan->n_ranges;
+        // the units of range r, first to last (those outside it give no piece)
+        int r = blockIdx.x;
+        int2 ru = r < n_ranges ? p.range_units[r] : make_int2(0, -1);
+        int step = 0;
+        auto next_item = [&](TcItem& item) {
+            item = TcItem{-1, 0, 0, 0, 1, 0, 0, 0, 0, 0, 0, 0};
+            while (r < n_ranges) {
+                const long long a = plan_range_begin(rw, total, n_ranges, r);
+                const long long e = min(total, plan_range_begin(rw, total, n_ranges, r + 1));
+                while (step <= ru.y - ru.x) {
+                    const int u = ru.x + step;
+                    ++step;
+                    const int b = u / p.Hkv, g = u - b * p.Hkv;
+                    const int Lk = checked_len(p, b);
+                    const int tiles = (Lk + kBlockN - 1) / kBlockN;
+                    const long long pu = p.seq_prefix[b] + (long long)g * (tiles + kDecodeSegCost);
+                    const long long k0 = pu + kDecodeSegCost;  // weight position of tile 0
+                    int t0 = 0, t1 = 0, nseg = 1, seg = 0;
+                    if (tiles == 0) {
+                        if (pu < a || pu >= e) continue;  // owned by the range holding pu
+                    } else {
+                        t0 = (int)min((long long)tiles, max(0ll, a - k0));
+                        t1 = (int)min((long long)tiles, max(0ll, e - k0));
+                        if (t1 <= t0) continue;
+                        const int r_first = (int)plan_range_of(rw, total, n_ranges, k0);
+                        nseg = (int)plan_range_of(rw, total, n_ranges, k0 + tiles - 1) - r_first + 1;
+                        seg = r - r_first;
+                    }
+                    item.b = b;
+                    item.g = g;
+                    item.key_begin = t0 * kBlockN;
+                    item.key_end = min(Lk, t1 * kBlockN);
+                    item.nseg = nseg;
+                    item.seg = seg;
+                    item.range = r;
+                    item.Lk = Lk;
+                    item.slot0 = p.cu_seqlens_k[b];
+                    return;
+                }
+                r += gridDim.x;  // this range is done
+                step = 0;
+                if (r < n_ranges) ru = p.range_units[r];
             }
+        };
+        int n = 0;        // items pushed
+        int it = 0;       // items with keys (Q loads)
+        int tg = 0;       // K/V tile pairs issued
+        int k_extra = 0;  // a K tile issued without its V tile (error exit)
+        TcItem item;
+        next_item(item);
+        while (true) {
             const int slot = n % kItemRing;
             if (!warp_wait(&bars->item_empty[slot], ((n / kItemRing) & 1) ^ 1, p.limit_ns,
                            abort_flag)) {
-                record_error(p.err, kErrDecodeBase + 2, &bars->abort);
+                record_error(p.err, kErrDecodeBase + 3, &bars->abort);
                 break;
             }
             if (lane == 0) {
@@ -354,6 +500,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (item.b < 0) break;
             int key_begin, key_end;
             const int nt = item_tiles(item, key_begin, key_end);
+            TcItem next;
+            bool have_next = false;
             bool ok = true;
             if (nt > 0) {
                 if (!warp_wait(&bars->q_empty, (it & 1) ^ 1, p.limit_ns, abort_flag)) {
@@ -399,10 +547,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              &tm_v, &bars->v_full[sv], c * 64, item.g, row0);
                     }
                     __syncwarp();
+                    if (j == 0) {
+                        // look the next piece up while this one's tiles stream in
+                        next_item(next);
+                        have_next = true;
+                    }
                 }
             }
             if (!ok) break;
-            w = __shfl_sync(0xffffffffu, w_next, 0);
+            if (!have_next) next_item(next);
+            item = next;
         }
         // leave no copy in flight: the last Q and up to KST / VST tiles
         int zero = 0;
@@ -501,30 +655,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool valid_row = (int)row < p.rows;
         const float sl2 = p.scale_log2;
         float* red = reinterpret_cast<float*>(smem + L::kRed);
-        float* row_lse = reinterpret_cast<float*>(smem + L::kRowLse);
         const uint32_t t_o = tmem + lane_addr + kColO + (uint32_t)(part * kPartD);
         uint64_t* row_bar = &bars->row_sync[quarter];
         bool ok = true;
-        int n = 0, it = 0, tg = 0, rs = 0, es = 0;
+        int n = 0, it = 0, tg = 0, rs = 0;
 
+        // The softmax warps keep an item's ring slot until they start the
+        // next item and read its fields from shared memory when needed
+        // (fewer live registers across the tile loop).
         while (ok) {
+            if (n > 0) {
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&bars->item_empty[(n - 1) % kItemRing]);
+            }
             const int slot = n % kItemRing;
             if (!warp_wait(&bars->item_full[slot], (n / kItemRing) & 1, p.limit_ns, abort_flag)) {
                 record_error(p.err, kErrDecodeBase + 12, &bars->abort);
                 break;
             }
-            const TcItem item = bars->item[slot];
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&bars->item_empty[slot]);
+            const TcItem* itp = &bars->item[slot];
             ++n;
-            if (item.b < 0) break;
-            const int b = item.b, g = item.g;
-            const int head = g * p.G + head_in_group;
-            const size_t o_elem = (((size_t)b * p.Nq + tok) * p.Hq + head) * D + part * kPartD;
-            const size_t lse_idx = ((size_t)b * p.Hq + head) * p.Nq + tok;
-            int key_begin, key_end;
-            const int nt = item_tiles(item, key_begin, key_end);
+            if (itp->b < 0) break;
+            auto out_index = [&](size_t& o_elem, size_t& lse_idx) {
+                const int head = itp->g * p.G + head_in_group;
+                o_elem = (((size_t)itp->b * p.Nq + tok) * p.Hq + head) * D + part * kPartD;
+                lse_idx = ((size_t)itp->b * p.Hq + head) * p.Nq + tok;
+            };
+            const int key_begin = itp->key_begin, key_end = itp->key_end;
+            const int nt = (key_end - key_begin + kBlockN - 1) / kBlockN;
             if (nt == 0) {
+                size_t o_elem, lse_idx;
+                out_index(o_elem, lse_idx);
                 // empty sequence: nothing to attend to
                 if (valid_row) {
                     float zeros[kPartD];
@@ -536,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 continue;
             }
             int row_lim = key_end - 1;  // last visible key (absolute index)
-            if (p.causal) row_lim = min(row_lim, tok + item.Lk - p.Nq);
+            if (p.causal) row_lim = min(row_lim, tok + itp->Lk - p.Nq);
 
             // ---- Q -> tensor memory (A operand of S = Q Kᵀ)
             if (!warp_wait(&bars->q_full, it & 1, p.limit_ns, abort_flag)) {
@@ -713,83 +874,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             float of[kPartD];
 #pragma unroll
             for (int e = 0; e < kPartD; ++e) of[e] = __uint_as_float(o[e]);
-            if (item.nsplit == 1) {
+            size_t o_elem, lse_idx;
+            out_index(o_elem, lse_idx);
+            const int nseg = itp->nseg;
+            if (nseg == 1) {
                 if (valid_row) {
                     store_row_part<kPartD, BF16>(p.o, o_elem, of, inv_l);
                     if (part == 0) p.lse[lse_idx] = lse_nat;
                 }
                 continue;
             }
-            // normalised partial O (fp32) and LSE of this split
-            const size_t unit = (size_t)b * p.Hkv + g;
-            const size_t pbase = (unit * p.max_splits + item.split) * kBlockM + row;
+            // normalised partial O (fp32) and LSE of this piece, in the slot
+            // of its range; the merge kernel combines the pieces
+            const size_t pbase = (size_t)piece_slot(itp->range, itp->seg) * kBlockM + row;
             float* po = p.part_o + pbase * D + part * kPartD;
 #pragma unroll
             for (int e = 0; e < kPartD; e += 4)
                 *reinterpret_cast<float4*>(po + e) = make_float4(
                     of[e] * inv_l, of[e + 1] * inv_l, of[e + 2] * inv_l, of[e + 3] * inv_l);
             if (part == 0) p.part_lse[pbase] = lse_nat;
-            // the CTA that completes the last split of this unit merges them
-            __threadfence();
-            if (!warp_barrier(&bars->ep_sync, es, p.limit_ns, abort_flag)) {
-                record_error(p.err, kErrDecodeBase + 15, &bars->abort);
-                break;
-            }
-            if (tid == 0) {
-                const unsigned prev = atomicAdd(p.counters + unit, 1u);
-                bars->is_last = (prev == (unsigned)(item.nsplit - 1)) ? 1 : 0;
-            }
-            if (!warp_barrier(&bars->ep_sync, es, p.limit_ns, abort_flag)) {
-                record_error(p.err, kErrDecodeBase + 15, &bars->abort);
-                break;
-            }
-            if (!bars->is_last) continue;
-            __threadfence();
-            const float* pl = p.part_lse + unit * p.max_splits * kBlockM;
-            const float* pov = p.part_o + unit * p.max_splits * kBlockM * D;
-            if (tid < kBlockM) {
-                float M = -INFINITY;
-                for (int s2 = 0; s2 < item.nsplit; ++s2)
-                    M = fmaxf(M, __ldcg(pl + s2 * kBlockM + tid));
-                float tot = -INFINITY;
-                if (M != -INFINITY) {
-                    float acc = 0.f;
-                    for (int s2 = 0; s2 < item.nsplit; ++s2) {
-                        const float ls = __ldcg(pl + s2 * kBlockM + tid);
-                        if (ls != -INFINITY) acc += __expf(ls - M);
-                    }
-                    tot = M + __logf(acc);
-                }
-                row_lse[tid] = tot;
-            }
-            if (!warp_barrier(&bars->ep_sync, es, p.limit_ns, abort_flag)) {
-                record_error(p.err, kErrDecodeBase + 15, &bars->abort);
-                break;
-            }
-            if (valid_row) {
-                const float tot = row_lse[row];
-                float acc[kPartD];
-#pragma unroll
-                for (int e = 0; e < kPartD; ++e) acc[e] = 0.f;
-                if (tot != -INFINITY) {
-                    for (int s2 = 0; s2 < item.nsplit; ++s2) {
-                        const float ls = __ldcg(pl + s2 * kBlockM + row);
-                        if (ls == -INFINITY) continue;
-                        const float wgt = __expf(ls - tot);
-                        const float* src = pov + ((size_t)s2 * kBlockM + row) * D + part * kPartD;
-#pragma unroll
-                        for (int e = 0; e < kPartD; e += 4) {
-                            const float4 v4 = __ldcg(reinterpret_cast<const float4*>(src + e));
-                            acc[e] += wgt * v4.x;
-                            acc[e + 1] += wgt * v4.y;
-                            acc[e + 2] += wgt * v4.z;
-                            acc[e + 3] += wgt * v4.w;
-                        }
-                    }
-                }
-                store_row_part<kPartD, BF16>(p.o, o_elem, acc, 1.f);
-                if (part == 0) p.lse[lse_idx] = tot;
-            }
         }
     }
 
@@ -811,10 +914,13 @@ cudaError_t launch_t(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUt
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc);
     if (e != cudaSuccess) return e;
-    attn_decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(p);
+    attn_decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(p, n_ctas);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     kern<<<n_ctas, kThreads, L::kAlloc, stream>>>(qmap, kmap, vmap, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attn_decode_merge_kernel<D, BF16><<<n_ctas, 4 * kBlockM, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

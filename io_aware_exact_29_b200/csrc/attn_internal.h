@@ -44,8 +44,12 @@ struct DecodeParams {
     float* part_o;         // [B, Hkv, n_mgroups, max_splits, R, d] fp32 (R = 16, or 128 for tc)
     float* part_lse;       // [B, Hkv, n_mgroups, max_splits, R]
     unsigned* counters;    // [B, Hkv, n_mgroups]
-    int4* items;           // tc: work list {b, g, split, nsplit}, longest first
-    int* work_meta;        // tc: [0] number of items, [1] next item to take
+    // tensor-core decode schedule (written by its plan kernel)
+    struct DecodePlan* plan;
+    long long* seq_prefix;  // [B + 1] weight before sequence b
+    int2* range_units;      // [max_ranges] first and last unit of range r
+    int max_seqlen_k;
+    int max_ranges;
     int B, Hq, Hkv, Nq, G;
     int rows;              // Nq * G query rows per (sequence, kv head)
     int n_mgroups;         // ceil(rows / 16)
@@ -57,10 +61,37 @@ struct DecodeParams {
     unsigned* err;
 };
 
+// Tensor-core decode schedule.  The work of unit (b, g) -- sequence b, kv
+// head g -- weighs its key tiles plus kDecodeSegCost tiles of per-segment
+// overhead; units are laid end to end in (b, g) order and the total weight
+// is cut into n_ranges equal ranges, one CTA each (stream-K style), so that
+// a unit is split only where a range boundary falls inside it.
+constexpr int kDecodeSegCost = 2;        // weight of a segment's set-up, in tiles
+constexpr int kDecodeMinRangeWeight = 8; // smallest range weight in automatic mode
+constexpr int kDecodeMaxRangesAuto = 192;
+
+struct DecodePlan {
+    long long range_weight;  // > 0: ranges of this weight; 0: n_ranges balanced ranges
+    long long total_weight;
+    int n_ranges;
+    int pad;
+};
+
+// First weight position of range r, and the range that holds position x.
+__host__ __device__ inline long long plan_range_begin(long long rw, long long total, long long n,
+                                                      long long r) {
+    return rw > 0 ? r * rw : (r * total) / n;
+}
+__host__ __device__ inline long long plan_range_of(long long rw, long long total, long long n,
+                                                   long long x) {
+    return rw > 0 ? x / rw : ((x + 1) * n - 1) / total;
+}
+
 struct DecodeLayout {
     int tc;  // 1: tensor-core kernel (one 128-row tile per unit), 0: mma.sync kernel
     int split_keys, max_splits, n_mgroups;
-    size_t part_o_off, part_lse_off, counters_off, items_off, meta_off, total;
+    int max_ranges;  // tc: bound on the number of ranges (two partial slots each)
+    size_t part_o_off, part_lse_off, counters_off, prefix_off, ranges_off, plan_off, total;
 };
 
 // The tensor-core decode takes the shapes whose Nq * G query rows per kv

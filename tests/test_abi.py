@@ -99,16 +99,26 @@ def test_decode_workspace_accounting():
 
 
 def test_decode_workspace_accounting_tensor_core_layout():
-    # 16 new tokens x 8 query heads per kv head = 128 rows: one 128-row tile
-    # per (sequence, kv head); automatic split 8192 keys (256 units x 4
-    # splits >= 148 x 4 work items), 128 rows x (128 + 1) floats per split,
-    # a counter per unit, the 16-byte work-list entries and the list's header
+    # 16 new tokens x 8 query heads per kv head = 128 rows: the tensor-core
+    # decode.  Automatic mode cuts the work into at most 192 ranges, each
+    # owning two 128-row partial slots of (128 + 1) floats; plus the weight
+    # prefix over sequences (int64), each range's first and last unit and the
+    # plan header.  Independent of the lengths.
     n = attn.decode_workspace_bytes(32, 64, 8, 16, 128, 32768)
-    units, splits = 32 * 8, 4
-    expect = (units * splits * 128 * 128 * 4 + units * splits * 128 * 4 + units * 4
-              + units * splits * 16 + 8)
-    assert expect <= n <= expect + 4 * 256
-    # a split that is not a multiple of 128 keeps the 16-row layout
+    ranges = 192
+    expect = (2 * ranges * 128 * 128 * 4 + 2 * ranges * 128 * 4 + 33 * 8 + ranges * 8 + 24)
+    assert expect <= n <= expect + 5 * 256
+    assert n < 32 << 20  # fits the no-alloc entry point's scratch
+    # small problems need fewer ranges (at least 8 tiles of weight each)
+    n_small = attn.decode_workspace_bytes(2, 16, 2, 16, 128, 1000)
+    r_small = (4 * (8 + 2) + 7) // 8
+    assert n_small >= 2 * r_small * 128 * 128 * 4
+    assert n_small < 2 * (r_small + 1) * 128 * 128 * 4
+    # with split_keys, ranges of split_keys / 128 tiles of weight
+    n_split = attn.decode_workspace_bytes(2, 16, 2, 16, 128, 1000, split_keys=256)
+    r_split = (4 * (8 + 2) + 1) // 2
+    assert 2 * r_split * 128 * 128 * 4 <= n_split < 2 * (r_split + 1) * 128 * 128 * 4
+    # a split that is not a multiple of 128 keeps the mma.sync layout
     n64 = attn.decode_workspace_bytes(32, 64, 8, 16, 128, 32768, split_keys=64)
     expect64 = 32 * 8 * 8 * 512 * 16 * 128 * 4 + 32 * 8 * 8 * 512 * 16 * 4 + 32 * 8 * 8 * 4
     assert expect64 <= n64 <= expect64 + 3 * 256
