@@ -4,9 +4,12 @@ A step is one pass of the whole path over one batch of synthetic inputs:
   forward  : B=4, H=16, N=4096, d=128, bf16, non-causal (the long-sequence
              sweep point at which the forward target is stated), then
   decode   : Llama2-70B shape, B=32, Hq=64, Hkv=8, d=128, one new token per
-             sequence, packed bf16 KV cache with lengths ~ U[1, 32768].
+             sequence, packed bf16 KV cache with lengths ~ U[1, 32768], then
+  decode16 : the same shape with a causal chunk of 16 new tokens per sequence
+             (its own cache of the same size).
 `value` is the forward's TFLOP/s (algorithmic FLOPs / device time of the
-forward launches, summed over ranks); the decode's GB/s is reported beside it.
+forward launches, summed over ranks); the decodes' GB/s are reported beside
+it.
 All inputs are larger than L2 (126 MB), so no flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -41,11 +44,12 @@ from io_aware_exact_29_b200.workloads import (DECODE_CASES, FWD_CASES, fwd_input
 
 FWD_CASE = FWD_CASES["sweep_d128_n4096"]
 DEC_CASE = DECODE_CASES["llama70b_decode"]
+DEC16_CASE = DECODE_CASES["llama70b_chunk16"]
 METRIC = "attn fwd TFLOP/s & % of BF16 TC peak; KV-cache decode GB/s & % of HBM peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = {
     "fwd": os.path.join(ROOT, "io_aware_exact_29_b200", "csrc", "attn_fwd_sm100a.cu"),
-    "decode": os.path.join(ROOT, "io_aware_exact_29_b200", "csrc", "attn_decode_sm100a.cu"),
+    "decode": os.path.join(ROOT, "io_aware_exact_29_b200", "csrc", "attn_decode_tc_sm100a.cu"),
 }
 L2_BYTES = 126 * 2 ** 20
 
@@ -196,8 +200,18 @@ def run_ours(args, rank, world, local):
     dlse = torch.empty((dc.B, dc.Hq, dc.Nq), dtype=torch.float32, device=dev)
     ws = torch.empty(attn.decode_workspace_bytes(dc.B, dc.Hq, dc.Hkv, dc.Nq, dc.d, max_len),
                      dtype=torch.uint8, device=dev)
+    # the 16-token chunk variant of the decode (same cache shape, causal chunk)
+    c16 = DEC16_CASE
+    din16 = kvcache_inputs(c16, seed=1000 * rank + 1, device=str(dev))
+    max16 = int(din16["seqlens_k"].max().item())
+    o16 = torch.empty_like(din16["q"])
+    l16 = torch.empty((c16.B, c16.Hq, c16.Nq), dtype=torch.float32, device=dev)
+    ws16 = torch.empty(attn.decode_workspace_bytes(c16.B, c16.Hq, c16.Hkv, c16.Nq, c16.d, max16),
+                       dtype=torch.uint8, device=dev)
     fflops = fwd_work(fc)
     dbytes = accounting.decode_bytes(sl.tolist(), dc.B, dc.Hq, dc.Hkv, dc.Nq, dc.d)
+    dbytes16 = accounting.decode_bytes(din16["seqlens_k"].tolist(), c16.B, c16.Hq, c16.Hkv,
+                                       c16.Nq, c16.d)
 
     def step(ev):
         ev[0].record(stream)
@@ -207,8 +221,13 @@ def run_ours(args, rank, world, local):
                                      causal=dc.causal, workspace=ws, out=do, lse=dlse,
                                      stream=stream)
         ev[2].record(stream)
+        attn.attn_fwd_varlen_kvcache(din16["q"], din16["k_cache"], din16["v_cache"],
+                                     din16["cu_seqlens_k"], din16["seqlens_k"], max16,
+                                     scale=c16.scale, causal=c16.causal, workspace=ws16, out=o16,
+                                     lse=l16, stream=stream)
+        ev[3].record(stream)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     for _ in range(args.warmup):
         step(evs[0])
     torch.cuda.synchronize()
@@ -229,7 +248,9 @@ def run_ours(args, rank, world, local):
     total_ms = t0.elapsed_time(t1)
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
     dec_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
-    total_ms, fwd_ms, dec_ms = reduce_max([total_ms, fwd_ms, dec_ms], world, dev)
+    dec16_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
+    total_ms, fwd_ms, dec_ms, dec16_ms = reduce_max([total_ms, fwd_ms, dec_ms, dec16_ms], world,
+                                                    dev)
     assert attn.get_device_error() == 0
 
     # ---- end to end through the public API with host buffers
@@ -244,6 +265,8 @@ def run_ours(args, rank, world, local):
     peak_t = peaks["bf16_tflops_sustained"]
     dec_launch_ms = dec_ms / args.steps
     dec_achieved = dbytes / (dec_launch_ms * 1e-3) / 1e9
+    dec16_call_ms = dec16_ms / args.steps
+    dec16_achieved = dbytes16 / (dec16_call_ms * 1e-3) / 1e9
 
     out = {
         "metric": METRIC,
@@ -265,7 +288,11 @@ def run_ours(args, rank, world, local):
             "fwd": {"B": fc.B, "H": fc.Hq, "N": fc.Nq, "d": fc.d, "causal": fc.causal},
             "decode": {"B": dc.B, "Hq": dc.Hq, "Hkv": dc.Hkv, "d": dc.d, "Nq": dc.Nq,
                        "sum_len": int(sl.sum().item()), "max_len": max_len},
-            "l2": "inputs larger than L2 (fwd 268 MB, decode cache 2.1 GB); no flush",
+            "decode_chunk16": {"B": c16.B, "Hq": c16.Hq, "Hkv": c16.Hkv, "d": c16.d,
+                               "Nq": c16.Nq, "causal": c16.causal,
+                               "sum_len": int(din16["seqlens_k"].sum().item()),
+                               "max_len": max16},
+            "l2": "inputs larger than L2 (fwd 268 MB, each decode cache 2.1 GB); no flush",
             "parallelism": f"replicas x{world} (independent problems per GPU, no collective)",
         },
         "roofline": {
@@ -283,21 +310,34 @@ def run_ours(args, rank, world, local):
         "decode": {
             "value": round(dec_gbs, 1),
             "unit": "GB/s",
-            "achieved_per_launch": round(dec_achieved, 1),
+            "achieved_per_call": round(dec_achieved, 1),
             "peak": peaks["hbm_gbs"],
             "frac": round(dec_achieved / peaks["hbm_gbs"], 4),
-            "bytes_per_launch": dbytes,
-            "ms_per_launch": round(dec_launch_ms, 4),
+            "bytes_per_call": dbytes,
+            "ms_per_call": round(dec_launch_ms, 4),
+            "kernels_per_call": "plan + attn_decode_tc_kernel + merge",
             "bound": "hbm",
             "traffic": load_traffic("decode"),
             "e2e": {"value": round(dbytes * world / (e2e_dec_ms * 1e-3) / 1e9, 1),
                     "unit": "GB/s", "h2d_bytes_per_step": e2e["dec_h2d"],
                     "d2h_bytes_per_step": e2e["dec_d2h"]},
         },
+        "decode_chunk16": {
+            "value": round(dbytes16 * args.steps * world / (dec16_ms * 1e-3) / 1e9, 1),
+            "unit": "GB/s",
+            "achieved_per_call": round(dec16_achieved, 1),
+            "peak": peaks["hbm_gbs"],
+            "frac": round(dec16_achieved / peaks["hbm_gbs"], 4),
+            "bytes_per_call": dbytes16,
+            "ms_per_call": round(dec16_call_ms, 4),
+            "kernels_per_call": "plan + attn_decode_tc_kernel + merge",
+            "bound": "hbm",
+        },
         "e2e": {"value": round(fflops * world / (e2e_fwd_ms * 1e-3) / 1e12, 2),
                 "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["fwd_h2d"],
                 "d2h_bytes_per_step": e2e["fwd_d2h"]},
-        "gpu_launches": 2 * args.steps,
+        # per step: the forward kernel, and plan + decode + merge for each decode
+        "gpu_launches": 7 * args.steps,
         "clocks": clk.summary(),
         "fwd_ms_per_launch": round(per_launch_ms, 4),
     }

@@ -8,6 +8,10 @@
 // 什么额外的事", point 3).  Within a split the keys are processed tile by tile
 // with a running max and sum (section "FlashAttention 拆的不是算法，是数据流").
 //
+// This kernel serves the shapes the tensor-core decode (attn_decode_tc_sm100a.cu)
+// does not take: query heads per kv head that do not divide 128, more than
+// 128 query rows per kv head, or a split size that is not a multiple of 128.
+//
 // Work unit = one CTA: (sequence b, kv head g, key split s, group of 16 query
 // rows).  The query rows of a kv head are the Nq tokens x G query heads that
 // share it (row r = token r / G, head g*G + r % G), so one pass over the cache

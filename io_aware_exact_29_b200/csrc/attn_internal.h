@@ -95,10 +95,13 @@ struct DecodeLayout {
 };
 
 // The tensor-core decode takes the shapes whose Nq * G query rows per kv
-// head fill 64..128 rows of one tile, with whole 128-key tiles per split.
+// head fit one 128-row tile with whole tokens (G divides 128), with ranges
+// of whole 128-key tiles.  Even one token (8 of 128 rows) runs faster there
+// than on the mma.sync kernel: the loop is bound by HBM, and the idle MMA
+// rows cost nothing that the memory pipe waits for.
 inline bool decode_use_tc(int G, int Nq, int split_keys) {
     const int rows = Nq * G;
-    return G <= 128 && 128 % G == 0 && rows >= 64 && rows <= 128 && split_keys % 128 == 0;
+    return G <= 128 && 128 % G == 0 && rows <= 128 && split_keys % 128 == 0;
 }
 
 DecodeLayout decode_layout(int B, int Hq, int Hkv, int Nq, int d, int max_seqlen_k,

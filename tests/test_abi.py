@@ -90,9 +90,10 @@ def test_decode_rejects_bad_arguments():
 
 
 def test_decode_workspace_accounting():
-    # B=32, Hkv=8 one row group (8 query rows), auto split of 1024 keys over
+    # mma.sync decode (12 query heads per kv head do not divide 128): B=32,
+    # Hkv=8, one row group (12 query rows), auto split of 1024 keys over
     # 32768 keys: 32 splits x 16 padded rows x (128 + 1) floats + counters
-    n = attn.decode_workspace_bytes(32, 64, 8, 1, 128, 32768)
+    n = attn.decode_workspace_bytes(32, 96, 8, 1, 128, 32768)
     units, splits = 32 * 8, 32
     expect = units * splits * 16 * 128 * 4 + units * splits * 16 * 4 + units * 4
     assert expect <= n <= expect + 3 * 256

@@ -82,9 +82,10 @@ def test_chunk_causal_bottom_right(nq):
         assert torch.all(torch.isneginf(lse[4, :, : nq - 3]))
 
 
-# Shapes whose Nq * G query rows per kv head fill 64..128 rows run on the
-# tensor-core decode kernel (one 128-row tile per CTA, 128-key tiles); the
-# rest, and split sizes that are not a multiple of 128, on the mma.sync one.
+# Shapes whose G query heads per kv head divide 128 and whose Nq * G query
+# rows fit 128 run on the tensor-core decode kernel (one 128-row tile, 128-key
+# tiles, stream-K ranges); the rest, and split sizes that are not a multiple
+# of 128, on the mma.sync one.
 TC_LENS = [0, 1, 15, 16, 17, 127, 128, 129, 511, 512, 513, 2047, 2048, 2049, 5000]
 
 
@@ -157,6 +158,19 @@ def test_max_seqlen_too_small_is_reported():
                                  dev["seqlens_k"], 1000, scale=c.scale, split_keys=256)
     torch.cuda.synchronize()
     assert attn.get_device_error() == attn.ERR_DECODE_BASE + 1
+
+
+# The mma.sync kernel: query heads per kv head that do not divide 128, more
+# than 128 query rows per kv head, or split sizes that are not a multiple of
+# 128.
+@pytest.mark.parametrize("hq,hkv,nq,split", [(24, 2, 1, 0), (24, 2, 11, 0), (12, 2, 5, 256),
+                                             (32, 2, 16, 0), (16, 2, 1, 64), (16, 2, 16, 320)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_mma_sync_path_shapes(hq, hkv, nq, split, causal):
+    lens = [0, 1, 63, 64, 65, 129, 1000, 2500]
+    c = DecodeCase("ms", len(lens), hq, hkv, nq, 128, (0, 2500), causal, slack=2)
+    inp = kvcache_inputs(c, seed=40 + nq, seqlens=lens)
+    _check(inp, c, split_keys=split, what=f"mma.sync {hq}/{hkv} nq {nq} split {split}")
 
 
 def test_tensor_core_max_seqlen_too_small_is_reported():

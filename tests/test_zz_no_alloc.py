@@ -40,11 +40,16 @@ def test_declared_and_exported():
 def test_rejects_sizes_beyond_the_scratch_before_any_work():
     fn = _noalloc_fn()
     P = 1 << 20
-    # Llama2-70B decode shape with the automatic 1024-key split needs ~68 MB
-    need = attn.decode_workspace_bytes(32, 64, 8, 1, 128, 32768)
+    # 12 query heads per kv head (the mma.sync decode) at the Llama2-70B
+    # batch and lengths, automatic 1024-key split: ~68 MB
+    need = attn.decode_workspace_bytes(32, 96, 8, 1, 128, 32768)
     assert need > SCRATCH_BYTES
-    rc = fn(P, P, P, P, P, 32768, 1 << 20, P, P, 32, 64, 8, 1, 128, 0.088, 0, 0, 0, None)
+    rc = fn(P, P, P, P, P, 32768, 1 << 20, P, P, 32, 96, 8, 1, 128, 0.088, 0, 0, 0, None)
     assert rc == -4  # ATTN_ERR_WORKSPACE
+    # the tensor-core decode with ranges of 128 keys: far beyond the scratch
+    assert attn.decode_workspace_bytes(32, 64, 8, 1, 128, 32768, split_keys=128) > SCRATCH_BYTES
+    rc = fn(P, P, P, P, P, 32768, 1 << 20, P, P, 32, 64, 8, 1, 128, 0.088, 0, 0, 128, None)
+    assert rc == -4
     # invalid sizes are reported as such
     rc = fn(P, P, P, P, P, 100, 100, P, P, 2, 8, 2, 17, 128, 0.088, 0, 0, 0, None)
     assert rc == -1
@@ -77,6 +82,7 @@ def test_matches_the_workspace_entry_point_on_two_calls_in_a_row():
     cases = [
         (DecodeCase("a", 16, 32, 4, 1, 128, (1, 6000), False), 0, 11),
         (DecodeCase("b", 6, 16, 2, 4, 128, (4, 3000), True), 256, 12),
+        (DecodeCase("c", 5, 24, 2, 1, 128, (1, 3000), False), 0, 13),  # mma.sync decode
     ]
     for case, split, seed in cases:
         inp = kvcache_inputs(case, seed=seed)
