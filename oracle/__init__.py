@@ -66,6 +66,10 @@ def _load():
             lib.oracle_lse_combine.restype = ctypes.c_int
             lib.oracle_lse_combine.argtypes = [_DP, _DP, ctypes.c_int, ctypes.c_int,
                                                ctypes.c_int, _DP, _DP]
+            lib.oracle_attn_bwd.restype = ctypes.c_int
+            lib.oracle_attn_bwd.argtypes = [
+                _DP, _DP, _DP, _DP, _DP, _DP, _DP, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, _IP]
             lib.oracle_max_threads.restype = ctypes.c_int
             lib.oracle_set_threads.argtypes = [ctypes.c_int]
             _lib = lib
@@ -161,4 +165,27 @@ def lse_combine(o_parts, lse_parts):
     return o, lse
 
 
-__all__ = ["build", "attn_fwd", "attn_kvcache", "lse_combine", "max_threads", "set_threads"]
+def attn_bwd(q, k, v, dout, scale: float, causal: bool, seqlens_k=None):
+    """Gradients (dq, dk, dv) of L = sum(dout * O) for O = attention(q, k, v).
+
+    q, dout [B, Nq, Hq, d]; k, v [B, Nk, Hkv, d]; seqlens_k optional [B].
+    Returns float64 numpy arrays dq [B, Nq, Hq, d], dk and dv [B, Nk, Hkv, d]
+    (dk, dv summed over the query heads that share a kv head; zero behind a
+    sequence's real key length).
+    """
+    qd, kd, vd, dod = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Nq, Hq, d = qd.shape
+    _, Nk, Hkv, _ = kd.shape
+    dq = np.full((B, Nq, Hq, d), np.nan)
+    dk = np.full((B, Nk, Hkv, d), np.nan)
+    dv = np.full((B, Nk, Hkv, d), np.nan)
+    sl = None if seqlens_k is None else _i32(seqlens_k)
+    rc = _load().oracle_attn_bwd(_dp(qd), _dp(kd), _dp(vd), _dp(dod), _dp(dq), _dp(dk), _dp(dv),
+                                 B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), _ip(sl))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_bwd rejected its arguments (rc={rc})")
+    return dq, dk, dv
+
+
+__all__ = ["build", "attn_fwd", "attn_kvcache", "lse_combine", "attn_bwd", "max_threads",
+           "set_threads"]

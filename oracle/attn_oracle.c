@@ -315,3 +315,144 @@ int oracle_lse_combine(const double* o_parts, const double* lse_parts, int npart
     }
     return 0;
 }
+
+/*
+ * Gradients of exact attention (the backward pass) -- the chain rule applied
+ * to the definition at the top of this file.  The pages report training
+ * speed-ups (effectstory.com article, "訓練性能量化提升" table) but print no
+ * backward algorithm, so this states the plain derivative of
+ *
+ *   L = sum_{b,i,h,t} dO[b,i,h,t] * O[b,i,h,t]
+ *
+ * for one (b, h) with kv head g and the row softmax P of the definition:
+ *
+ *   dV[j]    += sum_i P[i][j] * dO[i]                (summed over the G heads of g)
+ *   dP[i][j]  = dO[i] . V[j]
+ *   dS[i][j]  = P[i][j] * (dP[i][j] - sum_j' P[i][j'] * dP[i][j'])   (softmax Jacobian)
+ *   dQ[i]     = scale * sum_j dS[i][j] * K[j]
+ *   dK[j]    += scale * sum_i dS[i][j] * Q[i]       (summed over the G heads of g)
+ *
+ * Masked keys have P = 0 and therefore dS = 0; a row with no visible key
+ * contributes nothing.  P is recomputed here from q, k, v (no forward output
+ * or LSE is taken from the caller).  Every sum is compensated (Neumaier).
+ *   q, dout, dq [B, Nq, Hq, d]   k, v, dk, dv [B, Nk, Hkv, d]   seqlens_k: NULL or [B]
+ * Work is split over (b, g) so that the sums over the heads of a group are
+ * done by one thread in head order.  Returns 0, -1 (bad arguments) or -2.
+ */
+int oracle_attn_bwd(const double* q, const double* k, const double* v, const double* dout,
+                    double* dq, double* dk, double* dv, int B, int Hq, int Hkv, int Nq, int Nk,
+                    int d, double scale, int causal, const int* seqlens_k) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || d <= 0 || Hq % Hkv != 0) return -1;
+    if (seqlens_k)
+        for (int b = 0; b < B; ++b)
+            if (seqlens_k[b] < 0 || seqlens_k[b] > Nk) return -1;
+    const int G = Hq / Hkv;
+    const size_t nq1 = (size_t)(Nq > 0 ? Nq : 1), nk1 = (size_t)(Nk > 0 ? Nk : 1);
+    const size_t per_thread = (2 * nq1 * nk1 + 2 * nk1 * (size_t)d) * sizeof(double) +
+                              2 * nk1 * (size_t)d * sizeof(csum_t);
+    const int nthreads = pick_threads(per_thread);
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long bg = 0; bg < (long)B * Hkv; ++bg) {
+        const int b = (int)(bg / Hkv), g = (int)(bg % Hkv);
+        const int Lk = seqlens_k ? seqlens_k[b] : Nk;
+        double* P = (double*)malloc(nq1 * nk1 * sizeof(double));
+        double* dS = (double*)malloc(nq1 * nk1 * sizeof(double));
+        csum_t* dk_acc = (csum_t*)calloc(nk1 * (size_t)d, sizeof(csum_t));
+        csum_t* dv_acc = (csum_t*)calloc(nk1 * (size_t)d, sizeof(csum_t));
+        if (!P || !dS || !dk_acc || !dv_acc) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+            const long kv_stride = (long)Hkv * d;
+            const double* kb = k + ((size_t)b * Nk * Hkv + g) * (size_t)d;
+            const double* vb = v + ((size_t)b * Nk * Hkv + g) * (size_t)d;
+            for (int hh = 0; hh < G; ++hh) {
+                const int h = g * G + hh;
+                for (int i = 0; i < Nq; ++i) {
+                    const double* qi = q + (((size_t)b * Nq + i) * Hq + h) * (size_t)d;
+                    const double* doi = dout + (((size_t)b * Nq + i) * Hq + h) * (size_t)d;
+                    double* Prow = P + (size_t)i * nk1;
+                    double* dSrow = dS + (size_t)i * nk1;
+                    /* P row: scores, mask, softmax */
+                    double m = -INFINITY;
+                    for (int j = 0; j < Lk; ++j) {
+                        const int visible = causal ? (j <= i + (Lk - Nq)) : 1;
+                        if (!visible) {
+                            Prow[j] = -INFINITY;
+                            continue;
+                        }
+                        const double* kj = kb + (size_t)j * (size_t)kv_stride;
+                        csum_t dot = {0.0, 0.0};
+                        for (int t = 0; t < d; ++t) csum_add(&dot, qi[t] * kj[t]);
+                        Prow[j] = scale * csum_value(&dot);
+                        if (Prow[j] > m) m = Prow[j];
+                    }
+                    if (m == -INFINITY) {
+                        for (int j = 0; j < Lk; ++j) Prow[j] = 0.0, dSrow[j] = 0.0;
+                        continue;
+                    }
+                    csum_t l = {0.0, 0.0};
+                    for (int j = 0; j < Lk; ++j) {
+                        Prow[j] = (Prow[j] == -INFINITY) ? 0.0 : exp(Prow[j] - m);
+                        csum_add(&l, Prow[j]);
+                    }
+                    const double lsum = csum_value(&l);
+                    for (int j = 0; j < Lk; ++j) Prow[j] /= lsum;
+                    /* dP row and the softmax Jacobian */
+                    csum_t pdp = {0.0, 0.0};
+                    for (int j = 0; j < Lk; ++j) {
+                        if (Prow[j] == 0.0) {
+                            dSrow[j] = 0.0;
+                            continue;
+                        }
+                        const double* vj = vb + (size_t)j * (size_t)kv_stride;
+                        csum_t dot = {0.0, 0.0};
+                        for (int t = 0; t < d; ++t) csum_add(&dot, doi[t] * vj[t]);
+                        dSrow[j] = csum_value(&dot); /* dP for now */
+                        csum_add(&pdp, Prow[j] * dSrow[j]);
+                    }
+                    const double Di = csum_value(&pdp);
+                    for (int j = 0; j < Lk; ++j)
+                        if (Prow[j] != 0.0) dSrow[j] = Prow[j] * (dSrow[j] - Di);
+                    /* dQ row */
+                    double* dqi = dq + (((size_t)b * Nq + i) * Hq + h) * (size_t)d;
+                    for (int t = 0; t < d; ++t) {
+                        csum_t acc = {0.0, 0.0};
+                        for (int j = 0; j < Lk; ++j)
+                            if (dSrow[j] != 0.0)
+                                csum_add(&acc, dSrow[j] * kb[(size_t)j * (size_t)kv_stride + t]);
+                        dqi[t] = scale * csum_value(&acc);
+                    }
+                    /* this row's contributions to dK and dV */
+                    for (int j = 0; j < Lk; ++j) {
+                        if (Prow[j] == 0.0) continue;
+                        for (int t = 0; t < d; ++t) {
+                            csum_add(&dv_acc[(size_t)j * d + t], Prow[j] * doi[t]);
+                            csum_add(&dk_acc[(size_t)j * d + t], dSrow[j] * qi[t]);
+                        }
+                    }
+                }
+                /* rows of dq for queries are complete for this head */
+            }
+            for (int j = 0; j < Nk; ++j) {
+                double* dkj = dk + (((size_t)b * Nk + j) * Hkv + g) * (size_t)d;
+                double* dvj = dv + (((size_t)b * Nk + j) * Hkv + g) * (size_t)d;
+                for (int t = 0; t < d; ++t) {
+                    if (j < Lk) {
+                        dkj[t] = scale * csum_value(&dk_acc[(size_t)j * d + t]);
+                        dvj[t] = csum_value(&dv_acc[(size_t)j * d + t]);
+                    } else { /* keys behind the real length get no gradient */
+                        dkj[t] = 0.0;
+                        dvj[t] = 0.0;
+                    }
+                }
+            }
+        }
+        free(P);
+        free(dS);
+        free(dk_acc);
+        free(dv_acc);
+    }
+    return err ? -2 : 0;
+}
