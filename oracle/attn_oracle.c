@@ -388,8 +388,10 @@ int oracle_attn_bwd(const double* q, const double* k, const double* v, const dou
                         Prow[j] = scale * csum_value(&dot);
                         if (Prow[j] > m) m = Prow[j];
                     }
-                    if (m == -INFINITY) {
+                    if (m == -INFINITY) { /* no visible key: O = 0 whatever q is */
                         for (int j = 0; j < Lk; ++j) Prow[j] = 0.0, dSrow[j] = 0.0;
+                        double* dq0 = dq + (((size_t)b * Nq + i) * Hq + h) * (size_t)d;
+                        for (int t = 0; t < d; ++t) dq0[t] = 0.0;
                         continue;
                     }
                     csum_t l = {0.0, 0.0};

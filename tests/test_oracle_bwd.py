@@ -28,10 +28,11 @@ def _loss(q, k, v, do, scale, causal, seqlens):
 
 
 @pytest.mark.parametrize("causal,seqlens", [(False, None), (True, None), (False, [4]),
-                                            (True, [6])])
+                                            (True, [6]), (True, [3])])
 def test_central_differences_of_the_forward_oracle(causal, seqlens):
     # every element of dq, dk, dv against (L(x + e) - L(x - e)) / 2e computed
-    # with the forward oracle only; Nq != Nk exercises the bottom-right rule
+    # with the forward oracle only; Nq != Nk exercises the bottom-right rule,
+    # and causal with 3 keys for 5 queries leaves rows 0 and 1 with no key
     q, k, v, do = _inputs(1, 5, 6, 2, 1, 3, seed=1)
     scale = 0.7
     dq, dk, dv = oracle.attn_bwd(q, k, v, do, scale, causal, seqlens_k=seqlens)
@@ -80,9 +81,10 @@ def _torch_reference(q, k, v, do, scale, causal, seqlens):
 
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("hq,hkv", [(4, 4), (4, 2), (6, 1)])
-def test_matches_torch_autograd_fp64(causal, hq, hkv):
+@pytest.mark.parametrize("seqlens", [[50, 41], [50, 20]])
+def test_matches_torch_autograd_fp64(causal, hq, hkv, seqlens):
+    # with 20 keys for 37 causal queries, rows 0..16 of batch 1 see no key
     q, k, v, do = _inputs(2, 37, 50, hq, hkv, 16, seed=2)
-    seqlens = [50, 41]
     got = oracle.attn_bwd(q, k, v, do, 0.25, causal, seqlens_k=seqlens)
     ref = _torch_reference(q, k, v, do, 0.25, causal, seqlens)
     for name, a, r in zip(("dq", "dk", "dv"), got, ref):
