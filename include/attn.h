@@ -115,20 +115,59 @@ ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int 
  *                j <= i + seqlens_k[b] - Nq
  *   workspace    device buffer of at least attn_decode_workspace_bytes(...)
  *                bytes (256-byte aligned), owned by the caller; holds the
- *                split-K partial results and their counters.  Calls that
- *                share one workspace must not overlap on the GPU.
- *   split_keys   keys per split (multiple of 64) or 0 for automatic.
- * Each (sequence, kv head, split) work unit streams its keys once with
- * 128-bit loads, scores the Hq/Hkv query heads that share the kv head, and
- * keeps a running max and sum; the last unit of a (sequence, kv head) merges
- * the partial results in a fixed order: LSE = log sum_i exp(LSE_i),
- * O = sum_i exp(LSE_i - LSE) O_i.
+ *                work schedule, split-K partial results and counters.  Calls
+ *                that share one workspace must not overlap on the GPU.
+ *   split_keys   0 for automatic, else a multiple of 64: keys per split (or,
+ *                on the tensor-core path, per schedule range).
+ * The Nq tokens x Hq/Hkv query heads that share a kv head are scored together
+ * in one pass over its filled cache rows, with a running max and sum.  When
+ * Hq/Hkv divides 128, Nq * Hq/Hkv <= 128 and split_keys is 0 or a multiple of
+ * 128, the rows form one tcgen05 tile and the work of all sequences is cut
+ * into equal ranges, one per SM (a plan kernel, the decode kernel and a merge
+ * kernel); otherwise one CTA per (sequence, kv head, split, 16 rows) on
+ * mma.sync.  Pieces of a split sequence are merged in key order:
+ * LSE = log sum_i exp(LSE_i), O = sum_i exp(LSE_i - LSE) O_i.
  */
 ATTN_API int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_cache,
                             const int* cu_seqlens_k, const int* seqlens_k, int max_seqlen_k,
                             int cache_slots, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int d,
                             float scale, int causal, int dtype, void* workspace,
                             size_t workspace_bytes, int split_keys, void* stream);
+
+/*
+ * Bytes of device workspace that attn_bwd needs for these sizes: two float32
+ * arrays of B * Hq * Nq (per query row, the dot product of dO and O, and the
+ * forward's LSE in base 2), each 256-byte aligned.  Returns 0 for invalid
+ * sizes.
+ */
+ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq);
+
+/*
+ * Gradients of attention (the training backward pass) for
+ * L = sum(dout * O), O = attn_fwd[_kpad](q, k, v) with the same scale, causal
+ * flag and key lengths.  The pages report the method's training speed-ups
+ * (effectstory.com article, "訓練性能量化提升" table) without its backward
+ * algorithm; this recomputes every score tile on chip from q, k and the
+ * forward's lse, as the forward does, and never writes an N x N matrix.
+ *   q, o, dout, dq  [B, Nq, Hq, d]      k, v, dk, dv  [B, Nk, Hkv, d]
+ *   (all in dtype; o and lse are the forward's outputs, lse [B, Hq, Nq]
+ *   float32, -inf for a row with no visible key)
+ *   dk, dv are summed over the Hq/Hkv query heads that share a kv head; rows
+ *   of keys at or beyond seqlens_k[b] (NULL = Nk) are written as zero and
+ *   the K/V rows there may hold anything, NaN included.
+ *   workspace: at least attn_bwd_workspace_bytes(B, Hq, Nq) bytes, 256-byte
+ *   aligned, owned by the caller; calls sharing it must not overlap.
+ * Kernels, in order on `stream`: the per-row dot products, one CTA per
+ * 128-key tile of a kv head accumulating dK and dV in tensor memory over all
+ * query tiles of its group, one CTA per 128-row query tile accumulating dQ.
+ * No atomics: the result does not depend on scheduling.
+ * Returns the status codes of attn_fwd, or ATTN_ERR_WORKSPACE.
+ */
+ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                      const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                      int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype,
+                      const int* seqlens_k, void* workspace, size_t workspace_bytes,
+                      void* stream);
 
 /* Size in bytes of the scratch area built into the library for
  * attn_fwd_varlen_kvcache_noalloc (32 MiB). */

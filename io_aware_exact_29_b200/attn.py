@@ -21,7 +21,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "attn.h")
 ATTN_BF16, ATTN_FP16 = 0, 1
 STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "CUDA error",
           -4: "workspace", -5: "timeout"}
-ERR_FWD_BASE, ERR_DECODE_BASE = 16, 32
+ERR_FWD_BASE, ERR_DECODE_BASE, ERR_BWD_BASE = 16, 32, 48
 
 _lock = threading.Lock()
 _lib = None
@@ -52,6 +52,11 @@ def load_library():
             lib.attn_fwd_varlen_kvcache.argtypes = [vp, vp, vp, vp, vp, i, i, vp, vp, i, i, i, i,
                                                     i, f, i, i, vp, sz, i, vp]
             lib.attn_fwd_varlen_kvcache.restype = i
+            lib.attn_bwd_workspace_bytes.argtypes = [i, i, i]
+            lib.attn_bwd_workspace_bytes.restype = sz
+            lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i,
+                                     i, vp, vp, sz, vp]
+            lib.attn_bwd.restype = i
             lib.attn_status_string.argtypes = [i]
             lib.attn_status_string.restype = ctypes.c_char_p
             lib.attn_get_device_error.argtypes = [ctypes.POINTER(i), vp]
@@ -127,6 +132,45 @@ def attn_fwd(q, k, v, scale=None, causal=False, seqlens_k=None, out=None, lse=No
                                int(bool(causal)), _dtype_code(q), seqlens_k.data_ptr(), st)
         _check("attn_fwd_kpad", rc)
     return out, lse
+
+
+def bwd_workspace_bytes(B, Hq, Nq) -> int:
+    return int(load_library().attn_bwd_workspace_bytes(B, Hq, Nq))
+
+
+def attn_bwd(q, k, v, o, lse, dout, scale=None, causal=False, seqlens_k=None, workspace=None,
+             dq=None, dk=None, dv=None, stream=None):
+    """Gradients of L = sum(dout * O) for O = attn_fwd(q, k, v, ...).
+
+    o and lse are the forward's outputs for the same arguments.  Returns
+    (dq [B, Nq, Hq, d], dk, dv [B, Nk, Hkv, d]) in the input dtype; dk and dv
+    are summed over the query heads that share a kv head.
+    """
+    lib = load_library()
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (lse, "lse"), (dout, "dout")):
+        _dev(t, n)
+    if scale is None:
+        scale = float(d) ** -0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_bytes(B, Hq, Nq), dtype=torch.uint8,
+                                device=q.device)
+    sl = 0
+    if seqlens_k is not None:
+        _dev(seqlens_k, "seqlens_k")
+        if seqlens_k.dtype != torch.int32:
+            raise TypeError("seqlens_k must be int32")
+        sl = seqlens_k.data_ptr()
+    rc = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                      dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv,
+                      Nq, Nk, d, float(scale), int(bool(causal)), _dtype_code(q), sl or None,
+                      workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    _check("attn_bwd", rc)
+    return dq, dk, dv
 
 
 def decode_workspace_bytes(B, Hq, Hkv, Nq, d, max_seqlen_k, split_keys=0) -> int:

@@ -297,6 +297,74 @@ int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_ca
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq) {
+    if (B <= 0 || Hq <= 0 || Nq <= 0) return 0;
+    const size_t one = (((size_t)B * Hq * Nq * 4) + 255) & ~(size_t)255;
+    return 2 * one;
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+             int Nk, int d, float scale, int causal, int dtype, const int* seqlens_k,
+             void* workspace, size_t workspace_bytes, void* stream) {
+    if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk < 0 || Hq % Hkv != 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (B > 65535 || Hq > 65535) return ATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    if (!q || !o || !lse || !dout || !dq || !aligned16(q) || !aligned16(o) || !aligned16(lse) ||
+        !aligned16(dout) || !aligned16(dq))
+        return ATTN_ERR_INVALID_ARG;
+    if (Nk > 0 && (!k || !v || !dk || !dv || !aligned16(k) || !aligned16(v) || !aligned16(dk) ||
+                   !aligned16(dv)))
+        return ATTN_ERR_INVALID_ARG;
+    if (seqlens_k && (reinterpret_cast<uintptr_t>(seqlens_k) & 3u)) return ATTN_ERR_INVALID_ARG;
+    const size_t need = attn_bwd_workspace_bytes(B, Hq, Nq);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return ATTN_ERR_WORKSPACE;
+    int dev = 0;
+    const int st = check_device(&dev);
+    if (st == 0) return ATTN_ERR_CUDA;
+    if (st < 0) return ATTN_ERR_UNSUPPORTED;
+
+    BwdMaps maps;
+    // with no keys the K/V maps are never read; point them at Q
+    const void* kb = Nk > 0 ? k : q;
+    const void* vb = Nk > 0 ? v : q;
+    const int nk_map = Nk > 0 ? Nk : Nq;
+    const int hkv_map = Nk > 0 ? Hkv : Hq;
+    if (!map_bnhd(&maps.q, dtype, q, B, Nq, Hq, d) ||
+        !map_bnhd(&maps.k, dtype, kb, B, nk_map, hkv_map, d) ||
+        !map_bnhd(&maps.v, dtype, vb, B, nk_map, hkv_map, d) ||
+        !map_bnhd(&maps.dout, dtype, dout, B, Nq, Hq, d))
+        return ATTN_ERR_INVALID_ARG;
+
+    BwdParams p{};
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.G = Hq / Hkv;
+    p.causal = causal ? 1 : 0;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.seqlens_k = Nk > 0 ? seqlens_k : nullptr;
+    p.o = o;
+    p.dout = dout;
+    p.lse = lse;
+    p.lse2 = static_cast<float*>(workspace);
+    p.dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + need / 2);
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.limit_ns = kDefaultLimitNs;
+    p.err = g_err_addr[dev];
+    cudaError_t e = launch_bwd(maps, p, d, dtype == ATTN_BF16, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 const char* attn_status_string(int status) {
     switch (status) {
         case ATTN_OK: return "ok";

@@ -12,6 +12,7 @@ namespace attn {
 enum : unsigned {
     kErrFwdBase = 1 * 16,
     kErrDecodeBase = 2 * 16,
+    kErrBwdBase = 3 * 16,
 };
 
 struct FwdParams {
@@ -33,6 +34,33 @@ struct FwdMaps {
 
 // Launch the forward kernel for head dim d (64/128) and element type.
 cudaError_t launch_fwd(const FwdMaps& maps, const FwdParams& p, int d, bool bf16,
+                       cudaStream_t stream);
+
+struct BwdParams {
+    int B, Hq, Hkv, Nq, Nk;
+    int G;                 // Hq / Hkv
+    int causal;
+    float scale;
+    float scale_log2;      // scale * log2(e)
+    const int* seqlens_k;  // [B] or nullptr
+    const void* o;         // [B, Nq, Hq, d] forward output
+    const void* dout;      // [B, Nq, Hq, d]
+    const float* lse;      // [B, Hq, Nq] forward log-sum-exp (natural log)
+    float* lse2;           // workspace [B, Hq, Nq]: LSE * log2(e), +inf for empty rows
+    float* dsum;           // workspace [B, Hq, Nq]: sum_t dO * O
+    void* dq;              // [B, Nq, Hq, d]
+    void* dk;              // [B, Nk, Hkv, d]
+    void* dv;              // [B, Nk, Hkv, d]
+    unsigned long long limit_ns;
+    unsigned* err;
+};
+
+struct BwdMaps {
+    CUtensorMap q, k, v, dout;  // [B, N, H, d], box 64 columns x 1 head x 128 rows
+};
+
+// D and LSE * log2 e, then the dK/dV and dQ kernels, on `stream`.
+cudaError_t launch_bwd(const BwdMaps& maps, const BwdParams& p, int d, bool bf16,
                        cudaStream_t stream);
 
 struct DecodeParams {

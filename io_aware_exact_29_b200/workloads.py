@@ -104,6 +104,14 @@ def fwd_inputs(case: FwdCase, seed: int = 0, device: str = "cpu"):
     return dict(q=q, k=k, v=v, seqlens_k=seqlens)
 
 
+def upstream_grad(like: torch.Tensor, seed: int = 0, device: str = "cpu") -> torch.Tensor:
+    """dO for the backward pass: N(0, 1) values of q's shape and dtype, from
+    its own generator (seed + 1_000_003) so that the forward's inputs are the
+    same with or without it."""
+    g = torch.Generator(device=device).manual_seed(seed + 1_000_003)
+    return torch.randn(tuple(like.shape), generator=g, device=device).to(like.dtype)
+
+
 def kvcache_inputs(case: DecodeCase, seed: int = 0, device: str = "cpu",
                    slack_fill: float | None = None, seqlens=None):
     """Packed variable-length KV cache.
