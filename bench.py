@@ -40,7 +40,7 @@ if ROOT not in sys.path:
 
 from io_aware_exact_29_b200 import accounting  # noqa: E402
 from io_aware_exact_29_b200.workloads import (DECODE_CASES, FWD_CASES, fwd_inputs,  # noqa: E402
-                                              kvcache_inputs)
+                                              kvcache_inputs, upstream_grad)
 
 FWD_CASE = FWD_CASES["sweep_d128_n4096"]
 DEC_CASE = DECODE_CASES["llama70b_decode"]
@@ -489,7 +489,16 @@ def run_profile_case(kernel: str, launches: int):
     from io_aware_exact_29_b200.workloads import DecodeCase
 
     dev = torch.device("cuda", 0)
-    if kernel == "fwd":
+    if kernel == "bwd":
+        # backward of the bench's forward shape (inputs and gradients ~0.5 GB)
+        fc = FWD_CASE
+        fin = fwd_inputs(fc, seed=0, device="cuda")
+        o, lse = attn.attn_fwd(fin["q"], fin["k"], fin["v"], scale=fc.scale, causal=fc.causal)
+        dout = upstream_grad(fin["q"], seed=0, device="cuda")
+        for _ in range(2 + launches):
+            attn.attn_bwd(fin["q"], fin["k"], fin["v"], o, lse, dout, scale=fc.scale,
+                          causal=fc.causal)
+    elif kernel == "fwd":
         fc = FWD_CASE
         fin = fwd_inputs(fc, seed=0, device="cuda")
         for _ in range(2 + launches):
@@ -582,7 +591,7 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=32)
-    ap.add_argument("--profile", choices=["fwd", "decode", "decode_chunk16"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "bwd", "decode", "decode_chunk16"], default=None,
                     help="run a small case of one kernel for an ncu capture and exit")
     ap.add_argument("--profile-launches", type=int, default=3)
     ap.add_argument("--sweep", action="store_true",

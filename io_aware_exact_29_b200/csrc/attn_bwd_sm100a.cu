@@ -46,8 +46,11 @@ namespace attn {
 namespace {
 
 constexpr int kBlock = 128;  // rows of a Q tile and of a K/V tile
-constexpr int kThreads = 192;  // warps 0-3 compute, 4 loader, 5 MMA
-constexpr int kLoaderWarp = 4, kMmaWarp = 5;
+// warps 0-15 compute: rows 32*(w%4) .. +31 (their TMEM lanes), columns
+// 32*(w/4) .. +31 of the 128-column score tile; warp 16 loader, warp 17 MMA
+constexpr int kComputeWarps = 16;
+constexpr int kThreads = 32 * (kComputeWarps + 2);
+constexpr int kLoaderWarp = kComputeWarps, kMmaWarp = kComputeWarps + 1;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -75,26 +78,28 @@ __device__ __forceinline__ void store_row(void* out, size_t elem, const uint32_t
             ptx::pack2<BF16>(__uint_as_float(v[e + 6]) * sc, __uint_as_float(v[e + 7]) * sc));
 }
 
-// A row of D columns of tensor memory (32 at a time) to the output, scaled.
-// `zero` (the same for the whole warp) writes zeros without touching tensor
-// memory; `store` is this lane's own predicate.  The tensor-memory loads are
+// kPart columns of a row of tensor memory to the output, scaled.  `zero`
+// (the same for the whole warp) writes zeros without touching tensor memory;
+// `store` is this lane's own predicate.  The tensor-memory loads are
 // warp-collective, so every lane runs them and only the stores are
 // predicated.
-template <int D, bool BF16>
+template <int kPart, bool BF16>
 __device__ __forceinline__ void tmem_row_out(uint32_t taddr, void* out, size_t elem, float sc,
                                              bool zero, bool store) {
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        if (!zero) {
-            ptx::tmem_ld32(taddr + c * 32, r);
+    uint32_t r[kPart];
+    if (!zero) {
+        if constexpr (kPart == 32) {
+            ptx::tmem_ld32(taddr, r);
             ptx::tmem_wait_ld_dep(r);
         } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = 0u;
+            ptx::tmem_ld16(taddr, r);
+            ptx::tmem_wait_ld_dep16(r);
         }
-        if (store) store_row<32, BF16>(out, elem + c * 32, r, sc);
+    } else {
+#pragma unroll
+        for (int e = 0; e < kPart; ++e) r[e] = 0u;
     }
+    if (store) store_row<kPart, BF16>(out, elem, r, sc);
 }
 
 // ------------------------------------------------------------------ D, LSE
@@ -213,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&bars->q_empty[s], 1);
         }
         ptx::mbar_init(&bars->s_full, 1);
-        ptx::mbar_init(&bars->p_full, 4);
+        ptx::mbar_init(&bars->p_full, kComputeWarps);
         ptx::mbar_init(&bars->o_done, 1);
         ptx::mbar_init(&bars->drain, 1);
         bars->abort = 0;
@@ -334,8 +339,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < kBlock / 16; ++kk) {
                         const uint64_t r16 = (uint64_t)((kk * 16 * 128) >> 4);
                         const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-                        ptx::umma_ts_elect(tmem + kColDV, tmem + kk * 8, do_mn + r16, kIdescO, acc);
-                        ptx::umma_ts_elect(tmem + kColDK, tmem + kColDP + kk * 8, q_mn + r16,
+                        // queries 16kk..16kk+15 of P and dS: part kk/2 keeps its
+                        // 32 columns packed in the first 16 of its own 32
+                        const uint32_t a_col = (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1));
+                        ptx::umma_ts_elect(tmem + kColDV, tmem + a_col, do_mn + r16, kIdescO, acc);
+                        ptx::umma_ts_elect(tmem + kColDK, tmem + kColDP + a_col, q_mn + r16,
                                            kIdescO, acc);
                     }
                     ptx::umma_commit_elect(&bars->q_empty[st]);
@@ -353,11 +361,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ================================================= compute warps
-        const uint32_t row = (uint32_t)(warp * 32 + lane);  // key row of the tile
+        constexpr int kPartD = D / 4;
+        const uint32_t quarter = (uint32_t)(warp & 3);
+        const int part = warp >> 2;                   // query columns 32*part .. +31
+        const uint32_t row = quarter * 32u + (uint32_t)lane;  // key row of the tile
         const int kr = k0 + (int)row;
-        const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
-        const uint32_t t_s = tmem + lane_addr;
-        const uint32_t t_dp = tmem + lane_addr + kColDP;
+        const uint32_t lane_addr = (quarter * 32u) << 16;
+        const uint32_t t_s = tmem + lane_addr + (uint32_t)(32 * part);
+        const uint32_t t_dp = tmem + lane_addr + kColDP + (uint32_t)(32 * part);
         const float sl2 = p.scale_log2;
         const bool key_ok = kr < Lk;
         bool ok = true;
@@ -370,41 +381,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             ptx::tc_fence_after();
-            const float* lse_s = reinterpret_cast<const float*>(smem + L::kLse) + st * 128;
-            const float* ds_s = reinterpret_cast<const float*>(smem + L::kDs) + st * 128;
-            // every (key, query) pair of this thread's row visible?
-            const bool full = key_ok && i0 + kBlock <= p.Nq && (!p.causal || kr <= i0 + off);
+            const int qc0 = 32 * part;
+            const float* lse_s = reinterpret_cast<const float*>(smem + L::kLse) + st * 128 + qc0;
+            const float* ds_s = reinterpret_cast<const float*>(smem + L::kDs) + st * 128 + qc0;
+            uint32_t sv[32], dv[32];
+            ptx::tmem_ld32(t_s, sv);
+            ptx::tmem_ld32(t_dp, dv);
+            // every (key, query) pair of this thread's 32 columns visible?
+            const bool full = key_ok && i0 + qc0 + 32 <= p.Nq && (!p.causal || kr <= i0 + qc0 + off);
             const bool masked = __any_sync(0xffffffffu, !full);
+            ptx::tmem_wait_ld_dep(sv);
+            ptx::tmem_wait_ld_dep(dv);
+            uint32_t pk_p[16], pk_ds[16];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sv[32], dv[32];
-                ptx::tmem_ld32(t_s + c * 32, sv);
-                ptx::tmem_ld32(t_dp + c * 32, dv);
-                ptx::tmem_wait_ld_dep(sv);
-                ptx::tmem_wait_ld_dep(dv);
-                uint32_t pk_p[16], pk_ds[16];
+            for (int e = 0; e < 32; e += 2) {
+                float pr[2], dsr[2];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int qc = c * 32 + e;
-                    float pr[2], dsr[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        bool vis = true;
-                        if (masked) {
-                            const int qi = i0 + qc + u;
-                            vis = key_ok && qi < p.Nq && (!p.causal || kr <= qi + off);
-                        }
-                        const float pv =
-                            ptx::ex2_approx(__uint_as_float(sv[e + u]) * sl2 - lse_s[qc + u]);
-                        pr[u] = vis ? pv : 0.f;
-                        dsr[u] = vis ? pv * (__uint_as_float(dv[e + u]) - ds_s[qc + u]) : 0.f;
+                for (int u = 0; u < 2; ++u) {
+                    bool vis = true;
+                    if (masked) {
+                        const int qi = i0 + qc0 + e + u;
+                        vis = key_ok && qi < p.Nq && (!p.causal || kr <= qi + off);
                     }
-                    pk_p[e / 2] = ptx::pack2<BF16>(pr[0], pr[1]);
-                    pk_ds[e / 2] = ptx::pack2<BF16>(dsr[0], dsr[1]);
+                    const float pv = ptx::ex2_approx(__uint_as_float(sv[e + u]) * sl2 - lse_s[e + u]);
+                    pr[u] = vis ? pv : 0.f;
+                    dsr[u] = vis ? pv * (__uint_as_float(dv[e + u]) - ds_s[e + u]) : 0.f;
                 }
-                ptx::tmem_st16(t_s + c * 16, pk_p);
-                ptx::tmem_st16(t_dp + c * 16, pk_ds);
+                pk_p[e / 2] = ptx::pack2<BF16>(pr[0], pr[1]);
+                pk_ds[e / 2] = ptx::pack2<BF16>(dsr[0], dsr[1]);
             }
+            // P and dS of these 32 queries go to the first 16 of this warp's
+            // own 32 columns (no other warp reads them as scores)
+            ptx::tmem_st16(t_s, pk_p);
+            ptx::tmem_st16(t_dp, pk_ds);
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
@@ -417,13 +426,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ptx::tc_fence_after();
         }
-        // dV, dK of this key row (zero behind the real length or on an error)
+        // dV, dK of this key row, columns part * D/4 .. +D/4 (zero behind the
+        // real length or on an error)
         {
             const bool store = kr < p.Nk;
-            const size_t elem = (((size_t)b * p.Nk + (store ? kr : 0)) * p.Hkv + g) * D;
+            const size_t elem =
+                (((size_t)b * p.Nk + (store ? kr : 0)) * p.Hkv + g) * D + part * kPartD;
             const bool zero = !(__all_sync(0xffffffffu, ok) && nsteps > 0);
-            tmem_row_out<D, BF16>(tmem + lane_addr + kColDV, p.dv, elem, 1.f, zero, store);
-            tmem_row_out<D, BF16>(tmem + lane_addr + kColDK, p.dk, elem, p.scale, zero, store);
+            const uint32_t col = (uint32_t)(part * kPartD);
+            tmem_row_out<kPartD, BF16>(tmem + lane_addr + kColDV + col, p.dv, elem, 1.f, zero,
+                                       store);
+            tmem_row_out<kPartD, BF16>(tmem + lane_addr + kColDK + col, p.dk, elem, p.scale, zero,
+                                       store);
         }
     }
 
@@ -515,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&bars->v_empty[s], 1);
         }
         ptx::mbar_init(&bars->s_full, 1);
-        ptx::mbar_init(&bars->p_full, 4);
+        ptx::mbar_init(&bars->p_full, kComputeWarps);
         ptx::mbar_init(&bars->o_done, 1);
         ptx::mbar_init(&bars->drain, 1);
         bars->abort = 0;
@@ -631,7 +645,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ptx::sdesc_sw128(sbase + L::kK + st * kTile, kBlockBytes, 1024);
 #pragma unroll
                     for (int kk = 0; kk < kBlock / 16; ++kk)
-                        ptx::umma_ts_elect(tmem + kColDQ, tmem + kk * 8,
+                        ptx::umma_ts_elect(tmem + kColDQ,
+                                           tmem + (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1)),
                                            k_mn + (uint64_t)((kk * 16 * 128) >> 4), kIdescO,
                                            (j > 0 || kk > 0) ? 1u : 0u);
                     ptx::umma_commit_elect(&bars->k_empty[st]);
@@ -649,11 +664,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ================================================= compute warps
-        const uint32_t row = (uint32_t)(warp * 32 + lane);  // query row of the tile
+        constexpr int kPartD = D / 4;
+        const uint32_t quarter = (uint32_t)(warp & 3);
+        const int part = warp >> 2;                   // key columns 32*part .. +31
+        const uint32_t row = quarter * 32u + (uint32_t)lane;  // query row of the tile
         const int qi = i0 + (int)row;
-        const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
-        const uint32_t t_s = tmem + lane_addr;
-        const uint32_t t_dp = tmem + lane_addr + kColDP;
+        const uint32_t lane_addr = (quarter * 32u) << 16;
+        const uint32_t t_s = tmem + lane_addr + (uint32_t)(32 * part);
+        const uint32_t t_dp = tmem + lane_addr + kColDP + (uint32_t)(32 * part);
         const float sl2 = p.scale_log2;
         const bool row_ok = qi < p.Nq;
         const size_t sidx = ((size_t)b * p.Hq + h) * p.Nq + (row_ok ? qi : 0);
@@ -662,41 +680,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
             const int st = j % KST;
-            const int k0 = j * kBlock;
+            const int kc0 = j * kBlock + 32 * part;  // first key of this warp's columns
             if (!warp_wait(&bars->s_full, j & 1, p.limit_ns, abort_flag)) {
                 record_error(p.err, kErrBwdBase + 12, &bars->abort);
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
-            const bool full = row_ok && k0 + kBlock <= Lk && (!p.causal || k0 + kBlock - 1 <= qi + off);
+            uint32_t sv[32], dv[32];
+            ptx::tmem_ld32(t_s, sv);
+            ptx::tmem_ld32(t_dp, dv);
+            const bool full = row_ok && kc0 + 32 <= Lk && (!p.causal || kc0 + 31 <= qi + off);
             const bool masked = __any_sync(0xffffffffu, !full);
+            ptx::tmem_wait_ld_dep(sv);
+            ptx::tmem_wait_ld_dep(dv);
+            uint32_t pk[16];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sv[32], dv[32];
-                ptx::tmem_ld32(t_s + c * 32, sv);
-                ptx::tmem_ld32(t_dp + c * 32, dv);
-                ptx::tmem_wait_ld_dep(sv);
-                ptx::tmem_wait_ld_dep(dv);
-                uint32_t pk[16];
+            for (int e = 0; e < 32; e += 2) {
+                float dsr[2];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float dsr[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        bool vis = true;
-                        if (masked) {
-                            const int kj = k0 + c * 32 + e + u;
-                            vis = row_ok && kj < Lk && (!p.causal || kj <= qi + off);
-                        }
-                        const float pv = ptx::ex2_approx(__uint_as_float(sv[e + u]) * sl2 - lse2);
-                        dsr[u] = vis ? pv * (__uint_as_float(dv[e + u]) - dsum) : 0.f;
+                for (int u = 0; u < 2; ++u) {
+                    bool vis = true;
+                    if (masked) {
+                        const int kj = kc0 + e + u;
+                        vis = row_ok && kj < Lk && (!p.causal || kj <= qi + off);
                     }
-                    pk[e / 2] = ptx::pack2<BF16>(dsr[0], dsr[1]);
+                    const float pv = ptx::ex2_approx(__uint_as_float(sv[e + u]) * sl2 - lse2);
+                    dsr[u] = vis ? pv * (__uint_as_float(dv[e + u]) - dsum) : 0.f;
                 }
-                ptx::tmem_st16(t_s + c * 16, pk);
+                pk[e / 2] = ptx::pack2<BF16>(dsr[0], dsr[1]);
             }
-            if (k0 + kBlock > Lk && k0 + (int)row >= Lk) {
+            ptx::tmem_st16(t_s, pk);
+            const int k0 = j * kBlock;
+            if (part == 0 && k0 + kBlock > Lk && k0 + (int)row >= Lk) {
                 // key rows behind the real length: zero them in K (the B operand
                 // of dS K), so that 0 * NaN cannot reach dQ
                 uint8_t* kt = smem + L::kK + st * kTile;
@@ -721,9 +737,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_after();
         }
         {
-            const size_t elem = (((size_t)b * p.Nq + (row_ok ? qi : 0)) * p.Hq + h) * D;
+            const size_t elem =
+                (((size_t)b * p.Nq + (row_ok ? qi : 0)) * p.Hq + h) * D + part * kPartD;
             const bool zero = !(__all_sync(0xffffffffu, ok) && nt > 0);
-            tmem_row_out<D, BF16>(tmem + lane_addr + kColDQ, p.dq, elem, p.scale, zero, row_ok);
+            tmem_row_out<kPartD, BF16>(tmem + lane_addr + kColDQ + (uint32_t)(part * kPartD),
+                                       p.dq, elem, p.scale, zero, row_ok);
         }
     }
 
