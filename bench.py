@@ -3,6 +3,7 @@
 A step is one pass of the whole path over one batch of synthetic inputs:
   forward  : B=4, H=16, N=4096, d=128, bf16, non-causal (the long-sequence
              sweep point at which the forward target is stated), then
+  backward : dQ, dK, dV of that forward for a seeded dO, then
   decode   : Llama2-70B shape, B=32, Hq=64, Hkv=8, d=128, one new token per
              sequence, packed bf16 KV cache with lengths ~ U[1, 32768], then
   decode16 : the same shape with a causal chunk of 16 new tokens per sequence
@@ -208,7 +209,14 @@ def run_ours(args, rank, world, local):
     l16 = torch.empty((c16.B, c16.Hq, c16.Nq), dtype=torch.float32, device=dev)
     ws16 = torch.empty(attn.decode_workspace_bytes(c16.B, c16.Hq, c16.Hkv, c16.Nq, c16.d, max16),
                        dtype=torch.uint8, device=dev)
+    # the backward of the same forward (training step): dO seeded, O and LSE
+    # from the step's own forward launch
+    dout = upstream_grad(q, seed=1000 * rank + 2, device=str(dev))
+    dq_b, dk_b, dv_b = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_b = torch.empty(attn.bwd_workspace_bytes(fc.B, fc.Hq, fc.Nq), dtype=torch.uint8,
+                       device=dev)
     fflops = fwd_work(fc)
+    bflops = 2.5 * fflops  # five tile products of the forward's size (S, dP, dV, dK, dQ)
     dbytes = accounting.decode_bytes(sl.tolist(), dc.B, dc.Hq, dc.Hkv, dc.Nq, dc.d)
     dbytes16 = accounting.decode_bytes(din16["seqlens_k"].tolist(), c16.B, c16.Hq, c16.Hkv,
                                        c16.Nq, c16.d)
@@ -217,6 +225,9 @@ def run_ours(args, rank, world, local):
         ev[0].record(stream)
         attn.attn_fwd(q, k, v, scale=fc.scale, causal=fc.causal, out=o, lse=lse, stream=stream)
         ev[1].record(stream)
+        attn.attn_bwd(q, k, v, o, lse, dout, scale=fc.scale, causal=fc.causal, workspace=ws_b,
+                      dq=dq_b, dk=dk_b, dv=dv_b, stream=stream)
+        ev[4].record(stream)
         attn.attn_fwd_varlen_kvcache(dq, kc, vc, cu, sl, max_len, scale=dc.scale,
                                      causal=dc.causal, workspace=ws, out=do, lse=dlse,
                                      stream=stream)
@@ -227,7 +238,7 @@ def run_ours(args, rank, world, local):
                                      lse=l16, stream=stream)
         ev[3].record(stream)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     for _ in range(args.warmup):
         step(evs[0])
     torch.cuda.synchronize()
@@ -247,10 +258,11 @@ def run_ours(args, rank, world, local):
         barrier(world)
     total_ms = t0.elapsed_time(t1)
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
-    dec_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    bwd_ms = sum(e[1].elapsed_time(e[4]) for e in evs)
+    dec_ms = sum(e[4].elapsed_time(e[2]) for e in evs)
     dec16_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
-    total_ms, fwd_ms, dec_ms, dec16_ms = reduce_max([total_ms, fwd_ms, dec_ms, dec16_ms], world,
-                                                    dev)
+    total_ms, fwd_ms, bwd_ms, dec_ms, dec16_ms = reduce_max(
+        [total_ms, fwd_ms, bwd_ms, dec_ms, dec16_ms], world, dev)
     assert attn.get_device_error() == 0
 
     # ---- end to end through the public API with host buffers
@@ -322,6 +334,18 @@ def run_ours(args, rank, world, local):
                     "unit": "GB/s", "h2d_bytes_per_step": e2e["dec_h2d"],
                     "d2h_bytes_per_step": e2e["dec_d2h"]},
         },
+        "bwd": {
+            "value": round(bflops * args.steps * world / (bwd_ms * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s",
+            "flops_per_call": bflops,
+            "flop_count": "2.5 x the forward's (S, dP, dV, dK, dQ tile products); the kernels "
+                          "recompute S and dP once more for dQ, which is not counted",
+            "ms_per_call": round(bwd_ms / args.steps, 4),
+            "frac": round(bflops / (bwd_ms / args.steps * 1e-3) / 1e12 / peak_t, 4),
+            "peak": peak_t,
+            "kernels_per_call": "attn_bwd_pre + attn_bwd_dkdv + attn_bwd_dq",
+            "bound": "tensor",
+        },
         "decode_chunk16": {
             "value": round(dbytes16 * args.steps * world / (dec16_ms * 1e-3) / 1e9, 1),
             "unit": "GB/s",
@@ -336,8 +360,9 @@ def run_ours(args, rank, world, local):
         "e2e": {"value": round(fflops * world / (e2e_fwd_ms * 1e-3) / 1e12, 2),
                 "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["fwd_h2d"],
                 "d2h_bytes_per_step": e2e["fwd_d2h"]},
-        # per step: the forward kernel, and plan + decode + merge for each decode
-        "gpu_launches": 7 * args.steps,
+        # per step: the forward kernel, the three backward kernels, and
+        # plan + decode + merge for each decode
+        "gpu_launches": 10 * args.steps,
         "clocks": clk.summary(),
         "fwd_ms_per_launch": round(per_launch_ms, 4),
     }
@@ -560,7 +585,20 @@ def run_sweep(reps: int = 20):
                           "TFLOP/s": round(tf, 1),
                           "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 3),
                           "frac_burst": round(tf / peaks["bf16_tflops"], 3)}), flush=True)
-        del fin, o, lse
+        # the backward of the same forward (five tile products counted)
+        dout = upstream_grad(fin["q"], seed=0, device="cuda")
+        ws_b = torch.empty(attn.bwd_workspace_bytes(c.B, c.Hq, c.Nq), dtype=torch.uint8, device=dev)
+        grads = (torch.empty_like(fin["q"]), torch.empty_like(fin["k"]), torch.empty_like(fin["v"]))
+        ms_b = timed(lambda: attn.attn_bwd(fin["q"], fin["k"], fin["v"], o, lse, dout, scale=c.scale,
+                                           causal=c.causal, seqlens_k=sl, workspace=ws_b,
+                                           dq=grads[0], dk=grads[1], dv=grads[2]))
+        tb = 2.5 * flops / (ms_b * 1e-3) / 1e12
+        print(json.dumps({"sweep": name, "kind": "bwd", "dtype": c.dtype, "causal": c.causal,
+                          "B": c.B, "H": c.Hq, "N": c.Nq, "d": c.d, "ms": round(ms_b, 4),
+                          "TFLOP/s": round(tb, 1),
+                          "frac_sustained": round(tb / peaks["bf16_tflops_sustained"], 3)}),
+              flush=True)
+        del fin, o, lse, dout, ws_b, grads
     for name, c in DECODE_CASES.items():
         din = kvcache_inputs(c, seed=0, device="cuda")
         ml = int(din["seqlens_k"].max().item())

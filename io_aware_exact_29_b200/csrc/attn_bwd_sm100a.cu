@@ -167,8 +167,8 @@ struct DkdvBars {
     uint64_t kv_full;
     uint64_t q_full[QST];
     uint64_t q_empty[QST];
-    uint64_t s_full;
-    uint64_t p_full;
+    uint64_t s_full[2];  // per query half
+    uint64_t p_full[2];
     uint64_t o_done;
     uint64_t drain;
     uint32_t tmem_base;
@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kTile = L::kTile;
     constexpr int kDBlocks = D / 64;
     constexpr uint32_t kBlockBytes = kBlock * 128;
-    constexpr uint32_t kIdescS = ptx::idesc_f16(kBlock, kBlock, BF16, false);
+    constexpr uint32_t kIdescS = ptx::idesc_f16(kBlock, 64, BF16, false);  // half tiles
     constexpr uint32_t kIdescO = ptx::idesc_f16(kBlock, D, BF16, true);
     constexpr uint32_t kColDP = 128, kColDV = 256, kColDK = 256 + D;
     static_assert(sizeof(DkdvBars<QST>) <= 256, "barrier block");
@@ -217,8 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&bars->q_full[s], 1);
             ptx::mbar_init(&bars->q_empty[s], 1);
         }
-        ptx::mbar_init(&bars->s_full, 1);
-        ptx::mbar_init(&bars->p_full, kComputeWarps);
+        for (int hh = 0; hh < 2; ++hh) {
+            ptx::mbar_init(&bars->s_full[hh], 1);
+            ptx::mbar_init(&bars->p_full[hh], kComputeWarps / 2);
+        }
         ptx::mbar_init(&bars->o_done, 1);
         ptx::mbar_init(&bars->drain, 1);
         bars->abort = 0;
@@ -305,48 +307,69 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t k_desc = ptx::sdesc_sw128(sbase + L::kK, 16, 1024);
             const uint64_t v_desc = ptx::sdesc_sw128(sbase + L::kV, 16, 1024);
             constexpr uint64_t kTileUnits = kTile >> 4;
-            if (wait_or_fail(&bars->kv_full, 0, 2)) {
+            constexpr uint64_t kHalfUnits = (64 * 128) >> 4;  // 64 rows into a 128-row tile
+            // S^T and dP^T of query half h (queries 64h .. 64h+63) of step s
+            auto issue_sdp = [&](int s, int h) {
+                const int st = s % QST;
+                const uint64_t q_k = ptx::sdesc_sw128(sbase + L::kQ, 16, 1024) + st * kTileUnits +
+                                     h * kHalfUnits;
+                const uint64_t do_k = ptx::sdesc_sw128(sbase + L::kDO, 16, 1024) +
+                                      st * kTileUnits + h * kHalfUnits;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t o16 = (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
+                    ptx::umma_ss_elect(tmem + 64 * h, k_desc + o16, q_k + o16, kIdescS, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t o16 = (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
+                    ptx::umma_ss_elect(tmem + kColDP + 64 * h, v_desc + o16, do_k + o16, kIdescS,
+                                       kk > 0);
+                }
+                ptx::umma_commit_elect(&bars->s_full[h]);
+            };
+            // dV += P_h^T dO_h and dK += dS_h^T Q_h (K = the 64 queries of half h)
+            auto issue_dvk = [&](int s, int h) {
+                const int st = s % QST;
+                const uint64_t q_mn = ptx::sdesc_sw128(sbase + L::kQ + st * kTile, kBlockBytes, 1024);
+                const uint64_t do_mn =
+                    ptx::sdesc_sw128(sbase + L::kDO + st * kTile, kBlockBytes, 1024);
+#pragma unroll
+                for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
+                    const uint64_t r16 = (uint64_t)((kk * 16 * 128) >> 4);
+                    const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                    // queries 16kk..16kk+15 of P and dS: part kk/2 keeps its
+                    // 32 columns packed in the first 16 of its own 32
+                    const uint32_t a_col = (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1));
+                    ptx::umma_ts_elect(tmem + kColDV, tmem + a_col, do_mn + r16, kIdescO, acc);
+                    ptx::umma_ts_elect(tmem + kColDK, tmem + kColDP + a_col, q_mn + r16, kIdescO,
+                                       acc);
+                }
+            };
+            // Order per step s: dVK_0(s), SdP_0(s+1), dVK_1(s), SdP_1(s+1): the
+            // products of one half run while the other half's warps compute.
+            if (wait_or_fail(&bars->kv_full, 0, 2) && wait_or_fail(&bars->q_full[0], 0, 3)) {
+                ptx::tc_fence_after();
+                issue_sdp(0, 0);
+                issue_sdp(0, 1);
+                __syncwarp();
+                issued = true;
                 for (int s = 0; s < nsteps; ++s) {
-                    const int st = s % QST;
-                    if (!wait_or_fail(&bars->q_full[st], (s / QST) & 1, 3)) break;
+                    if (!wait_or_fail(&bars->p_full[0], s & 1, 4)) break;
                     ptx::tc_fence_after();
-                    const uint64_t q_k = ptx::sdesc_sw128(sbase + L::kQ, 16, 1024) + st * kTileUnits;
-                    const uint64_t do_k =
-                        ptx::sdesc_sw128(sbase + L::kDO, 16, 1024) + st * kTileUnits;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t o16 =
-                            (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
-                        ptx::umma_ss_elect(tmem, k_desc + o16, q_k + o16, kIdescS, kk > 0);
+                    issue_dvk(s, 0);
+                    if (s + 1 < nsteps) {
+                        const int s1 = s + 1;
+                        if (!wait_or_fail(&bars->q_full[s1 % QST], (s1 / QST) & 1, 3)) break;
+                        ptx::tc_fence_after();
+                        issue_sdp(s1, 0);
                     }
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t o16 =
-                            (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
-                        ptx::umma_ss_elect(tmem + kColDP, v_desc + o16, do_k + o16, kIdescS,
-                                           kk > 0);
-                    }
-                    ptx::umma_commit_elect(&bars->s_full);
                     __syncwarp();
-                    issued = true;
-                    if (!wait_or_fail(&bars->p_full, s & 1, 4)) break;
+                    if (!wait_or_fail(&bars->p_full[1], s & 1, 4)) break;
                     ptx::tc_fence_after();
-                    const uint64_t q_mn =
-                        ptx::sdesc_sw128(sbase + L::kQ + st * kTile, kBlockBytes, 1024);
-                    const uint64_t do_mn =
-                        ptx::sdesc_sw128(sbase + L::kDO + st * kTile, kBlockBytes, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < kBlock / 16; ++kk) {
-                        const uint64_t r16 = (uint64_t)((kk * 16 * 128) >> 4);
-                        const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-                        // queries 16kk..16kk+15 of P and dS: part kk/2 keeps its
-                        // 32 columns packed in the first 16 of its own 32
-                        const uint32_t a_col = (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1));
-                        ptx::umma_ts_elect(tmem + kColDV, tmem + a_col, do_mn + r16, kIdescO, acc);
-                        ptx::umma_ts_elect(tmem + kColDK, tmem + kColDP + a_col, q_mn + r16,
-                                           kIdescO, acc);
-                    }
-                    ptx::umma_commit_elect(&bars->q_empty[st]);
+                    issue_dvk(s, 1);
+                    ptx::umma_commit_elect(&bars->q_empty[s % QST]);
+                    if (s + 1 < nsteps) issue_sdp(s + 1, 1);
                     if (s == nsteps - 1) ptx::umma_commit_elect(&bars->o_done);
                     __syncwarp();
                 }
@@ -364,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kPartD = D / 4;
         const uint32_t quarter = (uint32_t)(warp & 3);
         const int part = warp >> 2;                   // query columns 32*part .. +31
+        const int half = part >> 1;                   // query half of those columns
         const uint32_t row = quarter * 32u + (uint32_t)lane;  // key row of the tile
         const int kr = k0 + (int)row;
         const uint32_t lane_addr = (quarter * 32u) << 16;
@@ -375,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < nsteps; ++s) {
             const int st = s % QST;
             const int i0 = (qt_first + s % nqs) * kBlock;
-            if (!warp_wait(&bars->s_full, s & 1, p.limit_ns, abort_flag)) {
+            if (!warp_wait(&bars->s_full[half], s & 1, p.limit_ns, abort_flag)) {
                 record_error(p.err, kErrBwdBase + 5, &bars->abort);
                 ok = false;
                 break;
@@ -417,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&bars->p_full);
+            if (lane == 0) ptx::mbar_arrive(&bars->p_full[half]);
         }
         if (ok && nsteps > 0) {
             if (!warp_wait(&bars->o_done, 0, p.limit_ns, abort_flag)) {
@@ -469,8 +493,8 @@ struct DqBars {
     uint64_t k_empty[KST];
     uint64_t v_full[KST];
     uint64_t v_empty[KST];
-    uint64_t s_full;
-    uint64_t p_full;
+    uint64_t s_full[2];  // per key half
+    uint64_t p_full[2];
     uint64_t o_done;
     uint64_t drain;
     uint32_t tmem_base;
@@ -499,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kTile = L::kTile;
     constexpr int kDBlocks = D / 64;
     constexpr uint32_t kBlockBytes = kBlock * 128;
-    constexpr uint32_t kIdescS = ptx::idesc_f16(kBlock, kBlock, BF16, false);
+    constexpr uint32_t kIdescS = ptx::idesc_f16(kBlock, 64, BF16, false);  // half tiles
     constexpr uint32_t kIdescO = ptx::idesc_f16(kBlock, D, BF16, true);
     constexpr uint32_t kColDP = 128, kColDQ = 256;
     static_assert(sizeof(DqBars<KST>) <= 256, "barrier block");
@@ -528,8 +552,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&bars->v_full[s], 1);
             ptx::mbar_init(&bars->v_empty[s], 1);
         }
-        ptx::mbar_init(&bars->s_full, 1);
-        ptx::mbar_init(&bars->p_full, kComputeWarps);
+        for (int hh = 0; hh < 2; ++hh) {
+            ptx::mbar_init(&bars->s_full[hh], 1);
+            ptx::mbar_init(&bars->p_full[hh], kComputeWarps / 2);
+        }
         ptx::mbar_init(&bars->o_done, 1);
         ptx::mbar_init(&bars->drain, 1);
         bars->abort = 0;
@@ -614,42 +640,69 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t q_desc = ptx::sdesc_sw128(sbase + L::kQ, 16, 1024);
             const uint64_t do_desc = ptx::sdesc_sw128(sbase + L::kDO, 16, 1024);
             constexpr uint64_t kTileUnits = kTile >> 4;
-            if (wait_or_fail(&bars->q_full, 0, 9)) {
+            constexpr uint64_t kHalfUnits = (64 * 128) >> 4;  // 64 rows into a 128-row tile
+            // S and dP of key half h (keys 64h .. 64h+63) of key tile j
+            auto issue_sdp = [&](int j, int h) {
+                const int st = j % KST;
+                const uint64_t k_k = ptx::sdesc_sw128(sbase + L::kK, 16, 1024) + st * kTileUnits +
+                                     h * kHalfUnits;
+                const uint64_t v_k = ptx::sdesc_sw128(sbase + L::kV, 16, 1024) + st * kTileUnits +
+                                     h * kHalfUnits;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t o16 = (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
+                    ptx::umma_ss_elect(tmem + 64 * h, q_desc + o16, k_k + o16, kIdescS, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t o16 = (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
+                    ptx::umma_ss_elect(tmem + kColDP + 64 * h, do_desc + o16, v_k + o16, kIdescS,
+                                       kk > 0);
+                }
+                ptx::umma_commit_elect(&bars->s_full[h]);
+            };
+            // dQ += dS_h K_h (K = the 64 keys of half h)
+            auto issue_dq = [&](int j, int h) {
+                const int st = j % KST;
+                const uint64_t k_mn = ptx::sdesc_sw128(sbase + L::kK + st * kTile, kBlockBytes, 1024);
+#pragma unroll
+                for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
+                    ptx::umma_ts_elect(tmem + kColDQ,
+                                       tmem + (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1)),
+                                       k_mn + (uint64_t)((kk * 16 * 128) >> 4), kIdescO,
+                                       (j > 0 || kk > 0) ? 1u : 0u);
+            };
+            auto wait_kv = [&](int j) {
+                const int st = j % KST;
+                return wait_or_fail(&bars->k_full[st], (j / KST) & 1, 10) &&
+                       wait_or_fail(&bars->v_full[st], (j / KST) & 1, 10);
+            };
+            // Order per key tile j: dQ_0(j), SdP_0(j+1), dQ_1(j), SdP_1(j+1).
+            if (wait_or_fail(&bars->q_full, 0, 9) && wait_kv(0)) {
+                ptx::tc_fence_after();
+                issue_sdp(0, 0);
+                issue_sdp(0, 1);
+                ptx::umma_commit_elect(&bars->v_empty[0]);
+                __syncwarp();
+                issued = true;
                 for (int j = 0; j < nt; ++j) {
-                    const int st = j % KST;
-                    if (!wait_or_fail(&bars->k_full[st], (j / KST) & 1, 10)) break;
-                    if (!wait_or_fail(&bars->v_full[st], (j / KST) & 1, 10)) break;
+                    if (!wait_or_fail(&bars->p_full[0], j & 1, 11)) break;
                     ptx::tc_fence_after();
-                    const uint64_t k_k = ptx::sdesc_sw128(sbase + L::kK, 16, 1024) + st * kTileUnits;
-                    const uint64_t v_k = ptx::sdesc_sw128(sbase + L::kV, 16, 1024) + st * kTileUnits;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t o16 =
-                            (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
-                        ptx::umma_ss_elect(tmem, q_desc + o16, k_k + o16, kIdescS, kk > 0);
+                    issue_dq(j, 0);
+                    if (j + 1 < nt) {
+                        if (!wait_kv(j + 1)) break;
+                        ptx::tc_fence_after();
+                        issue_sdp(j + 1, 0);
                     }
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t o16 =
-                            (uint64_t)(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
-                        ptx::umma_ss_elect(tmem + kColDP, do_desc + o16, v_k + o16, kIdescS,
-                                           kk > 0);
-                    }
-                    ptx::umma_commit_elect(&bars->s_full);
-                    ptx::umma_commit_elect(&bars->v_empty[st]);
                     __syncwarp();
-                    issued = true;
-                    if (!wait_or_fail(&bars->p_full, j & 1, 11)) break;
+                    if (!wait_or_fail(&bars->p_full[1], j & 1, 11)) break;
                     ptx::tc_fence_after();
-                    const uint64_t k_mn =
-                        ptx::sdesc_sw128(sbase + L::kK + st * kTile, kBlockBytes, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < kBlock / 16; ++kk)
-                        ptx::umma_ts_elect(tmem + kColDQ,
-                                           tmem + (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1)),
-                                           k_mn + (uint64_t)((kk * 16 * 128) >> 4), kIdescO,
-                                           (j > 0 || kk > 0) ? 1u : 0u);
-                    ptx::umma_commit_elect(&bars->k_empty[st]);
+                    issue_dq(j, 1);
+                    ptx::umma_commit_elect(&bars->k_empty[j % KST]);
+                    if (j + 1 < nt) {
+                        issue_sdp(j + 1, 1);
+                        ptx::umma_commit_elect(&bars->v_empty[(j + 1) % KST]);
+                    }
                     if (j == nt - 1) ptx::umma_commit_elect(&bars->o_done);
                     __syncwarp();
                 }
@@ -667,6 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kPartD = D / 4;
         const uint32_t quarter = (uint32_t)(warp & 3);
         const int part = warp >> 2;                   // key columns 32*part .. +31
+        const int half = part >> 1;                   // key half of those columns
         const uint32_t row = quarter * 32u + (uint32_t)lane;  // query row of the tile
         const int qi = i0 + (int)row;
         const uint32_t lane_addr = (quarter * 32u) << 16;
@@ -681,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < nt; ++j) {
             const int st = j % KST;
             const int kc0 = j * kBlock + 32 * part;  // first key of this warp's columns
-            if (!warp_wait(&bars->s_full, j & 1, p.limit_ns, abort_flag)) {
+            if (!warp_wait(&bars->s_full[half], j & 1, p.limit_ns, abort_flag)) {
                 record_error(p.err, kErrBwdBase + 12, &bars->abort);
                 ok = false;
                 break;
@@ -711,23 +765,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pk[e / 2] = ptx::pack2<BF16>(dsr[0], dsr[1]);
             }
             ptx::tmem_st16(t_s, pk);
-            const int k0 = j * kBlock;
-            if (part == 0 && k0 + kBlock > Lk && k0 + (int)row >= Lk) {
-                // key rows behind the real length: zero them in K (the B operand
-                // of dS K), so that 0 * NaN cannot reach dQ
+            // key rows of this half behind the real length: zero them in K (the
+            // B operand of dS K), so that 0 * NaN cannot reach dQ; the quarter-0
+            // warps of the half take its 64 rows (its S product is complete)
+            const int krow = 64 * half + 32 * (part & 1) + lane;
+            if (quarter == 0 && j * kBlock + kBlock > Lk && j * kBlock + krow >= Lk) {
                 uint8_t* kt = smem + L::kK + st * kTile;
 #pragma unroll
                 for (int c = 0; c < kDBlocks; ++c)
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch)
-                        *reinterpret_cast<uint4*>(kt + c * kBlockBytes + row * 128 + ch * 16) =
+                        *reinterpret_cast<uint4*>(kt + c * kBlockBytes + krow * 128 + ch * 16) =
                             make_uint4(0, 0, 0, 0);
             }
             ptx::fence_proxy_async_smem();
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&bars->p_full);
+            if (lane == 0) ptx::mbar_arrive(&bars->p_full[half]);
         }
         if (ok && nt > 0) {
             if (!warp_wait(&bars->o_done, 0, p.limit_ns, abort_flag)) {
