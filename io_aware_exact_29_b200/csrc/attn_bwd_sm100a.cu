@@ -156,8 +156,8 @@ struct DkdvSmem {
     static constexpr uint32_t kV = kK + kTile;
     static constexpr uint32_t kQ = kV + kTile;             // QST stages
     static constexpr uint32_t kDO = kQ + QST * kTile;      // QST stages
-    static constexpr uint32_t kLse = kDO + QST * kTile;    // QST x 128 fp32
-    static constexpr uint32_t kDs = kLse + QST * 128 * 4;  // QST x 128 fp32
+    static constexpr uint32_t kLse = kDO + QST * kTile;    // QST x 128 fp32: -LSE * log2 e
+    static constexpr uint32_t kDs = kLse + QST * 128 * 4;  // QST x 128 fp32: -D
     static constexpr uint32_t kBars = kDs + QST * 128 * 4;
     static constexpr uint32_t kAlloc = kBars + 256 + 1024;
 };
@@ -270,8 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int i = i0 + lane * 4 + u;
-                    lse_s[lane * 4 + u] = i < p.Nq ? p.lse2[base + i] : INFINITY;
-                    ds_s[lane * 4 + u] = i < p.Nq ? p.dsum[base + i] : 0.f;
+                    // negated, so that the compute warps add them with f32x2 FMAs
+                    lse_s[lane * 4 + u] = i < p.Nq ? -p.lse2[base + i] : -INFINITY;
+                    ds_s[lane * 4 + u] = i < p.Nq ? -p.dsum[base + i] : 0.f;
                 }
                 __syncwarp();
                 if (lane == 0) {
@@ -417,22 +418,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_wait_ld_dep(sv);
             ptx::tmem_wait_ld_dep(dv);
             uint32_t pk_p[16], pk_ds[16];
+            const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-                float pr[2], dsr[2];
+            for (int e4 = 0; e4 < 32; e4 += 4) {
+                // 16-byte loads of four queries' -LSE*log2e and -D
+                const float4 nl = *reinterpret_cast<const float4*>(lse_s + e4);
+                const float4 nd = *reinterpret_cast<const float4*>(ds_s + e4);
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    bool vis = true;
+                for (int e2 = 0; e2 < 4; e2 += 2) {
+                    const int e = e4 + e2;
+                    const uint64_t nl2 = e2 == 0 ? ptx::f2_pack(nl.x, nl.y) : ptx::f2_pack(nl.z, nl.w);
+                    const uint64_t nd2 = e2 == 0 ? ptx::f2_pack(nd.x, nd.y) : ptx::f2_pack(nd.z, nd.w);
+                    float t0, t1;
+                    ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(sv[e]),
+                                                            __uint_as_float(sv[e + 1])),
+                                               sl2_2, nl2), t0, t1);
+                    float p0 = ptx::ex2_approx(t0), p1 = ptx::ex2_approx(t1);
+                    const uint64_t d2 = ptx::f2_add(
+                        ptx::f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), nd2);
+                    float ds0, ds1;
+                    ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(p0, p1), d2), ds0, ds1);
                     if (masked) {
-                        const int qi = i0 + qc0 + e + u;
-                        vis = key_ok && qi < p.Nq && (!p.causal || kr <= qi + off);
+                        const int qi = i0 + qc0 + e;
+                        const bool v0 = key_ok && qi < p.Nq && (!p.causal || kr <= qi + off);
+                        const bool v1 = key_ok && qi + 1 < p.Nq && (!p.causal || kr <= qi + 1 + off);
+                        p0 = v0 ? p0 : 0.f;
+                        ds0 = v0 ? ds0 : 0.f;
+                        p1 = v1 ? p1 : 0.f;
+                        ds1 = v1 ? ds1 : 0.f;
                     }
-                    const float pv = ptx::ex2_approx(__uint_as_float(sv[e + u]) * sl2 - lse_s[e + u]);
-                    pr[u] = vis ? pv : 0.f;
-                    dsr[u] = vis ? pv * (__uint_as_float(dv[e + u]) - ds_s[e + u]) : 0.f;
+                    pk_p[e / 2] = ptx::pack2<BF16>(p0, p1);
+                    pk_ds[e / 2] = ptx::pack2<BF16>(ds0, ds1);
                 }
-                pk_p[e / 2] = ptx::pack2<BF16>(pr[0], pr[1]);
-                pk_ds[e / 2] = ptx::pack2<BF16>(dsr[0], dsr[1]);
             }
             // P and dS of these 32 queries go to the first 16 of this warp's
             // own 32 columns (no other warp reads them as scores)
@@ -749,20 +766,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_wait_ld_dep(sv);
             ptx::tmem_wait_ld_dep(dv);
             uint32_t pk[16];
+            const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
+            const uint64_t nl2 = ptx::f2_pack(-lse2, -lse2);
+            const uint64_t nd2 = ptx::f2_pack(-dsum, -dsum);
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
-                float dsr[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    bool vis = true;
-                    if (masked) {
-                        const int kj = kc0 + e + u;
-                        vis = row_ok && kj < Lk && (!p.causal || kj <= qi + off);
-                    }
-                    const float pv = ptx::ex2_approx(__uint_as_float(sv[e + u]) * sl2 - lse2);
-                    dsr[u] = vis ? pv * (__uint_as_float(dv[e + u]) - dsum) : 0.f;
+                float t0, t1;
+                ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(sv[e]),
+                                                        __uint_as_float(sv[e + 1])),
+                                           sl2_2, nl2), t0, t1);
+                const float p0 = ptx::ex2_approx(t0), p1 = ptx::ex2_approx(t1);
+                const uint64_t d2 = ptx::f2_add(
+                    ptx::f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), nd2);
+                float ds0, ds1;
+                ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(p0, p1), d2), ds0, ds1);
+                if (masked) {
+                    const int kj = kc0 + e;
+                    const bool v0 = row_ok && kj < Lk && (!p.causal || kj <= qi + off);
+                    const bool v1 = row_ok && kj + 1 < Lk && (!p.causal || kj + 1 <= qi + off);
+                    ds0 = v0 ? ds0 : 0.f;
+                    ds1 = v1 ? ds1 : 0.f;
                 }
-                pk[e / 2] = ptx::pack2<BF16>(dsr[0], dsr[1]);
+                pk[e / 2] = ptx::pack2<BF16>(ds0, ds1);
             }
             ptx::tmem_st16(t_s, pk);
             // key rows of this half behind the real length: zero them in K (the
