@@ -45,6 +45,10 @@ constexpr int kBlockN = 128;  // keys per K/V tile
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
+// one exponential pair in FWD_POLY_EVERY(D) is evaluated on the FMA pipe
+#ifndef FWD_POLY_EVERY
+#define FWD_POLY_EVERY(D) 4
+#endif
 
 template <int D, int KST, int VST>
 struct FwdSmem {
@@ -128,8 +132,9 @@ __device__ __forceinline__ void half_max(const uint32_t (&r)[2][32], int key_bas
 }
 
 // p = 2^(s * scale_log2 - m) for 64 score columns, accumulated into four
-// pair sums and packed two per 32-bit word (bf16 or fp16).
-template <bool kMask, bool BF16>
+// pair sums and packed two per 32-bit word (bf16 or fp16).  One pair in
+// kPolyEvery goes to the FMA pipe.
+template <bool kMask, bool BF16, int kPolyEvery>
 __device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_base, int row_lim,
                                          uint64_t sl2_2, uint64_t nm_2, uint64_t (&acc2)[4],
                                          uint32_t (&pk)[32]) {
@@ -143,9 +148,10 @@ __device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_bas
         }
         const uint64_t t2 = ptx::f2_fma(ptx::f2_pack(v0, v1), sl2_2, nm_2);
         float p0, p1;
-        if (((c >> 1) & 3) == 3) {
-            // every fourth pair on the FMA pipe: the exp2 unit and the tensor
-            // pipe carry equal work at d = 128, this takes a quarter off the former
+        if (((c >> 1) % kPolyEvery) == kPolyEvery - 1) {
+            // a share of the pairs on the FMA pipe: the exp2 unit and the tensor
+            // pipe carry equal work at d = 128 (a quarter moves), the exp2 unit
+            // twice the tensor pipe's at d = 64
             ptx::f2_unpack(ptx::exp2_poly2(t2), p0, p1);
         } else {
             float t0, t1;
@@ -170,6 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kBlockBytes = kBlockM * 128;
     constexpr uint32_t kIdescS = ptx::idesc_f16(kBlockM, kBlockN, BF16, false);
     constexpr uint32_t kIdescO = ptx::idesc_f16(kBlockM, D, BF16, true);
+    constexpr int kPolyEvery = FWD_POLY_EVERY(D);
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = ptx::smem_u32(smem_raw);
@@ -425,9 +432,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tmem_wait_ld_dep(r[1]);
                 uint32_t pk[32];
                 if (masked)
-                    half_exp<true, BF16>(r, key0 + hf * 64, row_lim, sl2_2, nm_2, acc2, pk);
+                    half_exp<true, BF16, kPolyEvery>(r, key0 + hf * 64, row_lim, sl2_2, nm_2, acc2,
+                                                     pk);
                 else
-                    half_exp<false, BF16>(r, key0 + hf * 64, row_lim, sl2_2, nm_2, acc2, pk);
+                    half_exp<false, BF16, kPolyEvery>(r, key0 + hf * 64, row_lim, sl2_2, nm_2,
+                                                      acc2, pk);
                 ptx::tmem_st32(t_s + hf * 32, pk);
             }
             float s0, s1, s2, s3, s4, s5, s6, s7;
