@@ -135,6 +135,36 @@ ATTN_API int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const v
                             size_t workspace_bytes, int split_keys, void* stream);
 
 /*
+ * The decode of attn_fwd_varlen_kvcache against a PAGED KV cache: the cache
+ * is cut into blocks of block_size rows and sequence b's logical key j lives
+ * in physical block block_table[b * max_blocks + j / block_size], row
+ * j % block_size (the pre-allocated, one-row-per-token cache of the ai6s.net
+ * article, adaptation point 3, with its rows found through a table).
+ *   k_cache, v_cache  [num_blocks, block_size, Hkv, d] (dtype)
+ *   block_table       device int32 [B, max_blocks]; entries past a sequence's
+ *                     last filled block are never read
+ *   block_size        a power of two, 16 .. 1024
+ *   seqlens_k         device int32 [B]: lengths INCLUDING the Nq new tokens
+ *   k_new, v_new      NULL, or device [B, Nq, Hkv, d]: the new tokens' K and V,
+ *                     written into the cache at logical positions
+ *                     seqlens_k[b] - Nq .. seqlens_k[b] - 1 before the
+ *                     attention reads them (so the cache is modified)
+ *   everything else as attn_fwd_varlen_kvcache, workspace of
+ *   attn_decode_workspace_bytes(B, Hq, Hkv, Nq, d, max_seqlen_k, split_keys).
+ * Only the tensor-core decode reads a paged cache: Hq/Hkv must divide 128,
+ * Nq * Hq/Hkv <= 128 and split_keys must be 0 or a multiple of 128, else
+ * ATTN_ERR_UNSUPPORTED.  A table entry outside [0, num_blocks) for a filled
+ * block is reported in the device error word (the rows read are block 0's).
+ */
+ATTN_API int attn_fwd_paged_kvcache(const void* q, void* k_cache, void* v_cache,
+                                    const int* block_table, int max_blocks, int block_size,
+                                    int num_blocks, const int* seqlens_k, int max_seqlen_k,
+                                    const void* k_new, const void* v_new, void* o, float* lse,
+                                    int B, int Hq, int Hkv, int Nq, int d, float scale,
+                                    int causal, int dtype, void* workspace,
+                                    size_t workspace_bytes, int split_keys, void* stream);
+
+/*
  * Bytes of device workspace that attn_bwd needs for these sizes: two float32
  * arrays of B * Hq * Nq (per query row, the dot product of dO and O, and the
  * forward's LSE in base 2), each 256-byte aligned.  Returns 0 for invalid

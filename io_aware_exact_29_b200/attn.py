@@ -52,6 +52,9 @@ def load_library():
             lib.attn_fwd_varlen_kvcache.argtypes = [vp, vp, vp, vp, vp, i, i, vp, vp, i, i, i, i,
                                                     i, f, i, i, vp, sz, i, vp]
             lib.attn_fwd_varlen_kvcache.restype = i
+            lib.attn_fwd_paged_kvcache.argtypes = [vp, vp, vp, vp, i, i, i, vp, i, vp, vp, vp,
+                                                   vp, i, i, i, i, i, f, i, i, vp, sz, i, vp]
+            lib.attn_fwd_paged_kvcache.restype = i
             lib.attn_bwd_workspace_bytes.argtypes = [i, i, i]
             lib.attn_bwd_workspace_bytes.restype = sz
             lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i,
@@ -208,6 +211,48 @@ def attn_fwd_varlen_kvcache(q, k_cache, v_cache, cu_seqlens_k, seqlens_k, max_se
         Hq, Hkv, Nq, d, float(scale), int(bool(causal)), _dtype_code(q), workspace.data_ptr(),
         workspace.numel(), int(split_keys), _stream_ptr(stream))
     _check("attn_fwd_varlen_kvcache", rc)
+    return out, lse
+
+
+def attn_fwd_paged_kvcache(q, k_cache, v_cache, block_table, seqlens_k, max_seqlen_k,
+                           scale=None, causal=False, k_new=None, v_new=None, split_keys=0,
+                           workspace=None, out=None, lse=None, stream=None):
+    """Decode attention against a paged KV cache.
+
+    q [B, Nq, Hq, d]; k_cache/v_cache [num_blocks, block_size, Hkv, d];
+    block_table int32 [B, max_blocks]; seqlens_k int32 [B] (lengths including
+    the new tokens); k_new/v_new optional [B, Nq, Hkv, d], written into the
+    cache before the attention.  Returns (o, lse).
+    """
+    lib = load_library()
+    B, Nq, Hq, d = q.shape
+    num_blocks, block_size, Hkv, _ = k_cache.shape
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"),
+                 (block_table, "block_table"), (seqlens_k, "seqlens_k")):
+        _dev(t, n)
+    if block_table.dtype != torch.int32 or seqlens_k.dtype != torch.int32:
+        raise TypeError("block_table and seqlens_k must be int32")
+    if scale is None:
+        scale = float(d) ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(decode_workspace_bytes(B, Hq, Hkv, Nq, d, max_seqlen_k, split_keys),
+                                dtype=torch.uint8, device=q.device)
+    kn = vn = None
+    if k_new is not None:
+        _dev(k_new, "k_new")
+        _dev(v_new, "v_new")
+        kn, vn = k_new.data_ptr(), v_new.data_ptr()
+    rc = lib.attn_fwd_paged_kvcache(
+        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
+        block_table.shape[1], block_size, num_blocks, seqlens_k.data_ptr(), int(max_seqlen_k),
+        kn, vn, out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Nq, d, float(scale),
+        int(bool(causal)), _dtype_code(q), workspace.data_ptr(), workspace.numel(),
+        int(split_keys), _stream_ptr(stream))
+    _check("attn_fwd_paged_kvcache", rc)
     return out, lse
 
 

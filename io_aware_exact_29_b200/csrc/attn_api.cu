@@ -297,6 +297,101 @@ int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_ca
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+int attn_fwd_paged_kvcache(const void* q, void* k_cache, void* v_cache, const int* block_table,
+                           int max_blocks, int block_size, int num_blocks, const int* seqlens_k,
+                           int max_seqlen_k, const void* k_new, const void* v_new, void* o,
+                           float* lse, int B, int Hq, int Hkv, int Nq, int d, float scale,
+                           int causal, int dtype, void* workspace, size_t workspace_bytes,
+                           int split_keys, void* stream) {
+    if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq <= 0 || Nq > 16)
+        return ATTN_ERR_INVALID_ARG;
+    if (B > 65535 || max_seqlen_k < 0 || max_blocks <= 0 || num_blocks <= 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (block_size < 16 || block_size > 1024 || (block_size & (block_size - 1)))
+        return ATTN_ERR_INVALID_ARG;
+    if ((long)max_blocks * block_size < max_seqlen_k) return ATTN_ERR_INVALID_ARG;
+    if ((long)num_blocks * block_size > 0x7fffffffL) return ATTN_ERR_INVALID_ARG;
+    if (split_keys < 0 || (split_keys % 64) != 0) return ATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    if (!q || !k_cache || !v_cache || !block_table || !seqlens_k || !o || !lse)
+        return ATTN_ERR_INVALID_ARG;
+    if ((k_new == nullptr) != (v_new == nullptr)) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+        !aligned16(lse) || (k_new && (!aligned16(k_new) || !aligned16(v_new))) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+        (reinterpret_cast<uintptr_t>(seqlens_k) & 3u))
+        return ATTN_ERR_INVALID_ARG;
+    const int G = Hq / Hkv;
+    // the paged path is the tensor-core decode's
+    if (!decode_use_tc(G, Nq, split_keys)) return ATTN_ERR_UNSUPPORTED;
+    int dev = 0;
+    const int st = check_device(&dev);
+    if (st == 0) return ATTN_ERR_CUDA;
+    if (st < 0) return ATTN_ERR_UNSUPPORTED;
+
+    const DecodeLayout lay = decode_layout(B, Hq, Hkv, Nq, d, max_seqlen_k, split_keys);
+    if (!workspace || workspace_bytes < lay.total ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return ATTN_ERR_WORKSPACE;
+
+    CUtensorMap kmap, vmap, qmap;
+    const uint64_t slots = (uint64_t)num_blocks * block_size;
+    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)Hkv, slots};
+    const uint64_t strides[2] = {(uint64_t)d * 2, (uint64_t)Hkv * d * 2};
+    const uint32_t box[3] = {64, 1, (uint32_t)std::min(128, block_size)};
+    if (!encode_map(&kmap, dtype, k_cache, 3, dims, strides, box) ||
+        !encode_map(&vmap, dtype, v_cache, 3, dims, strides, box))
+        return ATTN_ERR_INVALID_ARG;
+    const uint64_t qdims[5] = {(uint64_t)d, (uint64_t)G, (uint64_t)Hkv, (uint64_t)Nq, (uint64_t)B};
+    const uint64_t qstrides[4] = {(uint64_t)d * 2, (uint64_t)G * d * 2, (uint64_t)Hq * d * 2,
+                                  (uint64_t)Nq * Hq * d * 2};
+    const uint32_t qbox[5] = {64, (uint32_t)G, 1, (uint32_t)(128 / G), 1};
+    if (!encode_map(&qmap, dtype, q, 5, qdims, qstrides, qbox)) return ATTN_ERR_INVALID_ARG;
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    DecodeParams p{};
+    p.q = q;
+    p.o = o;
+    p.lse = lse;
+    p.cu_seqlens_k = nullptr;
+    p.seqlens_k = seqlens_k;
+    p.part_o = reinterpret_cast<float*>(ws + lay.part_o_off);
+    p.part_lse = reinterpret_cast<float*>(ws + lay.part_lse_off);
+    p.counters = reinterpret_cast<unsigned*>(ws + lay.counters_off);
+    p.plan = reinterpret_cast<DecodePlan*>(ws + lay.plan_off);
+    p.seq_prefix = reinterpret_cast<long long*>(ws + lay.prefix_off);
+    p.range_units = reinterpret_cast<int2*>(ws + lay.ranges_off);
+    p.max_seqlen_k = max_seqlen_k;
+    p.max_ranges = lay.max_ranges;
+    p.block_table = block_table;
+    p.max_blocks = max_blocks;
+    p.block_shift = __builtin_ctz((unsigned)block_size);
+    p.num_blocks = num_blocks;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nq = Nq;
+    p.G = G;
+    p.rows = Nq * G;
+    p.n_mgroups = lay.n_mgroups;
+    p.split_keys = lay.split_keys;
+    p.max_splits = lay.max_splits;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.limit_ns = kDefaultLimitNs;
+    p.err = g_err_addr[dev];
+    const int n_ctas = std::min(g_sm_count[dev], lay.max_ranges);
+    cudaError_t e = launch_decode_tc(qmap, kmap, vmap, p, d, dtype == ATTN_BF16, n_ctas,
+                                     static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq) {
     if (B <= 0 || Hq <= 0 || Nq <= 0) return 0;
     const size_t one = (((size_t)B * Hq * Nq * 4) + 255) & ~(size_t)255;

@@ -47,6 +47,8 @@
 //
 // Every wait is a bounded mbarrier wait (named barriers cannot time out, and
 // a persistent loop must be able to leave on an error at any point).
+#include <algorithm>
+
 #include "attn_internal.h"
 #include "ptx.cuh"
 
@@ -470,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     item.seg = seg;
                     item.range = r;
                     item.Lk = Lk;
-                    item.slot0 = p.cu_seqlens_k[b];
+                    item.slot0 = p.block_table ? 0 : p.cu_seqlens_k[b];  // packed cache only
                     return;
                 }
                 r += gridDim.x;  // this range is done
@@ -478,6 +480,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (r < n_ranges) ru = p.range_units[r];
             }
         };
+        // a paged cache is read in runs of sub_rows rows (one block, or one
+        // 128-row tile of a larger block)
+        const int sub_rows = p.block_table ? min(kBlockN, 1 << p.block_shift) : kBlockN;
+        const int n_sub = kBlockN / sub_rows;
         int n = 0;        // items pushed
         int it = 0;       // items with keys (Q loads)
         int tg = 0;       // K/V tile pairs issued
@@ -517,7 +523,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 ++it;
                 for (int j = 0; j < nt; ++j, ++tg) {
-                    const int row0 = item.slot0 + key_begin + j * kBlockN;
+                    // cache rows of the tile's keys: one contiguous run in a
+                    // packed cache; in a paged cache, runs of sub_rows keys
+                    // found through the block table (lane u: run u)
+                    int row0 = item.slot0 + key_begin + j * kBlockN;
+                    if (p.block_table) {
+                        row0 = 0;
+                        if (lane < n_sub) {
+                            const int pos = key_begin + j * kBlockN + lane * sub_rows;
+                            const int lb = pos >> p.block_shift;
+                            int blk = 0;
+                            if (pos < item.Lk) {
+                                blk = lb < p.max_blocks
+                                          ? p.block_table[(size_t)item.b * p.max_blocks + lb]
+                                          : -1;
+                                if (blk < 0 || blk >= p.num_blocks) {  // a bad table entry
+                                    atomicCAS(p.err, 0u, kErrDecodeBase + 8);
+                                    blk = 0;
+                                }
+                            }
+                            row0 = (blk << p.block_shift) + (pos & ((1 << p.block_shift) - 1));
+                        }
+                    }
+                    // issue the tile's copies: n_sub runs of sub_rows rows per
+                    // 64-column block, each at its own place in the tile; lane u
+                    // issues run u (the lanes' copies go out together)
+                    auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar) {
+                        if (lane < n_sub)
+                            for (int c = 0; c < kDBlocks; ++c)
+                                ptx::tma_load_3d(dst + c * kBlockBytes + lane * sub_rows * 128, map,
+                                                 bar, c * 64, item.g, row0);
+                    };
                     const int sk = tg % KST;
                     if (!warp_wait(&bars->k_empty[sk], ((tg / KST) & 1) ^ 1, p.limit_ns,
                                    abort_flag)) {
@@ -525,12 +561,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    if (lane == 0) {
-                        ptx::mbar_arrive_expect_tx(&bars->k_full[sk], kTileBytes);
-                        for (int c = 0; c < kDBlocks; ++c)
-                            ptx::tma_load_3d(smem + L::kK + sk * kTileBytes + c * kBlockBytes,
-                                             &tm_k, &bars->k_full[sk], c * 64, item.g, row0);
-                    }
+                    if (lane == 0) ptx::mbar_arrive_expect_tx(&bars->k_full[sk], kTileBytes);
+                    __syncwarp();
+                    load_tile(smem + L::kK + sk * kTileBytes, &tm_k, &bars->k_full[sk]);
                     __syncwarp();
                     const int sv = tg % VST;
                     if (!warp_wait(&bars->v_empty[sv], ((tg / VST) & 1) ^ 1, p.limit_ns,
@@ -540,12 +573,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         k_extra = 1;  // its K tile is in flight
                         break;
                     }
-                    if (lane == 0) {
-                        ptx::mbar_arrive_expect_tx(&bars->v_full[sv], kTileBytes);
-                        for (int c = 0; c < kDBlocks; ++c)
-                            ptx::tma_load_3d(smem + L::kV + sv * kTileBytes + c * kBlockBytes,
-                                             &tm_v, &bars->v_full[sv], c * 64, item.g, row0);
-                    }
+                    if (lane == 0) ptx::mbar_arrive_expect_tx(&bars->v_full[sv], kTileBytes);
+                    __syncwarp();
+                    load_tile(smem + L::kV + sv * kTileBytes, &tm_v, &bars->v_full[sv]);
                     __syncwarp();
                     if (j == 0) {
                         // look the next piece up while this one's tiles stream in
@@ -905,6 +935,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ------------------------------------------------------------------ append
+// Paged cache: write the new tokens' K and V rows (k_new, v_new [B, Nq, Hkv, d])
+// at logical positions seqlens_k[b] - Nq .. seqlens_k[b] - 1, through the
+// block table, before the decode reads them.  One warp per (b, t, g) row,
+// 16 bytes per lane.
+template <int D>
+__global__ void __launch_bounds__(256) attn_paged_append_kernel(const __grid_constant__ DecodeParams p) {
+    constexpr int kLanes = D / 8;  // 16-byte chunks per row
+    const long rows = (long)p.B * p.Nq * p.Hkv;
+    const int lane = threadIdx.x & 31;
+    for (long r = ((long)blockIdx.x * blockDim.x + threadIdx.x) / 32; r < rows;
+         r += (long)gridDim.x * blockDim.x / 32) {
+        const int g = (int)(r % p.Hkv);
+        const long bt = r / p.Hkv;
+        const int t = (int)(bt % p.Nq);
+        const int b = (int)(bt / p.Nq);
+        const int pos = p.seqlens_k[b] - p.Nq + t;
+        if (pos < 0 || lane >= kLanes) continue;
+        const int lb = pos >> p.block_shift;
+        const int blk = lb < p.max_blocks ? p.block_table[(size_t)b * p.max_blocks + lb] : -1;
+        if (blk < 0 || blk >= p.num_blocks) {
+            if (lane == 0) atomicCAS(p.err, 0u, kErrDecodeBase + 9);
+            continue;
+        }
+        const size_t row = ((size_t)blk << p.block_shift) + (pos & ((1 << p.block_shift) - 1));
+        const size_t dst = (row * p.Hkv + g) * (D / 8) + lane;
+        const size_t src = (((size_t)b * p.Nq + t) * p.Hkv + g) * (D / 8) + lane;
+        reinterpret_cast<uint4*>(p.k_cache)[dst] = reinterpret_cast<const uint4*>(p.k_new)[src];
+        reinterpret_cast<uint4*>(p.v_cache)[dst] = reinterpret_cast<const uint4*>(p.v_new)[src];
+    }
+}
+
 template <int D, bool BF16, int KST, int VST>
 cudaError_t launch_t(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUtensorMap& vmap,
                      const DecodeParams& p, int n_ctas, cudaStream_t stream) {
@@ -914,6 +976,13 @@ cudaError_t launch_t(const CUtensorMap& qmap, const CUtensorMap& kmap, const CUt
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc);
     if (e != cudaSuccess) return e;
+    if (p.block_table && p.k_new) {
+        const long warps = (long)p.B * p.Nq * p.Hkv;
+        const int blocks = (int)std::min<long>((warps + 7) / 8, 148L * 8);
+        attn_paged_append_kernel<D><<<blocks, 256, 0, stream>>>(p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
     attn_decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(p, n_ctas);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -78,6 +78,15 @@ struct DecodeParams {
     int2* range_units;      // [max_ranges] first and last unit of range r
     int max_seqlen_k;
     int max_ranges;
+    // paged cache (tensor-core decode): block_table == nullptr for a packed cache
+    const int* block_table;  // [B, max_blocks] physical block of each logical block
+    int max_blocks;
+    int block_shift;         // block_size = 1 << block_shift
+    int num_blocks;
+    void* k_cache;           // [num_blocks * block_size, Hkv, d], for the append
+    void* v_cache;
+    const void* k_new;       // [B, Nq, Hkv, d] rows to append, or nullptr
+    const void* v_new;
     int B, Hq, Hkv, Nq, G;
     int rows;              // Nq * G query rows per (sequence, kv head)
     int n_mgroups;         // ceil(rows / 16)

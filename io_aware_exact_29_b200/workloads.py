@@ -143,3 +143,57 @@ def kvcache_inputs(case: DecodeCase, seed: int = 0, device: str = "cpu",
             v_cache[s0:s1] = slack_fill
     return dict(q=q, k_cache=k_cache, v_cache=v_cache, cu_seqlens_k=cu.to(torch.int32),
                 seqlens_k=drawn)
+
+
+def paged_from_packed(inp, block_size: int, seed: int = 0, spare_blocks: int = 2,
+                      fill: float = float("nan"), new_tokens: int = 0):
+    """The same logical cache as ``kvcache_inputs`` laid out in blocks.
+
+    Sequence b's first seqlens_k[b] rows go, in order, into ceil(L/block_size)
+    physical blocks drawn from a seeded permutation; every other row (block
+    tails, spare blocks) holds ``fill``.  With ``new_tokens`` = n > 0 the last
+    n filled rows of each sequence are left as ``fill`` too and returned as
+    k_new/v_new [B, n, Hkv, d] (the rows an append would write).
+    Returns dict(k_cache, v_cache [num_blocks, block_size, Hkv, d],
+    block_table int32 [B, max_blocks] (-1 past a sequence's blocks),
+    seqlens_k, and k_new/v_new when requested).
+    """
+    kc, vc = inp["k_cache"], inp["v_cache"]
+    cu = inp["cu_seqlens_k"].tolist()
+    lens = inp["seqlens_k"].tolist()
+    B = len(lens)
+    nblk = [(L + block_size - 1) // block_size for L in lens]
+    total = sum(nblk) + spare_blocks
+    g = torch.Generator().manual_seed(seed + 7)
+    perm = torch.randperm(total, generator=g).tolist()
+    Hkv, d = kc.shape[1], kc.shape[2]
+    kp = torch.full((total, block_size, Hkv, d), fill, dtype=kc.dtype)
+    vp = torch.full((total, block_size, Hkv, d), fill, dtype=vc.dtype)
+    table = torch.full((B, max(1, max(nblk))), -1, dtype=torch.int32)
+    nxt = 0
+    for b in range(B):
+        for i in range(nblk[b]):
+            blk = perm[nxt]
+            nxt += 1
+            table[b, i] = blk
+            r0 = i * block_size
+            r1 = min(lens[b], r0 + block_size)
+            kp[blk, : r1 - r0] = kc[cu[b] + r0: cu[b] + r1]
+            vp[blk, : r1 - r0] = vc[cu[b] + r0: cu[b] + r1]
+    out = dict(k_cache=kp, v_cache=vp, block_table=table, seqlens_k=inp["seqlens_k"].clone())
+    if new_tokens:
+        n = new_tokens
+        kn = torch.zeros((B, n, Hkv, d), dtype=kc.dtype)
+        vn = torch.zeros((B, n, Hkv, d), dtype=vc.dtype)
+        for b in range(B):
+            for t in range(n):
+                pos = lens[b] - n + t
+                if pos < 0:
+                    continue
+                kn[b, t] = kc[cu[b] + pos]
+                vn[b, t] = vc[cu[b] + pos]
+                blk = int(table[b, pos // block_size])
+                kp[blk, pos % block_size] = fill
+                vp[blk, pos % block_size] = fill
+        out["k_new"], out["v_new"] = kn, vn
+    return out

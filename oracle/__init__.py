@@ -70,6 +70,11 @@ def _load():
             lib.oracle_attn_bwd.argtypes = [
                 _DP, _DP, _DP, _DP, _DP, _DP, _DP, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, _IP]
+            lib.oracle_attn_paged.restype = ctypes.c_int
+            lib.oracle_attn_paged.argtypes = [
+                _DP, _DP, _DP, _IP, ctypes.c_int, ctypes.c_int, ctypes.c_int, _IP, _DP, _DP,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_double, ctypes.c_int]
             lib.oracle_max_threads.restype = ctypes.c_int
             lib.oracle_set_threads.argtypes = [ctypes.c_int]
             _lib = lib
@@ -187,5 +192,55 @@ def attn_bwd(q, k, v, dout, scale: float, causal: bool, seqlens_k=None):
     return dq, dk, dv
 
 
-__all__ = ["build", "attn_fwd", "attn_kvcache", "lse_combine", "attn_bwd", "max_threads",
-           "set_threads"]
+def paged_append(k_cache, v_cache, block_table, seqlens_k, k_new, v_new):
+    """The cache after writing the new tokens' rows (a plain copy, no arithmetic).
+
+    k_cache/v_cache [num_blocks, block_size, Hkv, d]; k_new/v_new [B, Nq, Hkv, d];
+    token t of sequence b goes to logical position seqlens_k[b] - Nq + t, i.e.
+    block block_table[b][pos // block_size], row pos % block_size (positions
+    below 0 are dropped).  Returns float64 copies (k, v).
+    """
+    kc, vc = _f64(k_cache).copy(), _f64(v_cache).copy()
+    kn, vn = _f64(k_new), _f64(v_new)
+    bt, sl = _i32(block_table), _i32(seqlens_k)
+    bs = kc.shape[1]
+    B, Nq = kn.shape[0], kn.shape[1]
+    for b in range(B):
+        for t in range(Nq):
+            pos = int(sl[b]) - Nq + t
+            if pos < 0:
+                continue
+            blk, r = int(bt[b, pos // bs]), pos % bs
+            kc[blk, r] = kn[b, t]
+            vc[blk, r] = vn[b, t]
+    return kc, vc
+
+
+def attn_paged(q, k_cache, v_cache, block_table, seqlens_k, scale: float, causal: bool,
+               k_new=None, v_new=None):
+    """O, LSE against a paged KV cache (optionally after appending k_new/v_new).
+
+    q [B, Nq, Hq, d]; k_cache/v_cache [num_blocks, block_size, Hkv, d];
+    block_table [B, max_blocks] int; seqlens_k [B] (lengths after the append).
+    Returns float64 numpy arrays (o [B, Nq, Hq, d], lse [B, Hq, Nq]).
+    """
+    if k_new is not None:
+        kd, vd = paged_append(k_cache, v_cache, block_table, seqlens_k, k_new, v_new)
+    else:
+        kd, vd = _f64(k_cache), _f64(v_cache)
+    qd = _f64(q)
+    bt, sl = _i32(block_table), _i32(seqlens_k)
+    B, Nq, Hq, d = qd.shape
+    num_blocks, bs, Hkv, _ = kd.shape
+    o = np.full((B, Nq, Hq, d), np.nan)
+    lse = np.full((B, Hq, Nq), np.nan)
+    rc = _load().oracle_attn_paged(_dp(qd), _dp(kd), _dp(vd), _ip(bt), bt.shape[1], bs,
+                                   num_blocks, _ip(sl), _dp(o), _dp(lse), B, Hq, Hkv, Nq, d,
+                                   float(scale), int(bool(causal)))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_paged rejected its arguments (rc={rc})")
+    return o, lse
+
+
+__all__ = ["build", "attn_fwd", "attn_kvcache", "lse_combine", "attn_bwd", "attn_paged",
+           "paged_append", "max_threads", "set_threads"]

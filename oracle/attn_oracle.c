@@ -458,3 +458,82 @@ int oracle_attn_bwd(const double* q, const double* k, const double* v, const dou
     }
     return err ? -2 : 0;
 }
+
+/*
+ * Attention of new query tokens against a PAGED KV cache: the cache is cut
+ * into fixed blocks of block_size rows and sequence b's logical key j lives
+ * in physical block block_table[b][j / block_size], row j % block_size.
+ * (The ai6s.net article, adaptation point 3, has a pre-allocated cache that
+ * grows one row per token; paging is the same cache with its rows found
+ * through a table instead of one contiguous slice per sequence.)
+ *   q        [B, Nq, Hq, d]
+ *   k_cache, v_cache [num_blocks, block_size, Hkv, d]
+ *   block_table [B, max_blocks]; seqlens_k [B] (<= max_blocks * block_size)
+ *   o [B, Nq, Hq, d], lse [B, Hq, Nq]; causal is bottom-right, as above.
+ * Each sequence's keys are gathered into a contiguous scratch and attended
+ * exactly as in oracle_attn_kvcache.  Returns 0, -1 (bad arguments, or a
+ * table entry outside [0, num_blocks) for a filled block) or -2.
+ */
+int oracle_attn_paged(const double* q, const double* k_cache, const double* v_cache,
+                      const int* block_table, int max_blocks, int block_size, int num_blocks,
+                      const int* seqlens_k, double* o, double* lse, int B, int Hq, int Hkv, int Nq,
+                      int d, double scale, int causal) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || d <= 0 || Hq % Hkv != 0 || block_size <= 0 ||
+        max_blocks <= 0 || num_blocks <= 0)
+        return -1;
+    int maxlen = 0;
+    for (int b = 0; b < B; ++b) {
+        const int L = seqlens_k[b];
+        if (L < 0 || L > max_blocks * block_size) return -1;
+        for (int i = 0; i < (L + block_size - 1) / block_size; ++i) {
+            const int blk = block_table[(size_t)b * max_blocks + i];
+            if (blk < 0 || blk >= num_blocks) return -1;
+        }
+        if (L > maxlen) maxlen = L;
+    }
+    const int G = Hq / Hkv;
+    const size_t m1 = (size_t)(maxlen > 0 ? maxlen : 1);
+    const size_t per_thread = ((size_t)Nq * m1 + 2 * m1 * (size_t)d) * sizeof(double);
+    const int nthreads = pick_threads(per_thread);
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (long bh = 0; bh < (long)B * Hq; ++bh) {
+        const int b = (int)(bh / Hq), h = (int)(bh % Hq), g = h / G;
+        const int Lk = seqlens_k[b];
+        double* S = (double*)malloc((size_t)Nq * m1 * sizeof(double));
+        double* kg = (double*)malloc(m1 * (size_t)d * sizeof(double));
+        double* vg = (double*)malloc(m1 * (size_t)d * sizeof(double));
+        const double** qp = (const double**)malloc(sizeof(double*) * (size_t)Nq);
+        double** op = (double**)malloc(sizeof(double*) * (size_t)Nq);
+        double** lp = (double**)malloc(sizeof(double*) * (size_t)Nq);
+        int* ri = (int*)malloc(sizeof(int) * (size_t)Nq);
+        if (!S || !kg || !vg || !qp || !op || !lp || !ri) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+            for (int j = 0; j < Lk; ++j) { /* gather the sequence's rows through the table */
+                const int blk = block_table[(size_t)b * max_blocks + j / block_size];
+                const size_t row = (size_t)blk * block_size + (size_t)(j % block_size);
+                memcpy(kg + (size_t)j * d, k_cache + (row * Hkv + g) * (size_t)d,
+                       sizeof(double) * (size_t)d);
+                memcpy(vg + (size_t)j * d, v_cache + (row * Hkv + g) * (size_t)d,
+                       sizeof(double) * (size_t)d);
+            }
+            for (int i = 0; i < Nq; ++i) {
+                ri[i] = i;
+                qp[i] = q + (((size_t)b * Nq + i) * Hq + h) * (size_t)d;
+                op[i] = o + (((size_t)b * Nq + i) * Hq + h) * (size_t)d;
+                lp[i] = lse + ((size_t)b * Hq + h) * (size_t)Nq + i;
+            }
+            attend_head(Nq, qp, ri, kg, vg, (long)d, Nq, Lk, d, scale, causal, op, lp, S);
+        }
+        free(S);
+        free(kg);
+        free(vg);
+        free(qp);
+        free(op);
+        free(lp);
+        free(ri);
+    }
+    return err ? -2 : 0;
+}

@@ -130,3 +130,25 @@ def test_python_binding_fails_loudly_without_cuda_tensors():
     q = torch.zeros(1, 128, 1, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         attn.attn_fwd(q, q, q)
+
+
+def test_paged_decode_argument_checks():
+    lib = attn.load_library()
+    P = 1 << 20
+    f = lib.attn_fwd_paged_kvcache
+    base = dict(q=P, kc=P, vc=P, bt=P, mb=4, bs=16, nb=8, sl=P, ml=64, kn=None, vn=None, o=P,
+                lse=P, B=2, Hq=16, Hkv=2, Nq=1, d=128, scale=0.088, causal=0, dtype=0, ws=P,
+                wsb=1 << 30, split=0, st=None)
+
+    def call(**kw):
+        a = dict(base, **kw)
+        return f(a["q"], a["kc"], a["vc"], a["bt"], a["mb"], a["bs"], a["nb"], a["sl"], a["ml"],
+                 a["kn"], a["vn"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Nq"], a["d"],
+                 a["scale"], a["causal"], a["dtype"], a["ws"], a["wsb"], a["split"], a["st"])
+    assert call(bs=24) == -1          # not a power of two
+    assert call(bs=8) == -1           # below 16
+    assert call(ml=65) == -1          # max_blocks * block_size < max_seqlen_k
+    assert call(kn=P) == -1           # k_new without v_new
+    assert call(Nq=17) == -1
+    assert call(d=80) == -2
+    assert call(Hq=24) == -2          # 12 heads per kv head: not the tensor-core decode
