@@ -7,7 +7,8 @@ A step is one pass of the whole path over one batch of synthetic inputs:
   decode   : Llama2-70B shape, B=32, Hq=64, Hkv=8, d=128, one new token per
              sequence, packed bf16 KV cache with lengths ~ U[1, 32768], then
   decode16 : the same shape with a causal chunk of 16 new tokens per sequence
-             (its own cache of the same size).
+             (its own cache of the same size), then
+  paged    : the one-token decode again, its cache in 16-row blocks.
 `value` is the forward's TFLOP/s (algorithmic FLOPs / device time of the
 forward launches, summed over ranks); the decodes' GB/s are reported beside
 it.
@@ -41,7 +42,8 @@ if ROOT not in sys.path:
 
 from io_aware_exact_29_b200 import accounting  # noqa: E402
 from io_aware_exact_29_b200.workloads import (DECODE_CASES, FWD_CASES, fwd_inputs,  # noqa: E402
-                                              kvcache_inputs, upstream_grad)
+                                              kvcache_inputs, paged_from_packed,
+                                              upstream_grad)
 
 FWD_CASE = FWD_CASES["sweep_d128_n4096"]
 DEC_CASE = DECODE_CASES["llama70b_decode"]
@@ -201,6 +203,13 @@ def run_ours(args, rank, world, local):
     dlse = torch.empty((dc.B, dc.Hq, dc.Nq), dtype=torch.float32, device=dev)
     ws = torch.empty(attn.decode_workspace_bytes(dc.B, dc.Hq, dc.Hkv, dc.Nq, dc.d, max_len),
                      dtype=torch.uint8, device=dev)
+    # the one-token decode's cache in 16-row blocks behind a shuffled block table
+    pg = paged_from_packed({k: t.cpu() for k, t in din.items()}, 16, seed=1000 * rank + 3,
+                           fill=0.0)
+    pgd = {k: t.to(dev) for k, t in pg.items()}
+    del pg
+    do_pg = torch.empty_like(dq)
+    dl_pg = torch.empty_like(dlse)
     # the 16-token chunk variant of the decode (same cache shape, causal chunk)
     c16 = DEC16_CASE
     din16 = kvcache_inputs(c16, seed=1000 * rank + 1, device=str(dev))
@@ -237,8 +246,12 @@ def run_ours(args, rank, world, local):
                                      scale=c16.scale, causal=c16.causal, workspace=ws16, out=o16,
                                      lse=l16, stream=stream)
         ev[3].record(stream)
+        attn.attn_fwd_paged_kvcache(dq, pgd["k_cache"], pgd["v_cache"], pgd["block_table"],
+                                    pgd["seqlens_k"], max_len, scale=dc.scale, causal=dc.causal,
+                                    workspace=ws, out=do_pg, lse=dl_pg, stream=stream)
+        ev[5].record(stream)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     for _ in range(args.warmup):
         step(evs[0])
     torch.cuda.synchronize()
@@ -261,8 +274,9 @@ def run_ours(args, rank, world, local):
     bwd_ms = sum(e[1].elapsed_time(e[4]) for e in evs)
     dec_ms = sum(e[4].elapsed_time(e[2]) for e in evs)
     dec16_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
-    total_ms, fwd_ms, bwd_ms, dec_ms, dec16_ms = reduce_max(
-        [total_ms, fwd_ms, bwd_ms, dec_ms, dec16_ms], world, dev)
+    pg_ms = sum(e[3].elapsed_time(e[5]) for e in evs)
+    total_ms, fwd_ms, bwd_ms, dec_ms, dec16_ms, pg_ms = reduce_max(
+        [total_ms, fwd_ms, bwd_ms, dec_ms, dec16_ms, pg_ms], world, dev)
     assert attn.get_device_error() == 0
 
     # ---- end to end through the public API with host buffers
@@ -346,6 +360,16 @@ def run_ours(args, rank, world, local):
             "kernels_per_call": "attn_bwd_pre + attn_bwd_dkdv + attn_bwd_dq",
             "bound": "tensor",
         },
+        "decode_paged_bs16": {
+            "value": round(dbytes * args.steps * world / (pg_ms * 1e-3) / 1e9, 1),
+            "unit": "GB/s",
+            "ms_per_call": round(pg_ms / args.steps, 4),
+            "frac": round(dbytes / (pg_ms / args.steps * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "bytes_per_call": dbytes,
+            "layout": "the one-token decode's cache in 16-row blocks, shuffled block table",
+            "kernels_per_call": "plan + attn_decode_tc_kernel + merge",
+            "bound": "hbm",
+        },
         "decode_chunk16": {
             "value": round(dbytes16 * args.steps * world / (dec16_ms * 1e-3) / 1e9, 1),
             "unit": "GB/s",
@@ -361,8 +385,8 @@ def run_ours(args, rank, world, local):
                 "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["fwd_h2d"],
                 "d2h_bytes_per_step": e2e["fwd_d2h"]},
         # per step: the forward kernel, the three backward kernels, and
-        # plan + decode + merge for each decode
-        "gpu_launches": 10 * args.steps,
+        # plan + decode + merge for each of the three decodes
+        "gpu_launches": 13 * args.steps,
         "clocks": clk.summary(),
         "fwd_ms_per_launch": round(per_launch_ms, 4),
     }
