@@ -58,7 +58,7 @@ def _load():
             lib.oracle_attn_fwd.argtypes = [
                 _DP, _DP, _DP, _DP, _DP, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
-                _IP, _IP, ctypes.c_int]
+                _IP, _IP, ctypes.c_int, ctypes.c_int]
             lib.oracle_attn_kvcache.restype = ctypes.c_int
             lib.oracle_attn_kvcache.argtypes = [
                 _DP, _DP, _DP, _IP, _IP, _DP, _DP, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -69,7 +69,8 @@ def _load():
             lib.oracle_attn_bwd.restype = ctypes.c_int
             lib.oracle_attn_bwd.argtypes = [
                 _DP, _DP, _DP, _DP, _DP, _DP, _DP, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, _IP]
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, _IP,
+                ctypes.c_int]
             lib.oracle_attn_paged.restype = ctypes.c_int
             lib.oracle_attn_paged.argtypes = [
                 _DP, _DP, _DP, _IP, ctypes.c_int, ctypes.c_int, ctypes.c_int, _IP, _DP, _DP,
@@ -110,11 +111,13 @@ def set_threads(n: int) -> None:
     _load().oracle_set_threads(int(n))
 
 
-def attn_fwd(q, k, v, scale: float, causal: bool, seqlens_k=None, rows=None):
+def attn_fwd(q, k, v, scale: float, causal: bool, seqlens_k=None, rows=None, window_left=-1):
     """O, LSE of dense attention.
 
     q [B, Nq, Hq, d], k/v [B, Nk, Hkv, d] (any float dtype; widened exactly).
     seqlens_k: optional [B] key lengths (keys at or past it are masked).
+    window_left: -1, or the sliding window: keys more than window_left
+    positions before the query's own position i + (Lk - Nq) are masked.
     rows: optional list of query-row indices; only those rows are computed
     (the other entries of the returned arrays are NaN).
     Returns (o [B, Nq, Hq, d] float64, lse [B, Hq, Nq] float64) numpy arrays.
@@ -128,7 +131,7 @@ def attn_fwd(q, k, v, scale: float, causal: bool, seqlens_k=None, rows=None):
     rw = None if rows is None else _i32(rows)
     rc = _load().oracle_attn_fwd(_dp(qd), _dp(kd), _dp(vd), _dp(o), _dp(lse), B, Hq, Hkv, Nq,
                                  Nk, d, float(scale), int(bool(causal)), _ip(sl), _ip(rw),
-                                 0 if rw is None else len(rw))
+                                 0 if rw is None else len(rw), int(window_left))
     if rc != 0:
         raise ValueError(f"oracle_attn_fwd rejected its arguments (rc={rc})")
     return o, lse
@@ -170,7 +173,7 @@ def lse_combine(o_parts, lse_parts):
     return o, lse
 
 
-def attn_bwd(q, k, v, dout, scale: float, causal: bool, seqlens_k=None):
+def attn_bwd(q, k, v, dout, scale: float, causal: bool, seqlens_k=None, window_left=-1):
     """Gradients (dq, dk, dv) of L = sum(dout * O) for O = attention(q, k, v).
 
     q, dout [B, Nq, Hq, d]; k, v [B, Nk, Hkv, d]; seqlens_k optional [B].
@@ -186,7 +189,8 @@ def attn_bwd(q, k, v, dout, scale: float, causal: bool, seqlens_k=None):
     dv = np.full((B, Nk, Hkv, d), np.nan)
     sl = None if seqlens_k is None else _i32(seqlens_k)
     rc = _load().oracle_attn_bwd(_dp(qd), _dp(kd), _dp(vd), _dp(dod), _dp(dq), _dp(dk), _dp(dv),
-                                 B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), _ip(sl))
+                                 B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), _ip(sl),
+                                 int(window_left))
     if rc != 0:
         raise ValueError(f"oracle_attn_bwd rejected its arguments (rc={rc})")
     return dq, dk, dv

@@ -33,7 +33,10 @@
  *    j <= i + (Lk - Nq), which is the usual top-left rule when Nq == Lk and
  *    makes the newest query tokens the last rows of a growing KV cache;
  *  - a row with no visible key gives O = 0 and LSE = -inf;
- *  - grouped-query heads map contiguously: g = h / (Hq / Hkv).
+ *  - grouped-query heads map contiguously: g = h / (Hq / Hkv);
+ *  - a sliding window (window_left >= 0) also masks keys more than
+ *    window_left positions before the query's own position i + (Lk - Nq)
+ *    (the "extensions for masks" the pages list as a direction); -1 = none.
  *
  * Arithmetic: every input is fp64 (the caller widens the bf16/fp16 bits
  * exactly).  Row sums and output sums use Neumaier compensated summation so
@@ -65,6 +68,15 @@ static void csum_add(csum_t* a, double x) {
 
 static double csum_value(const csum_t* a) { return a->sum + a->comp; }
 
+/* ---- the mask: is key j visible to query row i? --------------------------
+ * causal: j <= i + (Lk - Nq); window_left >= 0: j >= i + (Lk - Nq) - window_left */
+static int key_visible(int i, int j, int Nq, int Lk, int causal, int window_left) {
+    const int pos = i + (Lk - Nq); /* the query's own position among the keys */
+    if (causal && j > pos) return 0;
+    if (window_left >= 0 && j < pos - window_left) return 0;
+    return 1;
+}
+
 /* ---- one query head against one key/value head --------------------------
  * q_rows[r]   : pointer to the d values of the r-th requested query row
  * row_index[r]: that row's index i in [0, Nq), used by the causal rule
@@ -74,15 +86,15 @@ static double csum_value(const csum_t* a) { return a->sum + a->comp; }
  */
 static void attend_head(int nrows, const double* const* q_rows, const int* row_index,
                         const double* k, const double* v, long kv_stride, int Nq, int Lk,
-                        int d, double scale, int causal, double* const* o_rows,
-                        double* const* lse_out, double* S) {
+                        int d, double scale, int causal, int window_left,
+                        double* const* o_rows, double* const* lse_out, double* S) {
     for (int r = 0; r < nrows; ++r) {
         const double* qi = q_rows[r];
         const int i = row_index[r];
         double* Srow = S + (size_t)r * (size_t)(Lk > 0 ? Lk : 1);
         /* step 1 + 2: scores, then the additive 0 / -inf mask */
         for (int j = 0; j < Lk; ++j) {
-            int visible = causal ? (j <= i + (Lk - Nq)) : 1;
+            const int visible = key_visible(i, j, Nq, Lk, causal, window_left);
             if (!visible) {
                 Srow[j] = -INFINITY;
                 continue;
@@ -172,7 +184,7 @@ void oracle_set_threads(int n) {
  */
 int oracle_attn_fwd(const double* q, const double* k, const double* v, double* o, double* lse,
                     int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale, int causal,
-                    const int* seqlens_k, const int* rows, int nrows) {
+                    const int* seqlens_k, const int* rows, int nrows, int window_left) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || d <= 0 || Hq % Hkv != 0) return -1;
     if (seqlens_k)
         for (int b = 0; b < B; ++b)
@@ -207,7 +219,8 @@ int oracle_attn_fwd(const double* q, const double* k, const double* v, double* o
             }
             const double* kb = k + ((size_t)b * Nk * Hkv + g) * (size_t)d;
             const double* vb = v + ((size_t)b * Nk * Hkv + g) * (size_t)d;
-            attend_head(nr, qp, ri, kb, vb, (long)Hkv * d, Nq, Lk, d, scale, causal, op, lp, S);
+            attend_head(nr, qp, ri, kb, vb, (long)Hkv * d, Nq, Lk, d, scale, causal, window_left,
+                        op, lp, S);
         }
         free(S);
         free(qp);
@@ -263,7 +276,8 @@ int oracle_attn_kvcache(const double* q, const double* k_cache, const double* v_
             }
             const double* kb = k_cache + ((size_t)cu_seqlens_k[b] * Hkv + g) * (size_t)d;
             const double* vb = v_cache + ((size_t)cu_seqlens_k[b] * Hkv + g) * (size_t)d;
-            attend_head(Nq, qp, ri, kb, vb, (long)Hkv * d, Nq, Lk, d, scale, causal, op, lp, S);
+            attend_head(Nq, qp, ri, kb, vb, (long)Hkv * d, Nq, Lk, d, scale, causal, -1, op, lp,
+                        S);
         }
         free(S);
         free(qp);
@@ -341,7 +355,7 @@ int oracle_lse_combine(const double* o_parts, const double* lse_parts, int npart
  */
 int oracle_attn_bwd(const double* q, const double* k, const double* v, const double* dout,
                     double* dq, double* dk, double* dv, int B, int Hq, int Hkv, int Nq, int Nk,
-                    int d, double scale, int causal, const int* seqlens_k) {
+                    int d, double scale, int causal, const int* seqlens_k, int window_left) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || d <= 0 || Hq % Hkv != 0) return -1;
     if (seqlens_k)
         for (int b = 0; b < B; ++b)
@@ -377,7 +391,7 @@ int oracle_attn_bwd(const double* q, const double* k, const double* v, const dou
                     /* P row: scores, mask, softmax */
                     double m = -INFINITY;
                     for (int j = 0; j < Lk; ++j) {
-                        const int visible = causal ? (j <= i + (Lk - Nq)) : 1;
+                        const int visible = key_visible(i, j, Nq, Lk, causal, window_left);
                         if (!visible) {
                             Prow[j] = -INFINITY;
                             continue;
@@ -525,7 +539,7 @@ int oracle_attn_paged(const double* q, const double* k_cache, const double* v_ca
                 op[i] = o + (((size_t)b * Nq + i) * Hq + h) * (size_t)d;
                 lp[i] = lse + ((size_t)b * Hq + h) * (size_t)Nq + i;
             }
-            attend_head(Nq, qp, ri, kg, vg, (long)d, Nq, Lk, d, scale, causal, op, lp, S);
+            attend_head(Nq, qp, ri, kg, vg, (long)d, Nq, Lk, d, scale, causal, -1, op, lp, S);
         }
         free(S);
         free(kg);

@@ -11,11 +11,12 @@ from __future__ import annotations
 import math
 
 
-def attention_rows(q, k, v, scale, causal=False, lk=None):
+def attention_rows(q, k, v, scale, causal=False, lk=None, window_left=None):
     """q: list of Nq rows, k/v: lists of Nk rows (lists of floats).
 
     Returns (o, lse): o is a list of Nq output rows, lse a list of Nq floats.
-    Key j is visible to query i iff j < lk and (not causal or j <= i + lk - Nq).
+    Key j is visible to query i iff j < lk and (not causal or j <= i + lk - Nq)
+    and (window_left is None or j >= i + lk - Nq - window_left).
     """
     nq = len(q)
     nk = len(k) if lk is None else lk
@@ -25,6 +26,8 @@ def attention_rows(q, k, v, scale, causal=False, lk=None):
         scores = []
         for j in range(nk):
             if causal and j > i + nk - nq:
+                continue
+            if window_left is not None and j < i + nk - nq - window_left:
                 continue
             s = 0.0
             for t in range(d):
