@@ -88,6 +88,20 @@ ATTN_API int attn_fwd_kpad(const void* q, const void* k, const void* v, void* o,
                   const int* seqlens_k, void* stream);
 
 /*
+ * Forward attention with a sliding window: as attn_fwd_kpad (seqlens_k may be
+ * NULL), plus window_left: -1 for none, else query i also masks every key
+ * j < i + (Lk - Nq) - window_left, i.e. it sees at most window_left keys
+ * before its own position (with causal: the window_left + 1 most recent
+ * keys).  The pages list mask extensions as a direction without a form
+ * (machinelearning.ru page, "directions"); key tiles wholly outside the
+ * window are skipped like those above the causal diagonal.
+ */
+ATTN_API int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                             int causal, int window_left, int dtype, const int* seqlens_k,
+                             void* stream);
+
+/*
  * Bytes of device workspace that attn_fwd_varlen_kvcache needs for these
  * sizes.  split_keys: keys per split-K work unit, a multiple of 64, or 0 to
  * let the library choose (the same rule the decode call applies).  Returns 0
@@ -198,6 +212,16 @@ ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o
                       int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype,
                       const int* seqlens_k, void* workspace, size_t workspace_bytes,
                       void* stream);
+
+/*
+ * attn_bwd for the sliding-window forward (attn_fwd_window): the same
+ * arguments plus window_left (-1 = none), which must match the forward's.
+ */
+ATTN_API int attn_bwd_window(const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                             int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                             int causal, int window_left, int dtype, const int* seqlens_k,
+                             void* workspace, size_t workspace_bytes, void* stream);
 
 /* Size in bytes of the scratch area built into the library for
  * attn_fwd_varlen_kvcache_noalloc (32 MiB). */

@@ -47,6 +47,12 @@ def load_library():
             lib.attn_fwd.restype = i
             lib.attn_fwd_kpad.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp, vp]
             lib.attn_fwd_kpad.restype = i
+            lib.attn_fwd_window.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp,
+                                            vp]
+            lib.attn_fwd_window.restype = i
+            lib.attn_bwd_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i,
+                                            f, i, i, i, vp, vp, sz, vp]
+            lib.attn_bwd_window.restype = i
             lib.attn_decode_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
             lib.attn_decode_workspace_bytes.restype = sz
             lib.attn_fwd_varlen_kvcache.argtypes = [vp, vp, vp, vp, vp, i, i, vp, vp, i, i, i, i,
@@ -102,7 +108,7 @@ def _dev(t: torch.Tensor, name: str):
 
 
 def attn_fwd(q, k, v, scale=None, causal=False, seqlens_k=None, out=None, lse=None,
-             stream=None):
+             stream=None, window_left=-1):
     """Exact attention forward.
 
     q [B, Nq, Hq, d], k/v [B, Nk, Hkv, d] (bf16/fp16, CUDA, contiguous);
@@ -121,7 +127,19 @@ def attn_fwd(q, k, v, scale=None, causal=False, seqlens_k=None, out=None, lse=No
     if lse is None:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     st = _stream_ptr(stream)
-    if seqlens_k is None:
+    if window_left >= 0:
+        sl = 0
+        if seqlens_k is not None:
+            _dev(seqlens_k, "seqlens_k")
+            if seqlens_k.dtype != torch.int32:
+                raise TypeError("seqlens_k must be int32")
+            sl = seqlens_k.data_ptr()
+        rc = lib.attn_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
+                                 int(bool(causal)), int(window_left), _dtype_code(q), sl or None,
+                                 st)
+        _check("attn_fwd_window", rc)
+    elif seqlens_k is None:
         rc = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                           lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)),
                           _dtype_code(q), st)
@@ -142,7 +160,7 @@ def bwd_workspace_bytes(B, Hq, Nq) -> int:
 
 
 def attn_bwd(q, k, v, o, lse, dout, scale=None, causal=False, seqlens_k=None, workspace=None,
-             dq=None, dk=None, dv=None, stream=None):
+             dq=None, dk=None, dv=None, stream=None, window_left=-1):
     """Gradients of L = sum(dout * O) for O = attn_fwd(q, k, v, ...).
 
     o and lse are the forward's outputs for the same arguments.  Returns
@@ -168,10 +186,11 @@ def attn_bwd(q, k, v, o, lse, dout, scale=None, causal=False, seqlens_k=None, wo
         if seqlens_k.dtype != torch.int32:
             raise TypeError("seqlens_k must be int32")
         sl = seqlens_k.data_ptr()
-    rc = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                      dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv,
-                      Nq, Nk, d, float(scale), int(bool(causal)), _dtype_code(q), sl or None,
-                      workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    rc = lib.attn_bwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                             dv.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
+                             int(bool(causal)), int(window_left), _dtype_code(q), sl or None,
+                             workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
     _check("attn_bwd", rc)
     return dq, dk, dv
 

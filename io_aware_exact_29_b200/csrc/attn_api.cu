@@ -115,7 +115,9 @@ bool map_bnhd(CUtensorMap* m, int dtype, const void* base, int B, int N, int H, 
 
 int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype,
-               const int* seqlens_k, void* stream, int inject, unsigned long long limit_ns) {
+               const int* seqlens_k, void* stream, int inject, unsigned long long limit_ns,
+               int window_left) {
+    if (window_left < -1) return ATTN_ERR_INVALID_ARG;
     if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk < 0 || Hq % Hkv != 0)
@@ -154,6 +156,7 @@ int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse,
     p.causal = causal ? 1 : 0;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.seqlens_k = Nk > 0 ? seqlens_k : nullptr;
+    p.window_left = window_left;
     p.lse = lse;
     p.limit_ns = limit_ns;
     p.inject = inject;
@@ -180,21 +183,28 @@ extern "C" {
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
              int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype, void* stream) {
     return fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, nullptr,
-                      stream, 0, kDefaultLimitNs);
+                      stream, 0, kDefaultLimitNs, -1);
 }
 
 int attn_fwd_kpad(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                   int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype,
                   const int* seqlens_k, void* stream) {
     return fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, seqlens_k,
-                      stream, 0, kDefaultLimitNs);
+                      stream, 0, kDefaultLimitNs, -1);
+}
+
+int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                    int window_left, int dtype, const int* seqlens_k, void* stream) {
+    return fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, seqlens_k,
+                      stream, 0, kDefaultLimitNs, window_left);
 }
 
 int attn_selftest_watchdog(const void* q, const void* k, const void* v, void* o, float* lse,
                            int limit_ms, void* stream) {
     if (limit_ms <= 0 || limit_ms > 10000) return ATTN_ERR_INVALID_ARG;
     return fwd_common(q, k, v, o, lse, 1, 1, 1, 128, 128, 64, 0.125f, 0, ATTN_BF16, nullptr,
-                      stream, 1, (unsigned long long)limit_ms * 1000000ull);
+                      stream, 1, (unsigned long long)limit_ms * 1000000ull, -1);
 }
 
 size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int d, int max_seqlen_k,
@@ -402,6 +412,16 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
              const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
              int Nk, int d, float scale, int causal, int dtype, const int* seqlens_k,
              void* workspace, size_t workspace_bytes, void* stream) {
+    return attn_bwd_window(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale,
+                           causal, -1, dtype, seqlens_k, workspace, workspace_bytes, stream);
+}
+
+int attn_bwd_window(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
+                    int Nq, int Nk, int d, float scale, int causal, int window_left, int dtype,
+                    const int* seqlens_k, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+    if (window_left < -1) return ATTN_ERR_INVALID_ARG;
     if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk < 0 || Hq % Hkv != 0)
@@ -446,6 +466,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.seqlens_k = Nk > 0 ? seqlens_k : nullptr;
+    p.window_left = window_left;
     p.o = o;
     p.dout = dout;
     p.lse = lse;

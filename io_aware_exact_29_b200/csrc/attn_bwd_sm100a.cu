@@ -208,7 +208,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     int qt_first = 0;
     if (p.causal) qt_first = max(0, k0 - off) / kBlock;
     const int n_qt = (p.Nq + kBlock - 1) / kBlock;
-    const int nqs = (k0 < Lk) ? max(0, n_qt - qt_first) : 0;
+    int qt_end = n_qt;
+    if (p.window_left >= 0) {
+        // the last query that sees a key of this tile: i <= key - off + window_left
+        const int i_max = min(Lk - 1, k0 + kBlock - 1) - off + p.window_left;
+        qt_end = i_max < 0 ? 0 : min(n_qt, i_max / kBlock + 1);
+    }
+    const int nqs = (k0 < Lk) ? max(0, qt_end - qt_first) : 0;
     const int nsteps = p.G * nqs;
 
     if (tid == 0) {
@@ -413,7 +419,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_ld32(t_s, sv);
             ptx::tmem_ld32(t_dp, dv);
             // every (key, query) pair of this thread's 32 columns visible?
-            const bool full = key_ok && i0 + qc0 + 32 <= p.Nq && (!p.causal || kr <= i0 + qc0 + off);
+            const bool full = key_ok && i0 + qc0 + 32 <= p.Nq && (!p.causal || kr <= i0 + qc0 + off) &&
+                              (p.window_left < 0 || kr >= i0 + qc0 + 31 + off - p.window_left);
             const bool masked = __any_sync(0xffffffffu, !full);
             ptx::tmem_wait_ld_dep(sv);
             ptx::tmem_wait_ld_dep(dv);
@@ -440,8 +447,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(p0, p1), d2), ds0, ds1);
                     if (masked) {
                         const int qi = i0 + qc0 + e;
-                        const bool v0 = key_ok && qi < p.Nq && (!p.causal || kr <= qi + off);
-                        const bool v1 = key_ok && qi + 1 < p.Nq && (!p.causal || kr <= qi + 1 + off);
+                        const bool w0 = p.window_left < 0 || kr >= qi + off - p.window_left;
+                        const bool w1 = p.window_left < 0 || kr >= qi + 1 + off - p.window_left;
+                        const bool v0 = key_ok && qi < p.Nq && (!p.causal || kr <= qi + off) && w0;
+                        const bool v1 =
+                            key_ok && qi + 1 < p.Nq && (!p.causal || kr <= qi + 1 + off) && w1;
                         p0 = v0 ? p0 : 0.f;
                         ds0 = v0 ? ds0 : 0.f;
                         p1 = v1 ? p1 : 0.f;
@@ -559,7 +569,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = h / p.G;
     const int Lk = p.seqlens_k ? p.seqlens_k[b] : p.Nk;
     const int off = Lk - p.Nq;
-    const int nt = dq_tiles(i0, p.Nq, Lk, p.causal);
+    // key tiles j0 .. j0 + nt - 1 (the sliding window's first tile is j0);
+    // stages and phases count from 0
+    const int j0 = p.window_left >= 0 ? max(0, i0 + off - p.window_left) / kBlock : 0;
+    const int nt = max(0, dq_tiles(i0, p.Nq, Lk, p.causal) - j0);
 
     if (tid == 0) {
         ptx::mbar_init(&bars->q_full, 1);
@@ -617,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::mbar_arrive_expect_tx(&bars->k_full[st], kTile);
                     for (int c = 0; c < kDBlocks; ++c)
                         ptx::tma_load_4d(smem + L::kK + st * kTile + c * kBlockBytes, &tm_k,
-                                         &bars->k_full[st], c * 64, g, j * kBlock, b);
+                                         &bars->k_full[st], c * 64, g, (j0 + j) * kBlock, b);
                 }
                 __syncwarp();
                 ++issued_k;
@@ -629,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::mbar_arrive_expect_tx(&bars->v_full[st], kTile);
                     for (int c = 0; c < kDBlocks; ++c)
                         ptx::tma_load_4d(smem + L::kV + st * kTile + c * kBlockBytes, &tm_v,
-                                         &bars->v_full[st], c * 64, g, j * kBlock, b);
+                                         &bars->v_full[st], c * 64, g, (j0 + j) * kBlock, b);
                 }
                 __syncwarp();
                 ++issued_v;
@@ -751,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
             const int st = j % KST;
-            const int kc0 = j * kBlock + 32 * part;  // first key of this warp's columns
+            const int kc0 = (j0 + j) * kBlock + 32 * part;  // first key of this warp's columns
             if (!warp_wait(&bars->s_full[half], j & 1, p.limit_ns, abort_flag)) {
                 record_error(p.err, kErrBwdBase + 12, &bars->abort);
                 ok = false;
@@ -761,7 +774,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t sv[32], dv[32];
             ptx::tmem_ld32(t_s, sv);
             ptx::tmem_ld32(t_dp, dv);
-            const bool full = row_ok && kc0 + 32 <= Lk && (!p.causal || kc0 + 31 <= qi + off);
+            const bool full = row_ok && kc0 + 32 <= Lk && (!p.causal || kc0 + 31 <= qi + off) &&
+                              (p.window_left < 0 || kc0 >= qi + off - p.window_left);
             const bool masked = __any_sync(0xffffffffu, !full);
             ptx::tmem_wait_ld_dep(sv);
             ptx::tmem_wait_ld_dep(dv);
@@ -782,8 +796,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(p0, p1), d2), ds0, ds1);
                 if (masked) {
                     const int kj = kc0 + e;
-                    const bool v0 = row_ok && kj < Lk && (!p.causal || kj <= qi + off);
-                    const bool v1 = row_ok && kj + 1 < Lk && (!p.causal || kj + 1 <= qi + off);
+                    const bool w0 = p.window_left < 0 || kj >= qi + off - p.window_left;
+                    const bool w1 = p.window_left < 0 || kj + 1 >= qi + off - p.window_left;
+                    const bool v0 = row_ok && kj < Lk && (!p.causal || kj <= qi + off) && w0;
+                    const bool v1 = row_ok && kj + 1 < Lk && (!p.causal || kj + 1 <= qi + off) && w1;
                     ds0 = v0 ? ds0 : 0.f;
                     ds1 = v1 ? ds1 : 0.f;
                 }
@@ -794,7 +810,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // B operand of dS K), so that 0 * NaN cannot reach dQ; the quarter-0
             // warps of the half take its 64 rows (its S product is complete)
             const int krow = 64 * half + 32 * (part & 1) + lane;
-            if (quarter == 0 && j * kBlock + kBlock > Lk && j * kBlock + krow >= Lk) {
+            if (quarter == 0 && (j0 + j) * kBlock + kBlock > Lk && (j0 + j) * kBlock + krow >= Lk) {
                 uint8_t* kt = smem + L::kK + st * kTile;
 #pragma unroll
                 for (int c = 0; c < kDBlocks; ++c)

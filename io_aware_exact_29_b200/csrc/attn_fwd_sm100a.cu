@@ -111,10 +111,10 @@ __device__ __forceinline__ int tiles_for(int q_first, int Nq, int Lk, int causal
 
 // Running maxima of 64 score columns (two 32-column TMEM loads) into eight
 // independent chains of three-input maxima.  kMask: the tile reaches past
-// the row's last visible key (key_base + c > row_lim is masked).
+// the row's visible keys [row_first, row_lim] (others are masked).
 template <bool kMask>
-__device__ __forceinline__ void half_max(const uint32_t (&r)[2][32], int key_base, int row_lim,
-                                         float (&mx8)[8]) {
+__device__ __forceinline__ void half_max(const uint32_t (&r)[2][32], int key_base, int row_first,
+                                         int row_lim, float (&mx8)[8]) {
 #pragma unroll
     for (int c = 0; c < 64; c += 16) {
 #pragma unroll
@@ -123,8 +123,8 @@ __device__ __forceinline__ void half_max(const uint32_t (&r)[2][32], int key_bas
             float v0 = __uint_as_float(r[c0 >> 5][c0 & 31]);
             float v1 = __uint_as_float(r[c1 >> 5][c1 & 31]);
             if (kMask) {
-                if (key_base + c0 > row_lim) v0 = -INFINITY;
-                if (key_base + c1 > row_lim) v1 = -INFINITY;
+                if (key_base + c0 > row_lim || key_base + c0 < row_first) v0 = -INFINITY;
+                if (key_base + c1 > row_lim || key_base + c1 < row_first) v1 = -INFINITY;
             }
             mx8[u] = ptx::max3(mx8[u], v0, v1);
         }
@@ -135,7 +135,8 @@ __device__ __forceinline__ void half_max(const uint32_t (&r)[2][32], int key_bas
 // pair sums and packed two per 32-bit word (bf16 or fp16).  One pair in
 // kPolyEvery goes to the FMA pipe.
 template <bool kMask, bool BF16, int kPolyEvery>
-__device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_base, int row_lim,
+__device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_base,
+                                         int row_first, int row_lim,
                                          uint64_t sl2_2, uint64_t nm_2, uint64_t (&acc2)[4],
                                          uint32_t (&pk)[32]) {
 #pragma unroll
@@ -143,8 +144,8 @@ __device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_bas
         float v0 = __uint_as_float(r[c >> 5][c & 31]);
         float v1 = __uint_as_float(r[c >> 5][(c & 31) + 1]);
         if (kMask) {
-            if (key_base + c > row_lim) v0 = -INFINITY;
-            if (key_base + c + 1 > row_lim) v1 = -INFINITY;
+            if (key_base + c > row_lim || key_base + c < row_first) v0 = -INFINITY;
+            if (key_base + c + 1 > row_lim || key_base + c + 1 < row_first) v1 = -INFINITY;
         }
         const uint64_t t2 = ptx::f2_fma(ptx::f2_pack(v0, v1), sl2_2, nm_2);
         float p0, p1;
@@ -199,7 +200,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qbase = ct * 2 * kBlockM;
     const int nt0 = tiles_for(qbase, p.Nq, Lk, p.causal);
     const int nt1 = tiles_for(qbase + kBlockM, p.Nq, Lk, p.causal);
-    const int nt = max(nt0, nt1);
+    // sliding window: the first key tile each Q tile needs (tiles before it
+    // are never loaded); stages and phases count from the CTA's first tile
+    // jstart and from each Q tile's own first tile
+    const int qoff = Lk - p.Nq;  // query i's own key position is i + qoff
+    int j00 = 0, j01 = 0;
+    if (p.window_left >= 0) {
+        j00 = max(0, qbase + qoff - p.window_left) / kBlockN;
+        j01 = max(0, qbase + kBlockM + qoff - p.window_left) / kBlockN;
+    }
+    const int cnt0 = max(0, nt0 - j00), cnt1 = max(0, nt1 - j01);
+    const int jstart = cnt0 > 0 ? j00 : j01;
+    const int nt = max(cnt0 > 0 ? nt0 : 0, cnt1 > 0 ? nt1 : 0);
 
     if (tid == 0) {
         for (int a = 0; a < 2; ++a) {
@@ -241,16 +253,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             int issued_k = 0, issued_v = 0;
             bool issued_q[2] = {false, false};
             for (int a = 0; a < 2; ++a) {
-                if ((a == 0 ? nt0 : nt1) == 0) continue;
+                if ((a == 0 ? cnt0 : cnt1) == 0) continue;
                 ptx::mbar_arrive_expect_tx(&bars->q_full[a], kTileBytes);
                 for (int c = 0; c < kDBlocks; ++c)
                     ptx::tma_load_4d(smem + L::kQ + a * kTileBytes + c * kBlockBytes, &tm_q,
                                      &bars->q_full[a], c * 64, h, qbase + a * kBlockM, b);
                 issued_q[a] = true;
             }
-            for (int j = 0; j < nt; ++j) {
-                const int sk = j % KST;
-                if (!ptx::mbar_wait(&bars->k_empty[sk], ((j / KST) & 1) ^ 1, p.limit_ns,
+            for (int j = jstart; j < nt; ++j) {
+                const int t = j - jstart;
+                const int sk = t % KST;
+                if (!ptx::mbar_wait(&bars->k_empty[sk], ((t / KST) & 1) ^ 1, p.limit_ns,
                                     abort_flag)) {
                     record_error(p.err, kErrFwdBase + 1, &bars->abort);
                     break;
@@ -260,8 +273,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tma_load_4d(smem + L::kK + sk * kTileBytes + c * kBlockBytes, &tm_k,
                                      &bars->k_full[sk], c * 64, g, j * kBlockN, b);
                 ++issued_k;
-                const int sv = j % VST;
-                if (!ptx::mbar_wait(&bars->v_empty[sv], ((j / VST) & 1) ^ 1, p.limit_ns,
+                const int sv = t % VST;
+                if (!ptx::mbar_wait(&bars->v_empty[sv], ((t / VST) & 1) ^ 1, p.limit_ns,
                                     abort_flag)) {
                     record_error(p.err, kErrFwdBase + 2, &bars->abort);
                     break;
@@ -305,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tc_fence_after();
                     q_ready[a] = true;
                 }
-                const uint32_t k_addr = sbase + L::kK + (j % KST) * kTileBytes;
+                const uint32_t k_addr = sbase + L::kK + ((j - jstart) % KST) * kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
@@ -315,39 +328,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::umma_commit(&bars->s_full[a]);
             };
             auto issue_pv = [&](int a, int j) {
-                if (!wait_or_fail(&bars->p_full[a], j & 1, 5)) return;
-                if (!wait_or_fail(&bars->v_full[j % VST], (j / VST) & 1, 6)) return;
+                const int ja = a == 0 ? j00 : j01;  // the Q tile's first key tile
+                const int t = j - jstart;
+                if (!wait_or_fail(&bars->p_full[a], (j - ja) & 1, 5)) return;
+                if (!wait_or_fail(&bars->v_full[t % VST], (t / VST) & 1, 6)) return;
                 ptx::tc_fence_after();
-                const uint32_t v_addr = sbase + L::kV + (j % VST) * kTileBytes;
+                const uint32_t v_addr = sbase + L::kV + (t % VST) * kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < kBlockN / 16; ++kk) {
                     ptx::umma_ts(tmem + col_o[a], tmem + col_s[a] + kk * 8,
                                  ptx::sdesc_sw128(v_addr + kk * 16 * 128, kBlockBytes, 1024),
-                                 kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+                                 kIdescO, (j > ja || kk > 0) ? 1u : 0u);
                 }
                 if (j == (a == 0 ? nt0 : nt1) - 1) ptx::umma_commit(&bars->o_done[a]);
             };
-            for (int j = 0; ok && j <= nt; ++j) {
+            // key tile j is used by Q0 when j in [j00, nt0), by Q1 when j in
+            // [j01, nt1); a stage is released after its last user's product
+            auto use = [&](int a, int j) {
+                return a == 0 ? (cnt0 > 0 && j >= j00 && j < nt0)
+                              : (cnt1 > 0 && j >= j01 && j < nt1);
+            };
+            for (int j = jstart; ok && j <= nt; ++j) {
+                const int t = j - jstart;
                 if (j < nt) {
-                    if (!wait_or_fail(&bars->k_full[j % KST], (j / KST) & 1, 4)) break;
+                    if (!wait_or_fail(&bars->k_full[t % KST], (t / KST) & 1, 4)) break;
                     ptx::tc_fence_after();
-                    if (j < nt0) issue_s(0, j);
+                    if (use(0, j)) issue_s(0, j);
                     if (!ok) break;
                 }
-                if (j >= 1 && j - 1 < nt1) {
+                if (j > jstart && use(1, j - 1)) {
                     issue_pv(1, j - 1);
                     if (!ok) break;
-                    ptx::umma_commit(&bars->v_empty[(j - 1) % VST]);
+                    ptx::umma_commit(&bars->v_empty[(t - 1) % VST]);
                 }
                 if (j < nt) {
-                    if (j < nt1) issue_s(1, j);
+                    if (use(1, j)) issue_s(1, j);
                     if (!ok) break;
-                    ptx::umma_commit(&bars->k_empty[j % KST]);
-                    if (j < nt0) {
+                    ptx::umma_commit(&bars->k_empty[t % KST]);
+                    if (use(0, j)) {
                         issue_pv(0, j);
                         if (!ok) break;
-                        if (j >= nt1) ptx::umma_commit(&bars->v_empty[j % VST]);
                     }
+                    if (!use(1, j)) ptx::umma_commit(&bars->v_empty[t % VST]);
                 }
             }
             if (!ok) {
@@ -361,7 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ================================================= softmax warpgroups
         const int a = warp >> 2;  // which Q tile
-        const int nta = a == 0 ? nt0 : nt1;
+        const int nta = a == 0 ? (cnt0 > 0 ? nt0 : 0) : (cnt1 > 0 ? nt1 : 0);
+        const int ja = a == 0 ? j00 : j01;  // its first key tile
         const uint32_t quarter = (uint32_t)(warp & 3);
         const uint32_t row = quarter * 32u + (uint32_t)lane;
         const uint32_t lane_addr = (quarter * 32u) << 16;
@@ -369,6 +392,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int i = qa + (int)row;
         int row_lim = Lk - 1;  // last visible key of this row
         if (p.causal) row_lim = min(row_lim, i + Lk - p.Nq);
+        // first visible key of this row (the sliding window's lower edge)
+        const int row_first = p.window_left >= 0 ? i + qoff - p.window_left : -(1 << 30);
         const float sl2 = p.scale_log2;
         float m_ref = -INFINITY;  // running reference max, scale*log2 units
         float l_sum = 0.f;        // running sum of exp2(s*sl2 - m_ref)
@@ -376,15 +401,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_s = tmem + lane_addr + (a == 0 ? 0u : 128u);
         const uint32_t t_o = tmem + lane_addr + (a == 0 ? 256u : 256u + D);
 
-        for (int j = 0; j < nta; ++j) {
-            if (!warp_wait(&bars->s_full[a], j & 1, p.limit_ns, abort_flag)) {
+        for (int j = ja; j < nta; ++j) {
+            if (!warp_wait(&bars->s_full[a], (j - ja) & 1, p.limit_ns, abort_flag)) {
                 record_error(p.err, kErrFwdBase + 7, &bars->abort);
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
             const int key0 = j * kBlockN;
-            const bool masked = key0 + kBlockN - 1 > row_lim;
+            const bool masked = key0 + kBlockN - 1 > row_lim || key0 < row_first;
             // pass 1: row maximum, two halves of 64 columns, eight independent
             // chains of three-input maxima
             float mx8[8];
@@ -402,9 +427,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tmem_wait_ld_dep(r[hf][0]);
                     ptx::tmem_wait_ld_dep(r[hf][1]);
                     if (masked)
-                        half_max<true>(r[hf], key0 + hf * 64, row_lim, mx8);
+                        half_max<true>(r[hf], key0 + hf * 64, row_first, row_lim, mx8);
                     else
-                        half_max<false>(r[hf], key0 + hf * 64, row_lim, mx8);
+                        half_max<false>(r[hf], key0 + hf * 64, row_first, row_lim, mx8);
                 }
             }
             const float mx = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]),
@@ -414,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool rescale = false;
             if (m_tile > m_ref + kRescaleThreshold) {
                 alpha = ptx::ex2_approx(m_ref - m_tile);  // 0 when m_ref = -inf
-                rescale = (j > 0) && (m_ref != -INFINITY);
+                rescale = (j > ja) && (m_ref != -INFINITY);
                 m_ref = m_tile;
             }
             const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
@@ -432,11 +457,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tmem_wait_ld_dep(r[1]);
                 uint32_t pk[32];
                 if (masked)
-                    half_exp<true, BF16, kPolyEvery>(r, key0 + hf * 64, row_lim, sl2_2, nm_2, acc2,
-                                                     pk);
+                    half_exp<true, BF16, kPolyEvery>(r, key0 + hf * 64, row_first, row_lim, sl2_2,
+                                                     nm_2, acc2, pk);
                 else
-                    half_exp<false, BF16, kPolyEvery>(r, key0 + hf * 64, row_lim, sl2_2, nm_2,
-                                                      acc2, pk);
+                    half_exp<false, BF16, kPolyEvery>(r, key0 + hf * 64, row_first, row_lim, sl2_2,
+                                                      nm_2, acc2, pk);
                 ptx::tmem_st32(t_s + hf * 32, pk);
             }
             float s0, s1, s2, s3, s4, s5, s6, s7;
@@ -462,13 +487,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tmem_wait_st();
             }
             ptx::tmem_wait_st();
+            // the Q tile that uses key tile j first zeroes its V rows behind
+            // the real length (Q0 if it uses the tile, else Q1)
             const bool zero_v = p.seqlens_k != nullptr && key0 + kBlockN > Lk &&
-                                (a == 0 ? true : j >= nt0);
+                                (a == 0 ? true : (cnt0 == 0 || j >= nt0));
             if (zero_v) {
                 // keys behind the real length: zero their V rows so that a
                 // non-finite value stored there cannot reach O through 0 * NaN
-                const int sv = j % VST;
-                if (!warp_wait(&bars->v_full[sv], (j / VST) & 1, p.limit_ns, abort_flag)) {
+                const int sv = (j - jstart) % VST;
+                if (!warp_wait(&bars->v_full[sv], ((j - jstart) / VST) & 1, p.limit_ns,
+                               abort_flag)) {
                     record_error(p.err, kErrFwdBase + 8, &bars->abort);
                     ok = false;
                     break;

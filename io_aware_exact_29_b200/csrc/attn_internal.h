@@ -22,6 +22,7 @@ struct FwdParams {
     int causal;
     float scale_log2; // scale * log2(e)
     const int* seqlens_k;  // [B] or nullptr
+    int window_left;       // -1, or keys before i + (Lk - Nq) - window_left are masked
     float* lse;            // [B, Hq, Nq]
     unsigned long long limit_ns;
     int inject;       // self-test: the loader skips everything
@@ -43,6 +44,7 @@ struct BwdParams {
     float scale;
     float scale_log2;      // scale * log2(e)
     const int* seqlens_k;  // [B] or nullptr
+    int window_left;       // -1, or keys before i + (Lk - Nq) - window_left are masked
     const void* o;         // [B, Nq, Hq, d] forward output
     const void* dout;      // [B, Nq, Hq, d]
     const float* lse;      // [B, Hq, Nq] forward log-sum-exp (natural log)
