@@ -112,7 +112,7 @@ __device__ __forceinline__ int tiles_for(int q_first, int Nq, int Lk, int causal
 // Running maxima of 64 score columns (two 32-column TMEM loads) into eight
 // independent chains of three-input maxima.  kMask: the tile reaches past
 // the row's visible keys [row_first, row_lim] (others are masked).
-template <bool kMask>
+template <bool kMask, bool kLow>
 __device__ __forceinline__ void half_max(const uint32_t (&r)[2][32], int key_base, int row_first,
                                          int row_lim, float (&mx8)[8]) {
 #pragma unroll
@@ -123,8 +123,8 @@ __device__ __forceinline__ void half_max(const uint32_t (&r)[2][32], int key_bas
             float v0 = __uint_as_float(r[c0 >> 5][c0 & 31]);
             float v1 = __uint_as_float(r[c1 >> 5][c1 & 31]);
             if (kMask) {
-                if (key_base + c0 > row_lim || key_base + c0 < row_first) v0 = -INFINITY;
-                if (key_base + c1 > row_lim || key_base + c1 < row_first) v1 = -INFINITY;
+                if (key_base + c0 > row_lim || (kLow && key_base + c0 < row_first)) v0 = -INFINITY;
+                if (key_base + c1 > row_lim || (kLow && key_base + c1 < row_first)) v1 = -INFINITY;
             }
             mx8[u] = ptx::max3(mx8[u], v0, v1);
         }
@@ -134,7 +134,7 @@ __device__ __forceinline__ void half_max(const uint32_t (&r)[2][32], int key_bas
 // p = 2^(s * scale_log2 - m) for 64 score columns, accumulated into four
 // pair sums and packed two per 32-bit word (bf16 or fp16).  One pair in
 // kPolyEvery goes to the FMA pipe.
-template <bool kMask, bool BF16, int kPolyEvery>
+template <bool kMask, bool kLow, bool BF16, int kPolyEvery>
 __device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_base,
                                          int row_first, int row_lim,
                                          uint64_t sl2_2, uint64_t nm_2, uint64_t (&acc2)[4],
@@ -144,8 +144,9 @@ __device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_bas
         float v0 = __uint_as_float(r[c >> 5][c & 31]);
         float v1 = __uint_as_float(r[c >> 5][(c & 31) + 1]);
         if (kMask) {
-            if (key_base + c > row_lim || key_base + c < row_first) v0 = -INFINITY;
-            if (key_base + c + 1 > row_lim || key_base + c + 1 < row_first) v1 = -INFINITY;
+            if (key_base + c > row_lim || (kLow && key_base + c < row_first)) v0 = -INFINITY;
+            if (key_base + c + 1 > row_lim || (kLow && key_base + c + 1 < row_first))
+                v1 = -INFINITY;
         }
         const uint64_t t2 = ptx::f2_fma(ptx::f2_pack(v0, v1), sl2_2, nm_2);
         float p0, p1;
@@ -165,7 +166,7 @@ __device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_bas
     }
 }
 
-template <int D, bool BF16, int KST, int VST>
+template <int D, bool BF16, int KST, int VST, bool kWindow>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -205,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // jstart and from each Q tile's own first tile
     const int qoff = Lk - p.Nq;  // query i's own key position is i + qoff
     int j00 = 0, j01 = 0;
-    if (p.window_left >= 0) {
+    if constexpr (kWindow) {  // kWindow: the instance launched for window_left >= 0
         j00 = max(0, qbase + qoff - p.window_left) / kBlockN;
         j01 = max(0, qbase + kBlockM + qoff - p.window_left) / kBlockN;
     }
@@ -393,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int row_lim = Lk - 1;  // last visible key of this row
         if (p.causal) row_lim = min(row_lim, i + Lk - p.Nq);
         // first visible key of this row (the sliding window's lower edge)
-        const int row_first = p.window_left >= 0 ? i + qoff - p.window_left : -(1 << 30);
+        const int row_first = kWindow ? i + qoff - p.window_left : 0;
         const float sl2 = p.scale_log2;
         float m_ref = -INFINITY;  // running reference max, scale*log2 units
         float l_sum = 0.f;        // running sum of exp2(s*sl2 - m_ref)
@@ -409,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ptx::tc_fence_after();
             const int key0 = j * kBlockN;
-            const bool masked = key0 + kBlockN - 1 > row_lim || key0 < row_first;
+            const bool masked = key0 + kBlockN - 1 > row_lim || (kWindow && key0 < row_first);
             // pass 1: row maximum, two halves of 64 columns, eight independent
             // chains of three-input maxima
             float mx8[8];
@@ -427,9 +428,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tmem_wait_ld_dep(r[hf][0]);
                     ptx::tmem_wait_ld_dep(r[hf][1]);
                     if (masked)
-                        half_max<true>(r[hf], key0 + hf * 64, row_first, row_lim, mx8);
+                        half_max<true, kWindow>(r[hf], key0 + hf * 64, row_first, row_lim, mx8);
                     else
-                        half_max<false>(r[hf], key0 + hf * 64, row_first, row_lim, mx8);
+                        half_max<false, kWindow>(r[hf], key0 + hf * 64, row_first, row_lim, mx8);
                 }
             }
             const float mx = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]),
@@ -457,10 +458,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tmem_wait_ld_dep(r[1]);
                 uint32_t pk[32];
                 if (masked)
-                    half_exp<true, BF16, kPolyEvery>(r, key0 + hf * 64, row_first, row_lim, sl2_2,
+                    half_exp<true, kWindow, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
+                                                              row_lim, sl2_2,
                                                      nm_2, acc2, pk);
                 else
-                    half_exp<false, BF16, kPolyEvery>(r, key0 + hf * 64, row_first, row_lim, sl2_2,
+                    half_exp<false, kWindow, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
+                                                               row_lim, sl2_2,
                                                       nm_2, acc2, pk);
                 ptx::tmem_st32(t_s + hf * 32, pk);
             }
@@ -578,17 +581,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int D, bool BF16, int KST, int VST>
-cudaError_t launch_fwd_t(const FwdMaps& maps, const FwdParams& p, cudaStream_t stream) {
+template <int D, bool BF16, int KST, int VST, bool kWindow>
+cudaError_t launch_fwd_w(const FwdMaps& maps, const FwdParams& p, cudaStream_t stream) {
     using L = FwdSmem<D, KST, VST>;
     static_assert(L::kAlloc <= 227 * 1024, "shared memory budget");
-    auto kern = attn_fwd_kernel<D, BF16, KST, VST>;
+    auto kern = attn_fwd_kernel<D, BF16, KST, VST, kWindow>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc);
     if (e != cudaSuccess) return e;
     dim3 grid((p.Nq + 2 * kBlockM - 1) / (2 * kBlockM), p.Hq, p.B);
     kern<<<grid, kThreads, L::kAlloc, stream>>>(maps.q, maps.k, maps.v, maps.o, p);
     return cudaGetLastError();
+}
+
+// the sliding-window masks and tile ranges are compiled only into the
+// instance that a window call launches
+template <int D, bool BF16, int KST, int VST>
+cudaError_t launch_fwd_t(const FwdMaps& maps, const FwdParams& p, cudaStream_t stream) {
+    return p.window_left >= 0 ? launch_fwd_w<D, BF16, KST, VST, true>(maps, p, stream)
+                              : launch_fwd_w<D, BF16, KST, VST, false>(maps, p, stream);
 }
 
 }  // namespace
