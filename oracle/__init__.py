@@ -33,6 +33,10 @@ _lib = None
 
 _DP = ctypes.POINTER(ctypes.c_double)
 _IP = ctypes.POINTER(ctypes.c_int)
+_U8P = ctypes.POINTER(ctypes.c_ubyte)
+# block_mask, mask_sb, mask_sh, mask_nqb, mask_nkb, block_m, block_n
+_MASK_ARGS = [_U8P, ctypes.c_long, ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+              ctypes.c_int]
 
 
 def build(force: bool = False) -> str:
@@ -71,6 +75,10 @@ def _load():
                 _DP, _DP, _DP, _DP, _DP, _DP, _DP, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, _IP,
                 ctypes.c_int]
+            lib.oracle_attn_fwd_mask.restype = ctypes.c_int
+            lib.oracle_attn_fwd_mask.argtypes = lib.oracle_attn_fwd.argtypes + _MASK_ARGS
+            lib.oracle_attn_bwd_mask.restype = ctypes.c_int
+            lib.oracle_attn_bwd_mask.argtypes = lib.oracle_attn_bwd.argtypes + _MASK_ARGS
             lib.oracle_attn_paged.restype = ctypes.c_int
             lib.oracle_attn_paged.argtypes = [
                 _DP, _DP, _DP, _IP, ctypes.c_int, ctypes.c_int, ctypes.c_int, _IP, _DP, _DP,
@@ -103,6 +111,27 @@ def _ip(a):
     return None if a is None else a.ctypes.data_as(_IP)
 
 
+def _block_mask_args(block_mask, block_size, B, Hq):
+    """(array kept alive, ctypes argument tuple) for an optional block mask.
+
+    block_mask: [Bm, Hm, nqb, nkb] with Bm in {1, B} and Hm in {1, Hq} (a
+    size-1 dimension is shared); nonzero = the block's keys take part.
+    block_size: int or (block_m, block_n).
+    """
+    if block_mask is None:
+        return None, (None, 0, 0, 0, 0, 1, 1)
+    if isinstance(block_mask, torch.Tensor):
+        block_mask = block_mask.detach().to("cpu").numpy()
+    m = np.ascontiguousarray(np.asarray(block_mask) != 0, dtype=np.uint8)
+    if m.ndim != 4 or m.shape[0] not in (1, B) or m.shape[1] not in (1, Hq):
+        raise ValueError(f"block_mask shape {m.shape} is not [1|B, 1|Hq, nqb, nkb]")
+    bm, bn = (block_size, block_size) if isinstance(block_size, int) else block_size
+    nqb, nkb = m.shape[2], m.shape[3]
+    sh = 0 if m.shape[1] == 1 else nqb * nkb
+    sb = 0 if m.shape[0] == 1 else m.shape[1] * nqb * nkb
+    return m, (m.ctypes.data_as(_U8P), sb, sh, nqb, nkb, int(bm), int(bn))
+
+
 def max_threads() -> int:
     return int(_load().oracle_max_threads())
 
@@ -111,13 +140,17 @@ def set_threads(n: int) -> None:
     _load().oracle_set_threads(int(n))
 
 
-def attn_fwd(q, k, v, scale: float, causal: bool, seqlens_k=None, rows=None, window_left=-1):
+def attn_fwd(q, k, v, scale: float, causal: bool, seqlens_k=None, rows=None, window_left=-1,
+             block_mask=None, block_size=128):
     """O, LSE of dense attention.
 
     q [B, Nq, Hq, d], k/v [B, Nk, Hkv, d] (any float dtype; widened exactly).
     seqlens_k: optional [B] key lengths (keys at or past it are masked).
     window_left: -1, or the sliding window: keys more than window_left
     positions before the query's own position i + (Lk - Nq) are masked.
+    block_mask: optional [1|B, 1|Hq, nqb, nkb]; a zero entry masks the keys
+    of block (i // block_m, j // block_n) for those queries (block_size is
+    block_m = block_n, or a pair).
     rows: optional list of query-row indices; only those rows are computed
     (the other entries of the returned arrays are NaN).
     Returns (o [B, Nq, Hq, d] float64, lse [B, Hq, Nq] float64) numpy arrays.
@@ -129,9 +162,12 @@ def attn_fwd(q, k, v, scale: float, causal: bool, seqlens_k=None, rows=None, win
     lse = np.full((B, Hq, Nq), np.nan)
     sl = None if seqlens_k is None else _i32(seqlens_k)
     rw = None if rows is None else _i32(rows)
-    rc = _load().oracle_attn_fwd(_dp(qd), _dp(kd), _dp(vd), _dp(o), _dp(lse), B, Hq, Hkv, Nq,
-                                 Nk, d, float(scale), int(bool(causal)), _ip(sl), _ip(rw),
-                                 0 if rw is None else len(rw), int(window_left))
+    keep, margs = _block_mask_args(block_mask, block_size, B, Hq)
+    rc = _load().oracle_attn_fwd_mask(_dp(qd), _dp(kd), _dp(vd), _dp(o), _dp(lse), B, Hq, Hkv,
+                                      Nq, Nk, d, float(scale), int(bool(causal)), _ip(sl),
+                                      _ip(rw), 0 if rw is None else len(rw), int(window_left),
+                                      *margs)
+    del keep
     if rc != 0:
         raise ValueError(f"oracle_attn_fwd rejected its arguments (rc={rc})")
     return o, lse
@@ -173,10 +209,12 @@ def lse_combine(o_parts, lse_parts):
     return o, lse
 
 
-def attn_bwd(q, k, v, dout, scale: float, causal: bool, seqlens_k=None, window_left=-1):
+def attn_bwd(q, k, v, dout, scale: float, causal: bool, seqlens_k=None, window_left=-1,
+             block_mask=None, block_size=128):
     """Gradients (dq, dk, dv) of L = sum(dout * O) for O = attention(q, k, v).
 
-    q, dout [B, Nq, Hq, d]; k, v [B, Nk, Hkv, d]; seqlens_k optional [B].
+    q, dout [B, Nq, Hq, d]; k, v [B, Nk, Hkv, d]; seqlens_k optional [B];
+    window_left, block_mask, block_size as in attn_fwd.
     Returns float64 numpy arrays dq [B, Nq, Hq, d], dk and dv [B, Nk, Hkv, d]
     (dk, dv summed over the query heads that share a kv head; zero behind a
     sequence's real key length).
@@ -188,9 +226,11 @@ def attn_bwd(q, k, v, dout, scale: float, causal: bool, seqlens_k=None, window_l
     dk = np.full((B, Nk, Hkv, d), np.nan)
     dv = np.full((B, Nk, Hkv, d), np.nan)
     sl = None if seqlens_k is None else _i32(seqlens_k)
-    rc = _load().oracle_attn_bwd(_dp(qd), _dp(kd), _dp(vd), _dp(dod), _dp(dq), _dp(dk), _dp(dv),
-                                 B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), _ip(sl),
-                                 int(window_left))
+    keep, margs = _block_mask_args(block_mask, block_size, B, Hq)
+    rc = _load().oracle_attn_bwd_mask(_dp(qd), _dp(kd), _dp(vd), _dp(dod), _dp(dq), _dp(dk),
+                                      _dp(dv), B, Hq, Hkv, Nq, Nk, d, float(scale),
+                                      int(bool(causal)), _ip(sl), int(window_left), *margs)
+    del keep
     if rc != 0:
         raise ValueError(f"oracle_attn_bwd rejected its arguments (rc={rc})")
     return dq, dk, dv

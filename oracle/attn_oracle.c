@@ -36,7 +36,10 @@
  *  - grouped-query heads map contiguously: g = h / (Hq / Hkv);
  *  - a sliding window (window_left >= 0) also masks keys more than
  *    window_left positions before the query's own position i + (Lk - Nq)
- *    (the "extensions for masks" the pages list as a direction); -1 = none.
+ *    (the "extensions for masks" the pages list as a direction); -1 = none;
+ *  - a block mask (the other mask extension: block-sparse attention) cuts
+ *    the (query, key) plane into blocks of block_m rows by block_n keys and
+ *    masks every key of a block whose entry is 0, on top of the other rules.
  *
  * Arithmetic: every input is fp64 (the caller widens the bf16/fp16 bits
  * exactly).  Row sums and output sums use Neumaier compensated summation so
@@ -77,6 +80,39 @@ static int key_visible(int i, int j, int Nq, int Lk, int causal, int window_left
     return 1;
 }
 
+/* ---- the block mask of one (batch, head) ---------------------------------
+ * m == NULL: no block mask.  Otherwise block (i / bm, j / bn) is
+ * m[(i / bm) * nkb + j / bn]; 0 masks every key of the block. */
+typedef struct {
+    const unsigned char* m;
+    int nkb, bm, bn;
+} bmask_t;
+
+static const bmask_t nomask = {NULL, 0, 1, 1};
+
+static int block_on(const bmask_t* mk, int i, int j) {
+    if (!mk->m) return 1;
+    return mk->m[(size_t)(i / mk->bm) * (size_t)mk->nkb + (size_t)(j / mk->bn)] != 0;
+}
+
+/* the block mask of (b, h) inside a [B?, H?, nqb, nkb] array with strides sb, sh */
+static bmask_t head_mask(const unsigned char* mask, long sb, long sh, int nkb, int bm, int bn,
+                         int b, int h) {
+    bmask_t r = {NULL, nkb, bm, bn};
+    if (mask) r.m = mask + (size_t)b * (size_t)sb + (size_t)h * (size_t)sh;
+    return r;
+}
+
+/* mask arguments: NULL mask, or block sizes > 0, rows and columns of blocks
+ * that cover Nq x Nk, non-negative strides */
+static int mask_args_ok(const unsigned char* mask, long sb, long sh, int nqb, int nkb, int bm,
+                        int bn, int Nq, int Nk) {
+    if (!mask) return 1;
+    if (bm <= 0 || bn <= 0 || sb < 0 || sh < 0) return 0;
+    if ((long)nqb * bm < Nq || (long)nkb * bn < Nk) return 0;
+    return 1;
+}
+
 /* ---- one query head against one key/value head --------------------------
  * q_rows[r]   : pointer to the d values of the r-th requested query row
  * row_index[r]: that row's index i in [0, Nq), used by the causal rule
@@ -86,7 +122,7 @@ static int key_visible(int i, int j, int Nq, int Lk, int causal, int window_left
  */
 static void attend_head(int nrows, const double* const* q_rows, const int* row_index,
                         const double* k, const double* v, long kv_stride, int Nq, int Lk,
-                        int d, double scale, int causal, int window_left,
+                        int d, double scale, int causal, int window_left, const bmask_t* mk,
                         double* const* o_rows, double* const* lse_out, double* S) {
     for (int r = 0; r < nrows; ++r) {
         const double* qi = q_rows[r];
@@ -94,7 +130,8 @@ static void attend_head(int nrows, const double* const* q_rows, const int* row_i
         double* Srow = S + (size_t)r * (size_t)(Lk > 0 ? Lk : 1);
         /* step 1 + 2: scores, then the additive 0 / -inf mask */
         for (int j = 0; j < Lk; ++j) {
-            const int visible = key_visible(i, j, Nq, Lk, causal, window_left);
+            const int visible = key_visible(i, j, Nq, Lk, causal, window_left) &&
+                                block_on(mk, i, j);
             if (!visible) {
                 Srow[j] = -INFINITY;
                 continue;
@@ -180,12 +217,22 @@ void oracle_set_threads(int n) {
  *              point on the ai6s.net page).
  *   rows, nrows: NULL/0 computes every query row; otherwise only the listed
  *              row indices, for every (b, h); other outputs are left alone.
+ *   window_left: -1, or the sliding window described at the top.
+ *   block_mask: NULL, or the block mask of (b, h) at
+ *              block_mask + b * mask_sb + h * mask_sh, mask_nqb rows of
+ *              mask_nkb entries (blocks of block_m queries by block_n keys;
+ *              a zero stride shares one mask across batches or heads).
  * Returns 0, or -1 on bad arguments.
  */
-int oracle_attn_fwd(const double* q, const double* k, const double* v, double* o, double* lse,
-                    int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale, int causal,
-                    const int* seqlens_k, const int* rows, int nrows, int window_left) {
+int oracle_attn_fwd_mask(const double* q, const double* k, const double* v, double* o,
+                         double* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                         double scale, int causal, const int* seqlens_k, const int* rows,
+                         int nrows, int window_left, const unsigned char* block_mask,
+                         long mask_sb, long mask_sh, int mask_nqb, int mask_nkb, int block_m,
+                         int block_n) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || d <= 0 || Hq % Hkv != 0) return -1;
+    if (!mask_args_ok(block_mask, mask_sb, mask_sh, mask_nqb, mask_nkb, block_m, block_n, Nq, Nk))
+        return -1;
     if (seqlens_k)
         for (int b = 0; b < B; ++b)
             if (seqlens_k[b] < 0 || seqlens_k[b] > Nk) return -1;
@@ -219,8 +266,10 @@ int oracle_attn_fwd(const double* q, const double* k, const double* v, double* o
             }
             const double* kb = k + ((size_t)b * Nk * Hkv + g) * (size_t)d;
             const double* vb = v + ((size_t)b * Nk * Hkv + g) * (size_t)d;
+            const bmask_t mk =
+                head_mask(block_mask, mask_sb, mask_sh, mask_nkb, block_m, block_n, b, h);
             attend_head(nr, qp, ri, kb, vb, (long)Hkv * d, Nq, Lk, d, scale, causal, window_left,
-                        op, lp, S);
+                        &mk, op, lp, S);
         }
         free(S);
         free(qp);
@@ -229,6 +278,14 @@ int oracle_attn_fwd(const double* q, const double* k, const double* v, double* o
         free(ri);
     }
     return err ? -2 : 0;
+}
+
+/* oracle_attn_fwd_mask without a block mask */
+int oracle_attn_fwd(const double* q, const double* k, const double* v, double* o, double* lse,
+                    int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale, int causal,
+                    const int* seqlens_k, const int* rows, int nrows, int window_left) {
+    return oracle_attn_fwd_mask(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, seqlens_k,
+                                rows, nrows, window_left, NULL, 0, 0, 0, 0, 1, 1);
 }
 
 /*
@@ -276,7 +333,8 @@ int oracle_attn_kvcache(const double* q, const double* k_cache, const double* v_
             }
             const double* kb = k_cache + ((size_t)cu_seqlens_k[b] * Hkv + g) * (size_t)d;
             const double* vb = v_cache + ((size_t)cu_seqlens_k[b] * Hkv + g) * (size_t)d;
-            attend_head(Nq, qp, ri, kb, vb, (long)Hkv * d, Nq, Lk, d, scale, causal, -1, op, lp,
+            attend_head(Nq, qp, ri, kb, vb, (long)Hkv * d, Nq, Lk, d, scale, causal, -1, &nomask,
+                        op, lp,
                         S);
         }
         free(S);
@@ -350,13 +408,18 @@ int oracle_lse_combine(const double* o_parts, const double* lse_parts, int npart
  * contributes nothing.  P is recomputed here from q, k, v (no forward output
  * or LSE is taken from the caller).  Every sum is compensated (Neumaier).
  *   q, dout, dq [B, Nq, Hq, d]   k, v, dk, dv [B, Nk, Hkv, d]   seqlens_k: NULL or [B]
+ *   window_left, block_mask and its layout: as in oracle_attn_fwd_mask.
  * Work is split over (b, g) so that the sums over the heads of a group are
  * done by one thread in head order.  Returns 0, -1 (bad arguments) or -2.
  */
-int oracle_attn_bwd(const double* q, const double* k, const double* v, const double* dout,
-                    double* dq, double* dk, double* dv, int B, int Hq, int Hkv, int Nq, int Nk,
-                    int d, double scale, int causal, const int* seqlens_k, int window_left) {
+int oracle_attn_bwd_mask(const double* q, const double* k, const double* v, const double* dout,
+                         double* dq, double* dk, double* dv, int B, int Hq, int Hkv, int Nq,
+                         int Nk, int d, double scale, int causal, const int* seqlens_k,
+                         int window_left, const unsigned char* block_mask, long mask_sb,
+                         long mask_sh, int mask_nqb, int mask_nkb, int block_m, int block_n) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || d <= 0 || Hq % Hkv != 0) return -1;
+    if (!mask_args_ok(block_mask, mask_sb, mask_sh, mask_nqb, mask_nkb, block_m, block_n, Nq, Nk))
+        return -1;
     if (seqlens_k)
         for (int b = 0; b < B; ++b)
             if (seqlens_k[b] < 0 || seqlens_k[b] > Nk) return -1;
@@ -383,6 +446,8 @@ int oracle_attn_bwd(const double* q, const double* k, const double* v, const dou
             const double* vb = v + ((size_t)b * Nk * Hkv + g) * (size_t)d;
             for (int hh = 0; hh < G; ++hh) {
                 const int h = g * G + hh;
+                const bmask_t mk =
+                    head_mask(block_mask, mask_sb, mask_sh, mask_nkb, block_m, block_n, b, h);
                 for (int i = 0; i < Nq; ++i) {
                     const double* qi = q + (((size_t)b * Nq + i) * Hq + h) * (size_t)d;
                     const double* doi = dout + (((size_t)b * Nq + i) * Hq + h) * (size_t)d;
@@ -391,7 +456,8 @@ int oracle_attn_bwd(const double* q, const double* k, const double* v, const dou
                     /* P row: scores, mask, softmax */
                     double m = -INFINITY;
                     for (int j = 0; j < Lk; ++j) {
-                        const int visible = key_visible(i, j, Nq, Lk, causal, window_left);
+                        const int visible = key_visible(i, j, Nq, Lk, causal, window_left) &&
+                                            block_on(&mk, i, j);
                         if (!visible) {
                             Prow[j] = -INFINITY;
                             continue;
@@ -473,6 +539,14 @@ int oracle_attn_bwd(const double* q, const double* k, const double* v, const dou
     return err ? -2 : 0;
 }
 
+/* oracle_attn_bwd_mask without a block mask */
+int oracle_attn_bwd(const double* q, const double* k, const double* v, const double* dout,
+                    double* dq, double* dk, double* dv, int B, int Hq, int Hkv, int Nq, int Nk,
+                    int d, double scale, int causal, const int* seqlens_k, int window_left) {
+    return oracle_attn_bwd_mask(q, k, v, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                                seqlens_k, window_left, NULL, 0, 0, 0, 0, 1, 1);
+}
+
 /*
  * Attention of new query tokens against a PAGED KV cache: the cache is cut
  * into fixed blocks of block_size rows and sequence b's logical key j lives
@@ -539,7 +613,8 @@ int oracle_attn_paged(const double* q, const double* k_cache, const double* v_ca
                 op[i] = o + (((size_t)b * Nq + i) * Hq + h) * (size_t)d;
                 lp[i] = lse + ((size_t)b * Hq + h) * (size_t)Nq + i;
             }
-            attend_head(Nq, qp, ri, kg, vg, (long)d, Nq, Lk, d, scale, causal, -1, op, lp, S);
+            attend_head(Nq, qp, ri, kg, vg, (long)d, Nq, Lk, d, scale, causal, -1, &nomask, op, lp,
+                        S);
         }
         free(S);
         free(kg);

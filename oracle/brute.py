@@ -11,12 +11,14 @@ from __future__ import annotations
 import math
 
 
-def attention_rows(q, k, v, scale, causal=False, lk=None, window_left=None):
+def attention_rows(q, k, v, scale, causal=False, lk=None, window_left=None, blocks=None,
+                   block=(1, 1)):
     """q: list of Nq rows, k/v: lists of Nk rows (lists of floats).
 
     Returns (o, lse): o is a list of Nq output rows, lse a list of Nq floats.
     Key j is visible to query i iff j < lk and (not causal or j <= i + lk - Nq)
-    and (window_left is None or j >= i + lk - Nq - window_left).
+    and (window_left is None or j >= i + lk - Nq - window_left) and (blocks
+    is None or blocks[i // block[0]][j // block[1]] is true).
     """
     nq = len(q)
     nk = len(k) if lk is None else lk
@@ -28,6 +30,8 @@ def attention_rows(q, k, v, scale, causal=False, lk=None, window_left=None):
             if causal and j > i + nk - nq:
                 continue
             if window_left is not None and j < i + nk - nq - window_left:
+                continue
+            if blocks is not None and not blocks[i // block[0]][j // block[1]]:
                 continue
             s = 0.0
             for t in range(d):
