@@ -101,6 +101,35 @@ ATTN_API int attn_fwd_window(const void* q, const void* k, const void* v, void* 
                              int causal, int window_left, int dtype, const int* seqlens_k,
                              void* stream);
 
+/* Rows and keys per entry of a block mask (the kernels' tile sizes). */
+#define ATTN_MASK_BLOCK 128
+
+/*
+ * Block-sparse forward attention: as attn_fwd_window (window_left -1 = none,
+ * seqlens_k may be NULL), plus a block mask that removes whole 128 x 128
+ * blocks of (query, key) pairs.  The pages name mask extensions as a
+ * direction without a form (machinelearning.ru page, "directions"); this is
+ * the block-granular one, which the tile loop can skip without touching the
+ * skipped keys.
+ *   block_mask: device bytes, owned by the caller; the entry for batch b,
+ *     query head h, query block qb = i / ATTN_MASK_BLOCK and key block
+ *     kb = j / ATTN_MASK_BLOCK is block_mask[b * mask_stride_b +
+ *     h * mask_stride_h + qb * mask_stride_row + kb].  Nonzero: the block
+ *     takes part (subject to the causal, length and window rules); 0: every
+ *     key of the block is masked for those queries and its K/V rows are not
+ *     read for them.  Strides count bytes; 0 shares one mask across batches
+ *     or heads.  mask_stride_row >= ceil(Nk / 128); ceil(Nq / 128) rows.
+ * A row whose visible keys are all masked gives O = 0, LSE = -inf.
+ * Returns the status codes of attn_fwd (ATTN_ERR_INVALID_ARG for a NULL
+ * mask, a negative stride or a row stride below the key-block count).
+ */
+ATTN_API int attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* o,
+                                  float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                                  float scale, int causal, int window_left, int dtype,
+                                  const int* seqlens_k, const unsigned char* block_mask,
+                                  long long mask_stride_b, long long mask_stride_h,
+                                  int mask_stride_row, void* stream);
+
 /*
  * Bytes of device workspace that attn_fwd_varlen_kvcache needs for these
  * sizes.  split_keys: keys per split-K work unit, a multiple of 64, or 0 to

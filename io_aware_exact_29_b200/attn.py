@@ -50,6 +50,10 @@ def load_library():
             lib.attn_fwd_window.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp,
                                             vp]
             lib.attn_fwd_window.restype = i
+            ll = ctypes.c_longlong
+            lib.attn_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i,
+                                                 vp, vp, ll, ll, i, vp]
+            lib.attn_fwd_blocksparse.restype = i
             lib.attn_bwd_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i,
                                             f, i, i, i, vp, vp, sz, vp]
             lib.attn_bwd_window.restype = i
@@ -107,13 +111,40 @@ def _dev(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
 
 
+MASK_BLOCK = 128  # queries and keys per block-mask entry
+
+
+def block_mask_args(block_mask, B, Hq, Nq, Nk):
+    """(pointer, stride_b, stride_h, stride_row) of a block mask tensor.
+
+    block_mask: uint8 or bool CUDA tensor [1|B, 1|Hq, nqb, nkb] with
+    nqb >= ceil(Nq / 128), nkb >= ceil(Nk / 128) and unit stride along key
+    blocks; a size-1 batch or head dimension is shared (stride 0).
+    """
+    _dev(block_mask, "block_mask")
+    if block_mask.dtype not in (torch.uint8, torch.bool):
+        raise TypeError("block_mask must be uint8 or bool")
+    if block_mask.dim() != 4 or block_mask.shape[0] not in (1, B) or \
+            block_mask.shape[1] not in (1, Hq):
+        raise ValueError(f"block_mask shape {tuple(block_mask.shape)} is not [1|B, 1|Hq, nqb, nkb]")
+    nqb, nkb = -(-Nq // MASK_BLOCK), -(-Nk // MASK_BLOCK)
+    if block_mask.shape[2] < nqb or block_mask.shape[3] < nkb or block_mask.stride(3) != 1:
+        raise ValueError("block_mask does not cover the (query, key) blocks")
+    sb = 0 if block_mask.shape[0] == 1 else block_mask.stride(0)
+    sh = 0 if block_mask.shape[1] == 1 else block_mask.stride(1)
+    return block_mask.data_ptr(), sb, sh, block_mask.stride(2)
+
+
 def attn_fwd(q, k, v, scale=None, causal=False, seqlens_k=None, out=None, lse=None,
-             stream=None, window_left=-1):
+             stream=None, window_left=-1, block_mask=None):
     """Exact attention forward.
 
     q [B, Nq, Hq, d], k/v [B, Nk, Hkv, d] (bf16/fp16, CUDA, contiguous);
-    seqlens_k: optional int32 [B] key lengths.  Returns (o, lse) with
-    o [B, Nq, Hq, d] and lse [B, Hq, Nq] float32.
+    seqlens_k: optional int32 [B] key lengths; window_left: -1 or the
+    sliding window; block_mask: optional [1|B, 1|Hq, ceil(Nq/128),
+    ceil(Nk/128)] uint8/bool, 0 removes a 128 x 128 block (see
+    block_mask_args).  Returns (o, lse) with o [B, Nq, Hq, d] and
+    lse [B, Hq, Nq] float32.
     """
     lib = load_library()
     B, Nq, Hq, d = q.shape
@@ -127,7 +158,20 @@ def attn_fwd(q, k, v, scale=None, causal=False, seqlens_k=None, out=None, lse=No
     if lse is None:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     st = _stream_ptr(stream)
-    if window_left >= 0:
+    if block_mask is not None:
+        sl = 0
+        if seqlens_k is not None:
+            _dev(seqlens_k, "seqlens_k")
+            if seqlens_k.dtype != torch.int32:
+                raise TypeError("seqlens_k must be int32")
+            sl = seqlens_k.data_ptr()
+        mp, sb, sh, sr = block_mask_args(block_mask, B, Hq, Nq, Nk)
+        rc = lib.attn_fwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                      lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
+                                      int(bool(causal)), int(window_left), _dtype_code(q),
+                                      sl or None, mp, sb, sh, sr, st)
+        _check("attn_fwd_blocksparse", rc)
+    elif window_left >= 0:
         sl = 0
         if seqlens_k is not None:
             _dev(seqlens_k, "seqlens_k")

@@ -113,11 +113,15 @@ bool map_bnhd(CUtensorMap* m, int dtype, const void* base, int B, int N, int H, 
     return encode_map(m, dtype, base, 4, dims, strides, box);
 }
 
+constexpr BlockMask kNoBlockMask{nullptr, 0, 0, 0};
+
 int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype,
                const int* seqlens_k, void* stream, int inject, unsigned long long limit_ns,
-               int window_left) {
+               int window_left, const BlockMask& bmask) {
     if (window_left < -1) return ATTN_ERR_INVALID_ARG;
+    if (bmask.m && (bmask.sb < 0 || bmask.sh < 0 || bmask.srow < (Nk + 127) / 128))
+        return ATTN_ERR_INVALID_ARG;
     if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk < 0 || Hq % Hkv != 0)
@@ -157,6 +161,7 @@ int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse,
     p.scale_log2 = scale * 1.4426950408889634f;
     p.seqlens_k = Nk > 0 ? seqlens_k : nullptr;
     p.window_left = window_left;
+    p.bmask = bmask;
     p.lse = lse;
     p.limit_ns = limit_ns;
     p.inject = inject;
@@ -183,28 +188,39 @@ extern "C" {
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
              int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype, void* stream) {
     return fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, nullptr,
-                      stream, 0, kDefaultLimitNs, -1);
+                      stream, 0, kDefaultLimitNs, -1, kNoBlockMask);
 }
 
 int attn_fwd_kpad(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                   int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, int dtype,
                   const int* seqlens_k, void* stream) {
     return fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, seqlens_k,
-                      stream, 0, kDefaultLimitNs, -1);
+                      stream, 0, kDefaultLimitNs, -1, kNoBlockMask);
 }
 
 int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                     int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                     int window_left, int dtype, const int* seqlens_k, void* stream) {
     return fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, seqlens_k,
-                      stream, 0, kDefaultLimitNs, window_left);
+                      stream, 0, kDefaultLimitNs, window_left, kNoBlockMask);
+}
+
+int attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                         int window_left, int dtype, const int* seqlens_k,
+                         const unsigned char* block_mask, long long mask_stride_b,
+                         long long mask_stride_h, int mask_stride_row, void* stream) {
+    if (!block_mask) return ATTN_ERR_INVALID_ARG;
+    const BlockMask bm{block_mask, mask_stride_b, mask_stride_h, mask_stride_row};
+    return fwd_common(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, dtype, seqlens_k,
+                      stream, 0, kDefaultLimitNs, window_left, bm);
 }
 
 int attn_selftest_watchdog(const void* q, const void* k, const void* v, void* o, float* lse,
                            int limit_ms, void* stream) {
     if (limit_ms <= 0 || limit_ms > 10000) return ATTN_ERR_INVALID_ARG;
     return fwd_common(q, k, v, o, lse, 1, 1, 1, 128, 128, 64, 0.125f, 0, ATTN_BF16, nullptr,
-                      stream, 1, (unsigned long long)limit_ms * 1000000ull, -1);
+                      stream, 1, (unsigned long long)limit_ms * 1000000ull, -1, kNoBlockMask);
 }
 
 size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int d, int max_seqlen_k,

@@ -45,6 +45,8 @@ constexpr int kBlockN = 128;  // keys per K/V tile
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
+// a window wider than any key range (i + Lk - Nq - kNoWindow stays negative)
+constexpr int kNoWindow = 1 << 30;
 // one exponential pair in FWD_POLY_EVERY(D) is evaluated on the FMA pipe
 #ifndef FWD_POLY_EVERY
 #define FWD_POLY_EVERY(D) 4
@@ -166,7 +168,7 @@ __device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_bas
     }
 }
 
-template <int D, bool BF16, int KST, int VST, bool kWindow>
+template <int D, bool BF16, int KST, int VST, bool kWindow, bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -213,6 +215,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cnt0 = max(0, nt0 - j00), cnt1 = max(0, nt1 - j01);
     const int jstart = cnt0 > 0 ? j00 : j01;
     const int nt = max(cnt0 > 0 ? nt0 : 0, cnt1 > 0 ? nt1 : 0);
+    // block-sparse instance: the mask rows of the two Q tiles
+    const unsigned char* mrow = nullptr;
+    if constexpr (kSparse)
+        mrow = p.bmask.m + (long long)b * p.bmask.sb + (long long)h * p.bmask.sh +
+               (long long)(qbase / kBlockM) * p.bmask.srow;
+    // key tile j is used by Q0 when j in [j00, nt0), by Q1 when j in
+    // [j01, nt1), and (block-sparse) when the mask entry of the pair is set;
+    // the K/V stream is the union of the two, in increasing j
+    auto use = [&](int a, int j) -> bool {
+        bool u = a == 0 ? (cnt0 > 0 && j >= j00 && j < nt0) : (cnt1 > 0 && j >= j01 && j < nt1);
+        if constexpr (kSparse) {
+            if (u) u = __ldg(mrow + (a == 0 ? 0 : p.bmask.srow) + j) != 0;
+        }
+        return u;
+    };
+    // the last key tile each Q tile uses (-1: none, the tile's rows get O = 0)
+    int last0 = -1, last1 = -1;
+    for (int j = nt0 - 1; cnt0 > 0 && j >= j00; --j)
+        if (use(0, j)) {
+            last0 = j;
+            break;
+        }
+    for (int j = nt1 - 1; cnt1 > 0 && j >= j01; --j)
+        if (use(1, j)) {
+            last1 = j;
+            break;
+        }
 
     if (tid == 0) {
         for (int a = 0; a < 2; ++a) {
@@ -254,15 +283,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             int issued_k = 0, issued_v = 0;
             bool issued_q[2] = {false, false};
             for (int a = 0; a < 2; ++a) {
-                if ((a == 0 ? cnt0 : cnt1) == 0) continue;
+                // only a Q tile that takes part: the epilogue of the others
+                // stages O in the Q buffer without waiting for anything
+                if ((a == 0 ? last0 : last1) < 0) continue;
                 ptx::mbar_arrive_expect_tx(&bars->q_full[a], kTileBytes);
                 for (int c = 0; c < kDBlocks; ++c)
                     ptx::tma_load_4d(smem + L::kQ + a * kTileBytes + c * kBlockBytes, &tm_q,
                                      &bars->q_full[a], c * 64, h, qbase + a * kBlockM, b);
                 issued_q[a] = true;
             }
+            int t = -1;  // position of tile j in the stream
             for (int j = jstart; j < nt; ++j) {
-                const int t = j - jstart;
+                if constexpr (kSparse) {
+                    if (!use(0, j) && !use(1, j)) continue;
+                }
+                ++t;
                 const int sk = t % KST;
                 if (!ptx::mbar_wait(&bars->k_empty[sk], ((t / KST) & 1) ^ 1, p.limit_ns,
                                     abort_flag)) {
@@ -313,13 +348,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 return ok;
             };
-            auto issue_s = [&](int a, int j) {
+            // S_a of the tile at stream position t
+            auto issue_s = [&](int a, int t) {
                 if (!q_ready[a]) {
                     if (!wait_or_fail(&bars->q_full[a], 0, 3)) return;
                     ptx::tc_fence_after();
                     q_ready[a] = true;
                 }
-                const uint32_t k_addr = sbase + L::kK + ((j - jstart) % KST) * kTileBytes;
+                const uint32_t k_addr = sbase + L::kK + (t % KST) * kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
@@ -328,10 +364,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ptx::umma_commit(&bars->s_full[a]);
             };
-            auto issue_pv = [&](int a, int j) {
-                const int ja = a == 0 ? j00 : j01;  // the Q tile's first key tile
-                const int t = j - jstart;
-                if (!wait_or_fail(&bars->p_full[a], (j - ja) & 1, 5)) return;
+            // P_a·V of the tile at stream position t, the Q tile's ia-th tile;
+            // last: the Q tile's O is complete after it
+            auto issue_pv = [&](int a, int t, int ia, bool last) {
+                if (!wait_or_fail(&bars->p_full[a], ia & 1, 5)) return;
                 if (!wait_or_fail(&bars->v_full[t % VST], (t / VST) & 1, 6)) return;
                 ptx::tc_fence_after();
                 const uint32_t v_addr = sbase + L::kV + (t % VST) * kTileBytes;
@@ -339,39 +375,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < kBlockN / 16; ++kk) {
                     ptx::umma_ts(tmem + col_o[a], tmem + col_s[a] + kk * 8,
                                  ptx::sdesc_sw128(v_addr + kk * 16 * 128, kBlockBytes, 1024),
-                                 kIdescO, (j > ja || kk > 0) ? 1u : 0u);
+                                 kIdescO, (ia > 0 || kk > 0) ? 1u : 0u);
                 }
-                if (j == (a == 0 ? nt0 : nt1) - 1) ptx::umma_commit(&bars->o_done[a]);
+                if (last) ptx::umma_commit(&bars->o_done[a]);
             };
-            // key tile j is used by Q0 when j in [j00, nt0), by Q1 when j in
-            // [j01, nt1); a stage is released after its last user's product
-            auto use = [&](int a, int j) {
-                return a == 0 ? (cnt0 > 0 && j >= j00 && j < nt0)
-                              : (cnt1 > 0 && j >= j01 && j < nt1);
-            };
+            // a stage is released after its last user's product
+            int t = 0, i0 = 0, i1 = 0;                      // stream position, per-tile counts
+            int prev_t = 0, prev_i1 = 0, prev_j = -1;       // the previous tile of the stream
+            bool prev_u1 = false;
             for (int j = jstart; ok && j <= nt; ++j) {
-                const int t = j - jstart;
+                bool u0 = false, u1 = false;
                 if (j < nt) {
+                    u0 = use(0, j);
+                    u1 = use(1, j);
+                    if (kSparse && !u0 && !u1) continue;
                     if (!wait_or_fail(&bars->k_full[t % KST], (t / KST) & 1, 4)) break;
                     ptx::tc_fence_after();
-                    if (use(0, j)) issue_s(0, j);
+                    if (u0) issue_s(0, t);
                     if (!ok) break;
                 }
-                if (j > jstart && use(1, j - 1)) {
-                    issue_pv(1, j - 1);
+                if (prev_u1) {
+                    issue_pv(1, prev_t, prev_i1, prev_j == last1);
                     if (!ok) break;
-                    ptx::umma_commit(&bars->v_empty[(t - 1) % VST]);
+                    ptx::umma_commit(&bars->v_empty[prev_t % VST]);
                 }
                 if (j < nt) {
-                    if (use(1, j)) issue_s(1, j);
+                    if (u1) issue_s(1, t);
                     if (!ok) break;
                     ptx::umma_commit(&bars->k_empty[t % KST]);
-                    if (use(0, j)) {
-                        issue_pv(0, j);
+                    if (u0) {
+                        issue_pv(0, t, i0, j == last0);
                         if (!ok) break;
                     }
-                    if (!use(1, j)) ptx::umma_commit(&bars->v_empty[t % VST]);
+                    if (!u1) ptx::umma_commit(&bars->v_empty[t % VST]);
                 }
+                prev_u1 = u1;
+                prev_t = t;
+                prev_i1 = i1;
+                prev_j = j;
+                i0 += u0 ? 1 : 0;
+                i1 += u1 ? 1 : 0;
+                ++t;
             }
             if (!ok) {
                 // make sure no MMA is still running before TMEM is freed
@@ -402,8 +446,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_s = tmem + lane_addr + (a == 0 ? 0u : 128u);
         const uint32_t t_o = tmem + lane_addr + (a == 0 ? 256u : 256u + D);
 
-        for (int j = ja; j < nta; ++j) {
-            if (!warp_wait(&bars->s_full[a], (j - ja) & 1, p.limit_ns, abort_flag)) {
+        int ia = 0;  // key tiles of this Q tile done so far
+        int tu = 0;  // block-sparse: stream position of the next tile of the union
+        for (int j = kSparse ? jstart : ja; j < nta; ++j) {
+            int t;  // stream position of tile j
+            if constexpr (kSparse) {
+                if (!use(a, j)) {
+                    if (use(1 - a, j)) ++tu;
+                    continue;
+                }
+                t = tu++;
+            } else {
+                t = j - jstart;
+            }
+            if (!warp_wait(&bars->s_full[a], ia & 1, p.limit_ns, abort_flag)) {
                 record_error(p.err, kErrFwdBase + 7, &bars->abort);
                 ok = false;
                 break;
@@ -440,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool rescale = false;
             if (m_tile > m_ref + kRescaleThreshold) {
                 alpha = ptx::ex2_approx(m_ref - m_tile);  // 0 when m_ref = -inf
-                rescale = (j > ja) && (m_ref != -INFINITY);
+                rescale = (ia > 0) && (m_ref != -INFINITY);
                 m_ref = m_tile;
             }
             const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
@@ -493,13 +549,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the Q tile that uses key tile j first zeroes its V rows behind
             // the real length (Q0 if it uses the tile, else Q1)
             const bool zero_v = p.seqlens_k != nullptr && key0 + kBlockN > Lk &&
-                                (a == 0 ? true : (cnt0 == 0 || j >= nt0));
+                                (a == 0 || !use(0, j));
             if (zero_v) {
                 // keys behind the real length: zero their V rows so that a
                 // non-finite value stored there cannot reach O through 0 * NaN
-                const int sv = (j - jstart) % VST;
-                if (!warp_wait(&bars->v_full[sv], ((j - jstart) / VST) & 1, p.limit_ns,
-                               abort_flag)) {
+                const int sv = t % VST;
+                if (!warp_wait(&bars->v_full[sv], (t / VST) & 1, p.limit_ns, abort_flag)) {
                     record_error(p.err, kErrFwdBase + 8, &bars->abort);
                     ok = false;
                     break;
@@ -517,25 +572,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bars->p_full[a]);
+            ++ia;
         }
 
         // ---- epilogue: O / l -> bf16/fp16 -> swizzled staging (the Q_a
         // buffer, free once the last S_a MMA is done) -> TMA store
-        if (ok && nta > 0) {
+        if (ok && ia > 0) {
             if (!warp_wait(&bars->o_done[a], 0, p.limit_ns, abort_flag)) {
                 record_error(p.err, kErrFwdBase + 9, &bars->abort);
                 ok = false;
             }
             ptx::tc_fence_after();
         }
-        const bool have = ok && nta > 0 && l_sum > 0.f;
+        const bool have = ok && ia > 0 && l_sum > 0.f;
         const float inv_l = have ? 1.f / l_sum : 0.f;
         uint8_t* stage = smem + L::kQ + a * kTileBytes;
         if (qa < p.Nq) {
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t r[32];
-                if (ok && nta > 0) {
+                if (ok && ia > 0) {
                     ptx::tmem_ld32(t_o + c * 32, r);
                     ptx::tmem_wait_ld_dep(r);
                 } else {
@@ -581,11 +637,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int D, bool BF16, int KST, int VST, bool kWindow>
+template <int D, bool BF16, int KST, int VST, bool kWindow, bool kSparse>
 cudaError_t launch_fwd_w(const FwdMaps& maps, const FwdParams& p, cudaStream_t stream) {
     using L = FwdSmem<D, KST, VST>;
     static_assert(L::kAlloc <= 227 * 1024, "shared memory budget");
-    auto kern = attn_fwd_kernel<D, BF16, KST, VST, kWindow>;
+    auto kern = attn_fwd_kernel<D, BF16, KST, VST, kWindow, kSparse>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc);
     if (e != cudaSuccess) return e;
@@ -595,11 +651,17 @@ cudaError_t launch_fwd_w(const FwdMaps& maps, const FwdParams& p, cudaStream_t s
 }
 
 // the sliding-window masks and tile ranges are compiled only into the
-// instance that a window call launches
+// instances that window and block-sparse calls launch; the block-sparse
+// instance takes a window that reaches past every key when it has none
 template <int D, bool BF16, int KST, int VST>
 cudaError_t launch_fwd_t(const FwdMaps& maps, const FwdParams& p, cudaStream_t stream) {
-    return p.window_left >= 0 ? launch_fwd_w<D, BF16, KST, VST, true>(maps, p, stream)
-                              : launch_fwd_w<D, BF16, KST, VST, false>(maps, p, stream);
+    if (p.bmask.m != nullptr) {
+        FwdParams q = p;
+        if (q.window_left < 0) q.window_left = kNoWindow;
+        return launch_fwd_w<D, BF16, KST, VST, true, true>(maps, q, stream);
+    }
+    return p.window_left >= 0 ? launch_fwd_w<D, BF16, KST, VST, true, false>(maps, p, stream)
+                              : launch_fwd_w<D, BF16, KST, VST, false, false>(maps, p, stream);
 }
 
 }  // namespace

@@ -15,6 +15,16 @@ enum : unsigned {
     kErrBwdBase = 3 * 16,
 };
 
+// Block mask of block-sparse attention, one entry per (128-query tile,
+// 128-key tile): the entry of batch b, query head h, query tile qt and key
+// tile kt is m[b * sb + h * sh + qt * srow + kt]; 0 masks every key of the
+// tile for those queries.  m == nullptr: no block mask.
+struct BlockMask {
+    const unsigned char* m;
+    long long sb, sh;
+    int srow;
+};
+
 struct FwdParams {
     int B, Hq, Hkv, Nq, Nk;
     int G;            // Hq / Hkv
@@ -23,6 +33,7 @@ struct FwdParams {
     float scale_log2; // scale * log2(e)
     const int* seqlens_k;  // [B] or nullptr
     int window_left;       // -1, or keys before i + (Lk - Nq) - window_left are masked
+    BlockMask bmask;       // block-sparse mask, or m == nullptr
     float* lse;            // [B, Hq, Nq]
     unsigned long long limit_ns;
     int inject;       // self-test: the loader skips everything

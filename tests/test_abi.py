@@ -63,6 +63,19 @@ def test_fwd_rejects_bad_arguments(args, expect):
     assert lib.attn_fwd(*args, None) == expect
 
 
+@pytest.mark.parametrize("mask,sb,sh,srow", [
+    (0, 0, 0, 8),       # no mask
+    (P, -1, 0, 8),      # negative batch stride
+    (P, 0, -16, 8),     # negative head stride
+    (P, 0, 0, 7),       # a row of the mask shorter than ceil(1000 / 128) = 8 key blocks
+])
+def test_blocksparse_rejects_bad_masks(mask, sb, sh, srow):
+    lib = attn.load_library()
+    rc = lib.attn_fwd_blocksparse(P, P, P, P, P, 1, 2, 1, 300, 1000, 128, 0.09, 0, -1, 0, None,
+                                  mask or None, sb, sh, srow, None)
+    assert rc == -1
+
+
 def test_decode_rejects_bad_arguments():
     lib = attn.load_library()
     base = dict(q=P, k=P, v=P, cu=P, sl=P, maxl=100, slots=100, o=P, lse=P, B=2, Hq=8, Hkv=2,
