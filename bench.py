@@ -41,7 +41,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from io_aware_exact_29_b200 import accounting  # noqa: E402
-from io_aware_exact_29_b200.workloads import (DECODE_CASES, FWD_CASES, fwd_inputs,  # noqa: E402
+from io_aware_exact_29_b200.workloads import (BLOCKSPARSE_CASES, DECODE_CASES,  # noqa: E402
+                                              FWD_CASES, block_mask_inputs, fwd_inputs,
                                               kvcache_inputs, paged_from_packed,
                                               upstream_grad)
 
@@ -623,6 +624,38 @@ def run_sweep(reps: int = 20):
                           "frac_sustained": round(tb / peaks["bf16_tflops_sustained"], 3)}),
               flush=True)
         del fin, o, lse, dout, ws_b, grads
+    for name, bc in BLOCKSPARSE_CASES.items():
+        c = bc.fwd
+        fin = fwd_inputs(c, seed=0, device="cuda")
+        m = block_mask_inputs(bc, seed=0, device="cuda")
+        o = torch.empty_like(fin["q"])
+        lse = torch.empty((c.B, c.Hq, c.Nq), dtype=torch.float32, device=dev)
+        ms = timed(lambda: attn.attn_fwd(fin["q"], fin["k"], fin["v"], scale=c.scale,
+                                         causal=c.causal, out=o, lse=lse, block_mask=m))
+        flops = accounting.blocksparse_flops(m.cpu().numpy(), c.Nq, c.Nk, c.d, c.causal, c.B,
+                                             c.Hq)
+        dense = accounting.fwd_flops(c.B, c.Hq, c.Nq, c.Nk, c.d, c.causal)
+        tf = flops / (ms * 1e-3) / 1e12
+        print(json.dumps({"sweep": name, "kind": "fwd", "dtype": c.dtype, "causal": c.causal,
+                          "B": c.B, "H": c.Hq, "N": c.Nq, "d": c.d,
+                          "kept": round(flops / dense, 4), "ms": round(ms, 4),
+                          "TFLOP/s": round(tf, 1),
+                          "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 3)}),
+              flush=True)
+        dout = upstream_grad(fin["q"], seed=0, device="cuda")
+        ws_b = torch.empty(attn.bwd_workspace_bytes(c.B, c.Hq, c.Nq), dtype=torch.uint8, device=dev)
+        grads = (torch.empty_like(fin["q"]), torch.empty_like(fin["k"]), torch.empty_like(fin["v"]))
+        ms_b = timed(lambda: attn.attn_bwd(fin["q"], fin["k"], fin["v"], o, lse, dout, scale=c.scale,
+                                           causal=c.causal, workspace=ws_b, dq=grads[0],
+                                           dk=grads[1], dv=grads[2], block_mask=m))
+        tb = 2.5 * flops / (ms_b * 1e-3) / 1e12
+        print(json.dumps({"sweep": name, "kind": "bwd", "dtype": c.dtype, "causal": c.causal,
+                          "B": c.B, "H": c.Hq, "N": c.Nq, "d": c.d,
+                          "kept": round(flops / dense, 4), "ms": round(ms_b, 4),
+                          "TFLOP/s": round(tb, 1),
+                          "frac_sustained": round(tb / peaks["bf16_tflops_sustained"], 3)}),
+              flush=True)
+        del fin, m, o, lse, dout, ws_b, grads
     for name, c in DECODE_CASES.items():
         din = kvcache_inputs(c, seed=0, device="cuda")
         ml = int(din["seqlens_k"].max().item())

@@ -252,6 +252,22 @@ ATTN_API int attn_bwd_window(const void* q, const void* k, const void* v, const 
                              int causal, int window_left, int dtype, const int* seqlens_k,
                              void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * attn_bwd for the block-sparse forward (attn_fwd_blocksparse): the same
+ * arguments as attn_bwd_window plus the forward's block mask and strides
+ * (NULL block_mask = attn_bwd_window).  Masked blocks are skipped in both
+ * gradient kernels: a key tile's dK/dV visits only the (head, query tile)
+ * pairs whose entry is set, a query tile's dQ only its set key tiles.
+ */
+ATTN_API int attn_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o,
+                                  const float* lse, const void* dout, void* dq, void* dk,
+                                  void* dv, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                                  float scale, int causal, int window_left, int dtype,
+                                  const int* seqlens_k, const unsigned char* block_mask,
+                                  long long mask_stride_b, long long mask_stride_h,
+                                  int mask_stride_row, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
 /* Size in bytes of the scratch area built into the library for
  * attn_fwd_varlen_kvcache_noalloc (32 MiB). */
 #define ATTN_NOALLOC_SCRATCH_BYTES (32u << 20)

@@ -11,6 +11,8 @@ query, the output and the LSE.
 """
 from __future__ import annotations
 
+import numpy as np
+
 
 def score_matrix_elements(n: int) -> int:
     """Entries of one head's N×N score matrix S."""
@@ -47,6 +49,35 @@ def fwd_flops(B, Hq, Nq, Nk, d, causal, seqlens_k=None) -> int:
     if seqlens_k is None:
         return 4 * d * B * Hq * visible_pairs(Nq, Nk, causal)
     return sum(4 * d * Hq * visible_pairs(Nq, int(l), causal) for l in seqlens_k)
+
+
+def block_pair_counts(Nq: int, Nk: int, causal: bool, block: int = 128) -> np.ndarray:
+    """[nqb, nkb] int64: visible (query, key) pairs inside each block of a
+    block mask, under the causal rule (bottom-right) when causal."""
+    nqb, nkb = -(-Nq // block), -(-Nk // block)
+    out = np.zeros((nqb, nkb), dtype=np.int64)
+    off = Nk - Nq
+    for qb in range(nqb):
+        rows = np.arange(qb * block, min(Nq, (qb + 1) * block))
+        for kb in range(nkb):
+            lo, hi = kb * block, min(Nk, (kb + 1) * block)
+            if causal:
+                top = np.minimum(hi, rows + off + 1)
+                out[qb, kb] = int(np.maximum(0, top - lo).sum())
+            else:
+                out[qb, kb] = len(rows) * (hi - lo)
+    return out
+
+
+def blocksparse_flops(mask, Nq: int, Nk: int, d: int, causal: bool, B: int, Hq: int,
+                      block: int = 128) -> int:
+    """4 d x (visible pairs) summed over batches and heads for a block mask
+    [1|B, 1|Hq, nqb, nkb] (a size-1 dimension is shared)."""
+    m = np.asarray(mask) != 0
+    cnt = block_pair_counts(Nq, Nk, causal, block)
+    per = (m * cnt[None, None]).sum(axis=(2, 3))  # [Bm, Hm]
+    per = np.broadcast_to(per, (B, Hq))
+    return int(4 * d * per.sum())
 
 
 def fwd_bytes(B, Hq, Hkv, Nq, Nk, d, elem_bytes=2) -> int:

@@ -54,6 +54,9 @@ def load_library():
             lib.attn_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i,
                                                  vp, vp, ll, ll, i, vp]
             lib.attn_fwd_blocksparse.restype = i
+            lib.attn_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i,
+                                                 i, i, f, i, i, i, vp, vp, ll, ll, i, vp, sz, vp]
+            lib.attn_bwd_blocksparse.restype = i
             lib.attn_bwd_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i,
                                             f, i, i, i, vp, vp, sz, vp]
             lib.attn_bwd_window.restype = i
@@ -204,10 +207,11 @@ def bwd_workspace_bytes(B, Hq, Nq) -> int:
 
 
 def attn_bwd(q, k, v, o, lse, dout, scale=None, causal=False, seqlens_k=None, workspace=None,
-             dq=None, dk=None, dv=None, stream=None, window_left=-1):
+             dq=None, dk=None, dv=None, stream=None, window_left=-1, block_mask=None):
     """Gradients of L = sum(dout * O) for O = attn_fwd(q, k, v, ...).
 
-    o and lse are the forward's outputs for the same arguments.  Returns
+    o and lse are the forward's outputs for the same arguments (window_left
+    and block_mask included).  Returns
     (dq [B, Nq, Hq, d], dk, dv [B, Nk, Hkv, d]) in the input dtype; dk and dv
     are summed over the query heads that share a kv head.
     """
@@ -230,11 +234,21 @@ def attn_bwd(q, k, v, o, lse, dout, scale=None, causal=False, seqlens_k=None, wo
         if seqlens_k.dtype != torch.int32:
             raise TypeError("seqlens_k must be int32")
         sl = seqlens_k.data_ptr()
-    rc = lib.attn_bwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                             lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                             dv.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
-                             int(bool(causal)), int(window_left), _dtype_code(q), sl or None,
-                             workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    if block_mask is not None:
+        mp, sb, sh, sr = block_mask_args(block_mask, B, Hq, Nq, Nk)
+        rc = lib.attn_bwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                      lse.data_ptr(), dout.data_ptr(), dq.data_ptr(),
+                                      dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
+                                      float(scale), int(bool(causal)), int(window_left),
+                                      _dtype_code(q), sl or None, mp, sb, sh, sr,
+                                      workspace.data_ptr(), workspace.numel(),
+                                      _stream_ptr(stream))
+    else:
+        rc = lib.attn_bwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                 lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                 dv.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
+                                 int(bool(causal)), int(window_left), _dtype_code(q), sl or None,
+                                 workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
     _check("attn_bwd", rc)
     return dq, dk, dv
 

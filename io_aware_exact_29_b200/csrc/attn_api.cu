@@ -437,7 +437,22 @@ int attn_bwd_window(const void* q, const void* k, const void* v, const void* o, 
                     int Nq, int Nk, int d, float scale, int causal, int window_left, int dtype,
                     const int* seqlens_k, void* workspace, size_t workspace_bytes,
                     void* stream) {
+    return attn_bwd_blocksparse(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale,
+                                causal, window_left, dtype, seqlens_k, nullptr, 0, 0, 0,
+                                workspace, workspace_bytes, stream);
+}
+
+int attn_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                         int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                         int window_left, int dtype, const int* seqlens_k,
+                         const unsigned char* block_mask, long long mask_stride_b,
+                         long long mask_stride_h, int mask_stride_row, void* workspace,
+                         size_t workspace_bytes, void* stream) {
     if (window_left < -1) return ATTN_ERR_INVALID_ARG;
+    if (block_mask && (mask_stride_b < 0 || mask_stride_h < 0 ||
+                       mask_stride_row < (Nk + 127) / 128))
+        return ATTN_ERR_INVALID_ARG;
     if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk < 0 || Hq % Hkv != 0)
@@ -483,6 +498,7 @@ int attn_bwd_window(const void* q, const void* k, const void* v, const void* o, 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.seqlens_k = Nk > 0 ? seqlens_k : nullptr;
     p.window_left = window_left;
+    p.bmask = BlockMask{block_mask, mask_stride_b, mask_stride_h, mask_stride_row};
     p.o = o;
     p.dout = dout;
     p.lse = lse;

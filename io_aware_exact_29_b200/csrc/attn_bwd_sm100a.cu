@@ -175,7 +175,7 @@ struct DkdvBars {
     int abort;
 };
 
-template <int D, bool BF16, int QST>
+template <int D, bool BF16, int QST, bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -215,7 +215,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         qt_end = i_max < 0 ? 0 : min(n_qt, i_max / kBlock + 1);
     }
     const int nqs = (k0 < Lk) ? max(0, qt_end - qt_first) : 0;
-    const int nsteps = p.G * nqs;
+    const int nsteps_all = p.G * nqs;
+    // step sa = (query head g*G + sa / nqs, query tile qt_first + sa % nqs);
+    // with a block mask only the steps whose entry for this key tile is set
+    // take part, and stages and phases count those
+    auto step_on = [&](int sa) -> bool {
+        if constexpr (kSparse) {
+            const long long hq = g * p.G + sa / nqs;
+            const long long qt = qt_first + sa % nqs;
+            return __ldg(p.bmask.m + (long long)b * p.bmask.sb + hq * p.bmask.sh +
+                         qt * p.bmask.srow + blockIdx.x) != 0;
+        }
+        return true;
+    };
+    // the step after sa that takes part (sa = -1: the first)
+    auto next_step = [&](int sa) -> int {
+        if constexpr (kSparse) {
+            do {
+                ++sa;
+            } while (sa < nsteps_all - 1 && !step_on(sa));
+            return sa;
+        } else {
+            return sa + 1;
+        }
+    };
+    int nsteps = nsteps_all;
+    if constexpr (kSparse) {
+        int c = 0;
+        for (int base = 0; base < nsteps_all; base += 32) {
+            const int sa = base + lane;
+            c += __popc(__ballot_sync(0xffffffffu, sa < nsteps_all && step_on(sa)));
+        }
+        nsteps = c;
+    }
 
     if (tid == 0) {
         ptx::mbar_init(&bars->kv_full, 1);
@@ -261,10 +293,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
             int issued = 0;
+            int sa = -1;
             for (int s = 0; s < nsteps; ++s) {
+                sa = next_step(sa);
                 const int st = s % QST;
-                const int h = g * p.G + s / nqs;
-                const int i0 = (qt_first + s % nqs) * kBlock;
+                const int h = g * p.G + sa / nqs;
+                const int i0 = (qt_first + sa % nqs) * kBlock;
                 if (!warp_wait(&bars->q_empty[st], ((s / QST) & 1) ^ 1, p.limit_ns, abort_flag)) {
                     record_error(p.err, kErrBwdBase + 1, &bars->abort);
                     break;
@@ -403,9 +437,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float sl2 = p.scale_log2;
         const bool key_ok = kr < Lk;
         bool ok = true;
+        int sa = -1;
         for (int s = 0; s < nsteps; ++s) {
+            sa = next_step(sa);
             const int st = s % QST;
-            const int i0 = (qt_first + s % nqs) * kBlock;
+            const int i0 = (qt_first + sa % nqs) * kBlock;
             if (!warp_wait(&bars->s_full[half], s & 1, p.limit_ns, abort_flag)) {
                 record_error(p.err, kErrBwdBase + 5, &bars->abort);
                 ok = false;
@@ -539,7 +575,7 @@ __device__ __forceinline__ int dq_tiles(int q_first, int Nq, int Lk, int causal)
     return nt;
 }
 
-template <int D, bool BF16, int KST>
+template <int D, bool BF16, int KST, bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -572,7 +608,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     // key tiles j0 .. j0 + nt - 1 (the sliding window's first tile is j0);
     // stages and phases count from 0
     const int j0 = p.window_left >= 0 ? max(0, i0 + off - p.window_left) / kBlock : 0;
-    const int nt = max(0, dq_tiles(i0, p.Nq, Lk, p.causal) - j0);
+    const int nt_all = max(0, dq_tiles(i0, p.Nq, Lk, p.causal) - j0);
+    // with a block mask only the key tiles whose entry for this query tile
+    // is set take part, and stages and phases count those
+    const unsigned char* mrow = nullptr;
+    if constexpr (kSparse)
+        mrow = p.bmask.m + (long long)b * p.bmask.sb + (long long)h * p.bmask.sh +
+               (long long)blockIdx.x * p.bmask.srow;
+    // the absolute key tile after jj that takes part (jj = j0 - 1: the first)
+    auto next_tile = [&](int jj) -> int {
+        if constexpr (kSparse) {
+            do {
+                ++jj;
+            } while (jj < j0 + nt_all - 1 && __ldg(mrow + jj) == 0);
+            return jj;
+        } else {
+            return jj + 1;
+        }
+    };
+    int nt = nt_all;
+    if constexpr (kSparse) {
+        int c = 0;
+        for (int base = 0; base < nt_all; base += 32) {
+            const int jj = j0 + base + lane;
+            c += __popc(__ballot_sync(0xffffffffu, base + lane < nt_all && __ldg(mrow + jj) != 0));
+        }
+        nt = c;
+    }
 
     if (tid == 0) {
         ptx::mbar_init(&bars->q_full, 1);
@@ -620,7 +682,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
             int issued_k = 0, issued_v = 0;
+            int jj = j0 - 1;  // absolute key tile
             for (int j = 0; j < nt; ++j) {
+                jj = next_tile(jj);
                 const int st = j % KST;
                 if (!warp_wait(&bars->k_empty[st], ((j / KST) & 1) ^ 1, p.limit_ns, abort_flag)) {
                     record_error(p.err, kErrBwdBase + 7, &bars->abort);
@@ -630,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::mbar_arrive_expect_tx(&bars->k_full[st], kTile);
                     for (int c = 0; c < kDBlocks; ++c)
                         ptx::tma_load_4d(smem + L::kK + st * kTile + c * kBlockBytes, &tm_k,
-                                         &bars->k_full[st], c * 64, g, (j0 + j) * kBlock, b);
+                                         &bars->k_full[st], c * 64, g, jj * kBlock, b);
                 }
                 __syncwarp();
                 ++issued_k;
@@ -642,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::mbar_arrive_expect_tx(&bars->v_full[st], kTile);
                     for (int c = 0; c < kDBlocks; ++c)
                         ptx::tma_load_4d(smem + L::kV + st * kTile + c * kBlockBytes, &tm_v,
-                                         &bars->v_full[st], c * 64, g, (j0 + j) * kBlock, b);
+                                         &bars->v_full[st], c * 64, g, jj * kBlock, b);
                 }
                 __syncwarp();
                 ++issued_v;
@@ -762,9 +826,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float lse2 = row_ok ? p.lse2[sidx] : INFINITY;
         const float dsum = row_ok ? p.dsum[sidx] : 0.f;
         bool ok = true;
+        int jj = j0 - 1;  // absolute key tile
         for (int j = 0; j < nt; ++j) {
+            jj = next_tile(jj);
             const int st = j % KST;
-            const int kc0 = (j0 + j) * kBlock + 32 * part;  // first key of this warp's columns
+            const int kc0 = jj * kBlock + 32 * part;  // first key of this warp's columns
             if (!warp_wait(&bars->s_full[half], j & 1, p.limit_ns, abort_flag)) {
                 record_error(p.err, kErrBwdBase + 12, &bars->abort);
                 ok = false;
@@ -810,7 +876,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // B operand of dS K), so that 0 * NaN cannot reach dQ; the quarter-0
             // warps of the half take its 64 rows (its S product is complete)
             const int krow = 64 * half + 32 * (part & 1) + lane;
-            if (quarter == 0 && (j0 + j) * kBlock + kBlock > Lk && (j0 + j) * kBlock + krow >= Lk) {
+            if (quarter == 0 && jj * kBlock + kBlock > Lk && jj * kBlock + krow >= Lk) {
                 uint8_t* kt = smem + L::kK + st * kTile;
 #pragma unroll
                 for (int c = 0; c < kDBlocks; ++c)
@@ -850,13 +916,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int D, bool BF16, int QST, int KST>
-cudaError_t launch_bwd_t(const BwdMaps& m, const BwdParams& p, cudaStream_t stream) {
+template <int D, bool BF16, int QST, int KST, bool kSparse>
+cudaError_t launch_bwd_s(const BwdMaps& m, const BwdParams& p, cudaStream_t stream) {
     using L1 = DkdvSmem<D, QST>;
     using L2 = DqSmem<D, KST>;
     static_assert(L1::kAlloc <= 227 * 1024 && L2::kAlloc <= 227 * 1024, "shared memory");
-    auto k1 = attn_bwd_dkdv_kernel<D, BF16, QST>;
-    auto k2 = attn_bwd_dq_kernel<D, BF16, KST>;
+    auto k1 = attn_bwd_dkdv_kernel<D, BF16, QST, kSparse>;
+    auto k2 = attn_bwd_dq_kernel<D, BF16, KST, kSparse>;
     cudaError_t e =
         cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L1::kAlloc);
     if (e != cudaSuccess) return e;
@@ -876,6 +942,14 @@ cudaError_t launch_bwd_t(const BwdMaps& m, const BwdParams& p, cudaStream_t stre
     dim3 g2((p.Nq + kBlock - 1) / kBlock, p.Hq, p.B);
     k2<<<g2, kThreads, L2::kAlloc, stream>>>(m.q, m.k, m.v, m.dout, p);
     return cudaGetLastError();
+}
+
+// the block-mask reads are compiled only into the instances a block-sparse
+// call launches
+template <int D, bool BF16, int QST, int KST>
+cudaError_t launch_bwd_t(const BwdMaps& m, const BwdParams& p, cudaStream_t stream) {
+    return p.bmask.m != nullptr ? launch_bwd_s<D, BF16, QST, KST, true>(m, p, stream)
+                                : launch_bwd_s<D, BF16, QST, KST, false>(m, p, stream);
 }
 
 }  // namespace

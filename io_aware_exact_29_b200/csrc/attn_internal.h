@@ -56,6 +56,7 @@ struct BwdParams {
     float scale_log2;      // scale * log2(e)
     const int* seqlens_k;  // [B] or nullptr
     int window_left;       // -1, or keys before i + (Lk - Nq) - window_left are masked
+    BlockMask bmask;       // block-sparse mask, or m == nullptr
     const void* o;         // [B, Nq, Hq, d] forward output
     const void* dout;      // [B, Nq, Hq, d]
     const float* lse;      // [B, Hq, Nq] forward log-sum-exp (natural log)

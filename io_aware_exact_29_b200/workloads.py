@@ -88,6 +88,42 @@ def _cases():
 FWD_CASES, DECODE_CASES = _cases()
 
 
+@dataclass
+class BlockSparseCase:
+    """A forward problem plus a seeded block mask of 128 x 128 blocks."""
+    name: str
+    fwd: FwdCase
+    density: float  # probability that an off-diagonal block is kept
+
+
+# the long-sequence sweep's N = 8192, d = 128 point with a quarter of the
+# blocks kept per head (the pages give no block-sparse workload; this is the
+# dense sweep point thinned out)
+BLOCKSPARSE_CASES = {
+    "blocksparse_d128_n8192_25pct": BlockSparseCase(
+        "blocksparse_d128_n8192_25pct", FwdCase("bs", 2, 16, 16, 8192, 8192, 128, False), 0.25),
+    "blocksparse_d128_n8192_causal_25pct": BlockSparseCase(
+        "blocksparse_d128_n8192_causal_25pct", FwdCase("bsc", 2, 16, 16, 8192, 8192, 128, True),
+        0.25),
+}
+
+
+def block_mask_inputs(case: BlockSparseCase, seed: int = 0, device: str = "cpu",
+                      block: int = 128) -> torch.Tensor:
+    """uint8 [B, H, ceil(Nq/block), ceil(Nk/block)]: each block kept with
+    probability case.density, and the block on the diagonal of the query's
+    own position always kept (so that no causal row is left without keys)."""
+    c = case.fwd
+    g = torch.Generator(device="cpu").manual_seed(seed + 7_000_003)
+    nqb, nkb = -(-c.Nq // block), -(-c.Nk // block)
+    m = (torch.rand((c.B, c.Hq, nqb, nkb), generator=g) < case.density).to(torch.uint8)
+    for qb in range(nqb):
+        kb = min(nkb - 1, (qb * block + c.Nk - c.Nq) // block) if c.Nk > 0 else -1
+        if kb >= 0:
+            m[:, :, qb, kb] = 1
+    return m.to(device)
+
+
 def fwd_inputs(case: FwdCase, seed: int = 0, device: str = "cpu"):
     """Q [B,Nq,Hq,d], K/V [B,Nk,Hkv,d] in the case's dtype, and the optional
     per-batch key lengths [B] int32."""

@@ -1,15 +1,16 @@
-"""Block-sparse forward (attn_fwd_blocksparse) against the fp64 oracle with
-the same block mask: random masks of several densities, per-head, per-batch
-and shared masks, causal and not, ragged sizes, key padding, a window on
-top, rows with no block, and skipped key blocks holding NaN."""
+"""Block-sparse attention (attn_fwd_blocksparse, attn_bwd_blocksparse)
+against the fp64 oracle with the same block mask: random masks of several
+densities, per-head, per-batch and shared masks, causal and not, ragged
+sizes, key padding, a window on top, rows with no block, skipped key blocks
+holding NaN, and the gradients under the same masks."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 from io_aware_exact_29_b200 import attn
-from io_aware_exact_29_b200.workloads import FwdCase, fwd_inputs
-from tests.parity import compare
+from io_aware_exact_29_b200.workloads import FwdCase, fwd_inputs, upstream_grad
+from tests.parity import compare, compare_grads
 
 pytestmark = pytest.mark.gpu
 
@@ -146,3 +147,59 @@ def test_fp16_and_long_rows_sampled():
     o_ref, l_ref = oracle.attn_fwd(inp["q"], inp["k"], inp["v"], c.scale, True, rows=rows,
                                    block_mask=m, block_size=BLK)
     compare(o, lse, o_ref, l_ref, rows=rows, what="fp16 block-sparse, sampled rows")
+
+
+def _bwd(inp, c, m, window_left=-1, seed=0):
+    o, lse, dev = _fwd(inp, c, m, window_left)
+    mt = torch.from_numpy(np.ascontiguousarray(m)).cuda()
+    dout = upstream_grad(inp["q"], seed=seed)
+    got = attn.attn_bwd(dev["q"], dev["k"], dev["v"], o, lse, dout.cuda(), scale=c.scale,
+                        causal=c.causal, seqlens_k=dev["seqlens_k"], window_left=window_left,
+                        block_mask=mt)
+    torch.cuda.synchronize()
+    assert attn.get_device_error() == 0
+    ref = oracle.attn_bwd(inp["q"], inp["k"], inp["v"], dout, c.scale, c.causal,
+                          seqlens_k=inp["seqlens_k"], window_left=window_left, block_mask=m,
+                          block_size=BLK)
+    return got, ref
+
+
+@pytest.mark.parametrize("density", [0.3, 0.7])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_random_masks(density, causal, d):
+    # GQA: the four query heads of a kv head carry different masks, so dK and
+    # dV sum over differently masked heads
+    c = FwdCase("bsb", 2, 8, 2, 448, 520, d, causal)
+    inp = fwd_inputs(c, seed=230 + d)
+    nqb, nkb = _nb(c)
+    m = _mask((c.B, c.Hq, nqb, nkb), density, seed=231 + int(density * 10) + causal)
+    got, ref = _bwd(inp, c, m, seed=232)
+    compare_grads(got, ref, what=f"bwd block-sparse {density} causal {causal} d{d}")
+
+
+def test_backward_empty_rows_and_columns():
+    c = FwdCase("bse", 1, 2, 1, 384, 512, 128, False)
+    inp = fwd_inputs(c, seed=233)
+    m = np.ones((1, 2, 3, 4), np.uint8)
+    m[0, :, :, 1] = 0  # key block 1 masked for every query: dK, dV = 0 there
+    m[0, 0, 2, :] = 0  # head 0, query block 2: no key: dQ = 0 there
+    got, ref = _bwd(inp, c, m, seed=234)
+    dq, dk, dv = (t.float().cpu() for t in got)
+    assert not dk[0, 128:256].any() and not dv[0, 128:256].any()
+    assert not dq[0, 256:384, 0].any()
+    compare_grads(got, ref, what="bwd empty rows and columns")
+
+
+def test_backward_with_key_padding_and_window():
+    c = FwdCase("bsbw", 2, 4, 2, 384, 700, 128, True)
+    inp = fwd_inputs(c, seed=235)
+    inp["seqlens_k"] = torch.tensor([700, 333], dtype=torch.int32)
+    for b, L in enumerate(inp["seqlens_k"].tolist()):
+        inp["k"][b, L:] = float("nan")
+        inp["v"][b, L:] = float("nan")
+    nqb, nkb = _nb(c)
+    m = _mask((1, c.Hq, nqb, nkb), 0.6, seed=236)
+    for w in (-1, 250):
+        got, ref = _bwd(inp, c, m, window_left=w, seed=237)
+        compare_grads(got, ref, what=f"bwd block-sparse + key padding, window {w}")

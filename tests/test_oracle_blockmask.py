@@ -179,3 +179,19 @@ def test_gradients_torch_autograd(causal):
     of, _ = oracle.attn_fwd(q, k, v, 0.25, causal, seqlens_k=seqlens, block_mask=m,
                             block_size=bs)
     assert np.abs(of - o.detach().numpy()).max() < 1e-12
+
+
+@pytest.mark.parametrize("nq,nk,causal", [(300, 500, True), (300, 500, False), (600, 200, True),
+                                          (256, 256, True)])
+def test_block_pair_counts_of_the_flop_accounting(nq, nk, causal):
+    # the per-block visible pairs add up to the whole problem's, and a block
+    # mask's count equals the element-by-element count of its visible pairs
+    from io_aware_exact_29_b200 import accounting
+    cnt = accounting.block_pair_counts(nq, nk, causal, block=128)
+    assert cnt.sum() == accounting.visible_pairs(nq, nk, causal)
+    m = _mask((2, 3) + cnt.shape, 0.5, seed=nq + nk)
+    i = np.arange(nq)[:, None]
+    j = np.arange(nk)[None, :]
+    vis = (j <= i + nk - nq) if causal else np.ones((nq, nk), bool)
+    el = m.repeat(128, 2).repeat(128, 3)[:, :, :nq, :nk].astype(bool) & vis
+    assert accounting.blocksparse_flops(m, nq, nk, 64, causal, 2, 3) == 4 * 64 * int(el.sum())
