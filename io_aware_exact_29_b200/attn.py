@@ -124,7 +124,8 @@ def block_mask_args(block_mask, B, Hq, Nq, Nk):
     nqb >= ceil(Nq / 128), nkb >= ceil(Nk / 128) and unit stride along key
     blocks; a size-1 batch or head dimension is shared (stride 0).
     """
-    _dev(block_mask, "block_mask")
+    if not block_mask.is_cuda:  # strided views are fine: only the key-block stride must be 1
+        raise ValueError("block_mask must be a CUDA tensor")
     if block_mask.dtype not in (torch.uint8, torch.bool):
         raise TypeError("block_mask must be uint8 or bool")
     if block_mask.dim() != 4 or block_mask.shape[0] not in (1, B) or \
