@@ -24,7 +24,9 @@
 // while the softmax of Q1 works on S1_j it runs PV0_j and S0_{j+1}.  MMAs from
 // one thread execute in issue order, so when S_a_j is complete the previous
 // P_a·V has finished reading P_a and updating O_a: the softmax may rescale
-// O_a and overwrite P_a without another wait.
+// O_a and overwrite P_a without another wait.  Each P_a·V is issued in two
+// halves of 64 keys, the first as soon as the softmax has written the first
+// half of P_a, so that it overlaps the exponentials of the second half.
 //
 // Fused masks: the causal rule (adaptation point 2 of the ai6s.net article)
 // and the per-sequence key length (point 3) are index arithmetic on the score
@@ -72,6 +74,7 @@ struct FwdBars {
     uint64_t v_empty[VST];
     uint64_t s_full[2];
     uint64_t p_full[2];
+    uint64_t p_half[2];  // first half of P (keys 0..63) is in tensor memory
     uint64_t o_done[2];
     uint64_t drain;
     uint32_t tmem_base;
@@ -248,6 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&bars->q_full[a], 1);
             ptx::mbar_init(&bars->s_full[a], 1);
             ptx::mbar_init(&bars->p_full[a], 128);
+            ptx::mbar_init(&bars->p_half[a], 128);
             ptx::mbar_init(&bars->o_done[a], 1);
         }
         for (int s = 0; s < KST; ++s) {
@@ -367,12 +371,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             // P_a·V of the tile at stream position t, the Q tile's ia-th tile;
             // last: the Q tile's O is complete after it
             auto issue_pv = [&](int a, int t, int ia, bool last) {
-                if (!wait_or_fail(&bars->p_full[a], ia & 1, 5)) return;
+                if (!wait_or_fail(&bars->p_half[a], ia & 1, 5)) return;
                 if (!wait_or_fail(&bars->v_full[t % VST], (t / VST) & 1, 6)) return;
                 ptx::tc_fence_after();
                 const uint32_t v_addr = sbase + L::kV + (t % VST) * kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                    if (kk == kBlockN / 32) {
+                        if (!wait_or_fail(&bars->p_full[a], ia & 1, 5)) return;
+                        ptx::tc_fence_after();
+                    }
                     ptx::umma_ts(tmem + col_o[a], tmem + col_s[a] + kk * 8,
                                  ptx::sdesc_sw128(v_addr + kk * 16 * 128, kBlockBytes, 1024),
                                  kIdescO, (ia > 0 || kk > 0) ? 1u : 0u);
@@ -502,37 +510,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
             const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
             const uint64_t nm_2 = ptx::f2_pack(-m_use, -m_use);
-            uint64_t acc2[4] = {0, 0, 0, 0};  // four pair accumulators of the row sum
-            // pass 2: exponentials per half; P of half hf goes to columns
-            // [32 hf, 32 hf + 32) of S_a, which pass 2 has already consumed
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t r[2][32];
-                ptx::tmem_ld32(t_s + hf * 64, r[0]);
-                ptx::tmem_ld32(t_s + hf * 64 + 32, r[1]);
-                ptx::tmem_wait_ld_dep(r[0]);
-                ptx::tmem_wait_ld_dep(r[1]);
-                uint32_t pk[32];
-                if (masked)
-                    half_exp<true, kWindow, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
-                                                              row_lim, sl2_2,
-                                                     nm_2, acc2, pk);
-                else
-                    half_exp<false, kWindow, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
-                                                               row_lim, sl2_2,
-                                                      nm_2, acc2, pk);
-                ptx::tmem_st32(t_s + hf * 32, pk);
-            }
-            float s0, s1, s2, s3, s4, s5, s6, s7;
-            ptx::f2_unpack(acc2[0], s0, s1);
-            ptx::f2_unpack(acc2[1], s2, s3);
-            ptx::f2_unpack(acc2[2], s4, s5);
-            ptx::f2_unpack(acc2[3], s6, s7);
-            const float rowsum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
-            l_sum = l_sum * alpha + rowsum;
             if (__any_sync(0xffffffffu, rescale)) {
                 // the previous P_a V has completed (it precedes S_a_j); done
-                // after the exponentials so that the score registers are free
+                // before the exponentials, since the first half of P_a V may
+                // start while the second half of P_a is still being formed
                 const float s = rescale ? alpha : 1.f;
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
@@ -570,8 +551,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ptx::fence_proxy_async_smem();
             }
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&bars->p_full[a]);
+            uint64_t acc2[4] = {0, 0, 0, 0};  // four pair accumulators of the row sum
+            // pass 2: exponentials per half; P of half hf goes to columns
+            // [32 hf, 32 hf + 32) of S_a, which pass 2 has already consumed,
+            // and is published on its own barrier (p_half, then p_full) so
+            // that the MMA of keys 0..63 overlaps the exponentials of 64..127
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t r[2][32];
+                ptx::tmem_ld32(t_s + hf * 64, r[0]);
+                ptx::tmem_ld32(t_s + hf * 64 + 32, r[1]);
+                ptx::tmem_wait_ld_dep(r[0]);
+                ptx::tmem_wait_ld_dep(r[1]);
+                uint32_t pk[32];
+                if (masked)
+                    half_exp<true, kWindow, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
+                                                              row_lim, sl2_2,
+                                                     nm_2, acc2, pk);
+                else
+                    half_exp<false, kWindow, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
+                                                               row_lim, sl2_2,
+                                                      nm_2, acc2, pk);
+                ptx::tmem_st32(t_s + hf * 32, pk);
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(hf == 0 ? &bars->p_half[a] : &bars->p_full[a]);
+            }
+            float s0, s1, s2, s3, s4, s5, s6, s7;
+            ptx::f2_unpack(acc2[0], s0, s1);
+            ptx::f2_unpack(acc2[1], s2, s3);
+            ptx::f2_unpack(acc2[2], s4, s5);
+            ptx::f2_unpack(acc2[3], s6, s7);
+            const float rowsum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+            l_sum = l_sum * alpha + rowsum;
             ++ia;
         }
 
