@@ -225,7 +225,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                (long long)(qbase / kBlockM) * p.bmask.srow;
     // key tile j is used by Q0 when j in [j00, nt0), by Q1 when j in
     // [j01, nt1), and (block-sparse) when the mask entry of the pair is set;
-    // the K/V stream is the union of the two, in increasing j
+    // without a block mask the K/V stream is the union of the two, in
+    // increasing j
     auto use = [&](int a, int j) -> bool {
         bool u = a == 0 ? (cnt0 > 0 && j >= j00 && j < nt0) : (cnt1 > 0 && j >= j01 && j < nt1);
         if constexpr (kSparse) {
@@ -245,6 +246,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             last1 = j;
             break;
         }
+    // Block-sparse schedule: the two Q tiles walk their own tile lists in
+    // lockstep.  Step i pairs the i-th key tile of Q0 with the i-th of Q1, and
+    // the K/V stream loads Q0's tile, then Q1's when it is a different one, so
+    // that masks that differ between the two cost max(n0, n1) steps, not the
+    // size of the union.
+    int n0 = 0, n1 = 0;  // key tiles of each Q tile
+    if constexpr (kSparse) {
+        for (int j = j00; cnt0 > 0 && j < nt0; ++j) n0 += use(0, j) ? 1 : 0;
+        for (int j = j01; cnt1 > 0 && j < nt1; ++j) n1 += use(1, j) ? 1 : 0;
+    }
+    const int nsteps = max(n0, n1);
+    struct PairStep {
+        int x0, x1;      // key tiles of Q0 and Q1 (when has0 / has1)
+        int pos0, pos1;  // their positions in the K/V stream
+        bool has0, has1, shared;
+    };
+    // c0, c1: next candidate tile of each Q tile; si: step; pos: next position
+    auto next_pair = [&](int& c0, int& c1, int& si, int& pos) -> PairStep {
+        PairStep st;
+        st.has0 = si < n0;
+        st.has1 = si < n1;
+        st.x0 = st.x1 = st.pos0 = st.pos1 = -1;
+        if (st.has0) {
+            while (c0 < nt0 - 1 && !use(0, c0)) ++c0;
+            st.x0 = c0++;
+        }
+        if (st.has1) {
+            while (c1 < nt1 - 1 && !use(1, c1)) ++c1;
+            st.x1 = c1++;
+        }
+        st.shared = st.has0 && st.has1 && st.x0 == st.x1;
+        if (st.has0) st.pos0 = pos++;
+        if (st.has1) st.pos1 = st.shared ? st.pos0 : pos++;
+        ++si;
+        return st;
+    };
 
     if (tid == 0) {
         for (int a = 0; a < 2; ++a) {
@@ -297,9 +334,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 issued_q[a] = true;
             }
             int t = -1;  // position of tile j in the stream
-            for (int j = jstart; j < nt; ++j) {
+            int c0 = j00, c1 = j01, si = 0, spos = 0;  // block-sparse schedule
+            PairStep st{};
+            int e = 1;   // block-sparse: which tile of step st comes next
+            const int n_iter = kSparse ? 2 * nsteps : nt - jstart;
+            for (int it = 0; it < n_iter; ++it) {
+                int j;
                 if constexpr (kSparse) {
-                    if (!use(0, j) && !use(1, j)) continue;
+                    if (e == 1) {
+                        st = next_pair(c0, c1, si, spos);
+                        e = 0;
+                    } else {
+                        e = 1;
+                    }
+                    const bool has = e == 0 ? st.has0 : (st.has1 && !st.shared);
+                    if (!has) continue;
+                    j = e == 0 ? st.x0 : st.x1;
+                } else {
+                    j = jstart + it;
                 }
                 ++t;
                 const int sk = t % KST;
@@ -387,6 +439,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (last) ptx::umma_commit(&bars->o_done[a]);
             };
+            if constexpr (kSparse) {
+                // lockstep steps: S0_i, PV1_{i-1}, S1_i, PV0_i, a stage is
+                // released after its last user's product
+                int c0 = j00, c1 = j01, si = 0, spos = 0;
+                PairStep prev{};
+                bool have_prev = false;
+                for (int i = 0; ok && i <= nsteps; ++i) {
+                    PairStep st{};
+                    if (i < nsteps) {
+                        st = next_pair(c0, c1, si, spos);
+                        if (st.has0) {
+                            if (!wait_or_fail(&bars->k_full[st.pos0 % KST], (st.pos0 / KST) & 1,
+                                              4))
+                                break;
+                            ptx::tc_fence_after();
+                            issue_s(0, st.pos0);
+                            if (!ok) break;
+                            if (!st.shared) ptx::umma_commit(&bars->k_empty[st.pos0 % KST]);
+                        }
+                    }
+                    if (have_prev && prev.has1) {
+                        issue_pv(1, prev.pos1, i - 1, i - 1 == n1 - 1);
+                        if (!ok) break;
+                        ptx::umma_commit(&bars->v_empty[prev.pos1 % VST]);
+                    }
+                    if (i < nsteps) {
+                        if (st.has1) {
+                            if (!st.shared) {
+                                if (!wait_or_fail(&bars->k_full[st.pos1 % KST],
+                                                  (st.pos1 / KST) & 1, 4))
+                                    break;
+                                ptx::tc_fence_after();
+                            }
+                            issue_s(1, st.pos1);
+                            if (!ok) break;
+                            ptx::umma_commit(&bars->k_empty[st.pos1 % KST]);
+                        }
+                        if (st.has0) {
+                            issue_pv(0, st.pos0, i, i == n0 - 1);
+                            if (!ok) break;
+                            if (!st.shared) ptx::umma_commit(&bars->v_empty[st.pos0 % VST]);
+                        }
+                    }
+                    prev = st;
+                    have_prev = i < nsteps;
+                }
+            } else {
             // a stage is released after its last user's product
             int t = 0, i0 = 0, i1 = 0;                      // stream position, per-tile counts
             int prev_t = 0, prev_i1 = 0, prev_j = -1;       // the previous tile of the stream
@@ -396,7 +495,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (j < nt) {
                     u0 = use(0, j);
                     u1 = use(1, j);
-                    if (kSparse && !u0 && !u1) continue;
                     if (!wait_or_fail(&bars->k_full[t % KST], (t / KST) & 1, 4)) break;
                     ptx::tc_fence_after();
                     if (u0) issue_s(0, t);
@@ -425,6 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 i1 += u1 ? 1 : 0;
                 ++t;
             }
+            }  // dense / window stream
             if (!ok) {
                 // make sure no MMA is still running before TMEM is freed
                 int zero = 0;
@@ -455,17 +554,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_o = tmem + lane_addr + (a == 0 ? 256u : 256u + D);
 
         int ia = 0;  // key tiles of this Q tile done so far
-        int tu = 0;  // block-sparse: stream position of the next tile of the union
-        for (int j = kSparse ? jstart : ja; j < nta; ++j) {
-            int t;  // stream position of tile j
+        int c0 = j00, c1 = j01, si = 0, spos = 0;  // block-sparse schedule
+        const int n_iter = kSparse ? (a == 0 ? n0 : n1) : max(0, nta - ja);
+        for (int it = 0; it < n_iter; ++it) {
+            int j, t;         // key tile, its stream position
+            bool first_user;  // this Q tile's P·V is the first to read V_j
             if constexpr (kSparse) {
-                if (!use(a, j)) {
-                    if (use(1 - a, j)) ++tu;
-                    continue;
-                }
-                t = tu++;
+                const PairStep st = next_pair(c0, c1, si, spos);
+                j = a == 0 ? st.x0 : st.x1;
+                t = a == 0 ? st.pos0 : st.pos1;
+                first_user = a == 0 || !st.shared;
             } else {
+                j = ja + it;
                 t = j - jstart;
+                first_user = a == 0 || !use(0, j);
             }
             if (!warp_wait(&bars->s_full[a], ia & 1, p.limit_ns, abort_flag)) {
                 record_error(p.err, kErrFwdBase + 7, &bars->abort);
@@ -527,10 +629,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tmem_wait_st();
             }
             ptx::tmem_wait_st();
-            // the Q tile that uses key tile j first zeroes its V rows behind
-            // the real length (Q0 if it uses the tile, else Q1)
-            const bool zero_v = p.seqlens_k != nullptr && key0 + kBlockN > Lk &&
-                                (a == 0 || !use(0, j));
+            // the Q tile whose P·V reads V_j first zeroes its rows behind the
+            // real length (Q0 if it uses the tile, else Q1)
+            const bool zero_v = p.seqlens_k != nullptr && key0 + kBlockN > Lk && first_user;
             if (zero_v) {
                 // keys behind the real length: zero their V rows so that a
                 // non-finite value stored there cannot reach O through 0 * NaN
