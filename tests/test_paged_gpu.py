@@ -100,3 +100,25 @@ def test_bad_table_entry_is_reported():
                                 dev["block_table"], dev["seqlens_k"], 500, scale=c.scale)
     torch.cuda.synchronize()
     assert attn.get_device_error() == attn.ERR_DECODE_BASE + 8
+
+
+def test_llama70b_shape_paged_bs16_sampled_sequences():
+    # the bench's paged decode at full size (B=32, Hq=64, Hkv=8, d=128, lengths
+    # up to 32768, 16-row blocks, shuffled table); sampled sequences against
+    # the oracle, the shortest and longest included
+    from io_aware_exact_29_b200.workloads import DECODE_CASES
+    c = DECODE_CASES["llama70b_decode"]
+    inp = kvcache_inputs(c, seed=0)
+    pg = paged_from_packed(inp, 16, seed=0)
+    o, lse, _ = _run(inp, pg, c)
+    lens = inp["seqlens_k"].tolist()
+    cu = inp["cu_seqlens_k"].tolist()
+    pick = sorted(set([int(np.argmin(lens)), int(np.argmax(lens)), 3, 11, 30]))
+    for b in pick:
+        sub_k = inp["k_cache"][cu[b]:cu[b + 1]]
+        sub_v = inp["v_cache"][cu[b]:cu[b + 1]]
+        o_ref, lse_ref = oracle.attn_kvcache(inp["q"][b:b + 1], sub_k, sub_v,
+                                             torch.tensor([0, cu[b + 1] - cu[b]]),
+                                             inp["seqlens_k"][b:b + 1], c.scale, c.causal)
+        compare(o[b:b + 1], lse[b:b + 1], o_ref, lse_ref,
+                what=f"paged bs16 seq {b} len {lens[b]}")
