@@ -582,8 +582,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             float mx8[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
+            // d = 128 keeps the first half of the row in registers for pass 2
+            // (one tensor-memory round trip less per tile; at d = 64 the
+            // extra registers cost more than the load)
+            uint32_t rs[2][2][32];
             {
-                uint32_t r[2][2][32];
+                auto& r = rs;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     ptx::tmem_ld32(t_s + hf * 64, r[hf][0]);
@@ -659,11 +663,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             // that the MMA of keys 0..63 overlaps the exponentials of 64..127
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                uint32_t r[2][32];
-                ptx::tmem_ld32(t_s + hf * 64, r[0]);
-                ptx::tmem_ld32(t_s + hf * 64 + 32, r[1]);
-                ptx::tmem_wait_ld_dep(r[0]);
-                ptx::tmem_wait_ld_dep(r[1]);
+                constexpr int kKept = D == 128 ? 1 : 0;  // halves kept from pass 1
+                uint32_t rl[2][32];
+                if (hf >= kKept) {
+                    ptx::tmem_ld32(t_s + hf * 64, rl[0]);
+                    ptx::tmem_ld32(t_s + hf * 64 + 32, rl[1]);
+                    ptx::tmem_wait_ld_dep(rl[0]);
+                    ptx::tmem_wait_ld_dep(rl[1]);
+                }
+                auto& r = hf >= kKept ? rl : rs[hf];
                 uint32_t pk[32];
                 if (masked)
                     half_exp<true, kWindow, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
