@@ -487,10 +487,28 @@ def cpu_baseline(budget_s: float = 15.0):
         t = time.perf_counter()
         oracle.attn_fwd(inp["q"], inp["k"], inp["v"], fc.scale, fc.causal, rows=rows)
         dt = time.perf_counter() - t
-    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s",
-            "cores": oracle.max_threads(), "kind": "oracle",
-            "sample": (f"fwd workload B=4 H=16 N=4096 d=128: {len(rows)} seeded query rows "
-                       f"per head x all 64 heads x all 4096 keys, fp64 ({dt:.1f} s)")}
+    cores = oracle.max_threads()
+    out = {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s",
+           "cores": cores, "kind": "oracle",
+           "sample": (f"fwd workload B=4 H=16 N=4096 d=128: {len(rows)} seeded query rows "
+                      f"per head x all 64 heads x all 4096 keys, fp64 ({dt:.1f} s)")}
+    # the tiny configuration (B=1 H=2 N=128 d=64, non-causal and causal) on one core
+    tc = FWD_CASES["tiny"]
+    tin = fwd_inputs(tc, seed=0)
+    oracle.set_threads(1)
+    try:
+        per = {}
+        for causal in (False, True):
+            reps, t = 0, time.perf_counter()
+            while reps < 3 or time.perf_counter() - t < 0.5:
+                oracle.attn_fwd(tin["q"], tin["k"], tin["v"], tc.scale, causal)
+                reps += 1
+            per["causal" if causal else "non_causal"] = round(
+                (time.perf_counter() - t) / reps * 1e3, 3)
+    finally:
+        oracle.set_threads(cores)
+    out["tiny_one_core_ms"] = per
+    return out
 
 
 def run_reference(args, rank, world):
