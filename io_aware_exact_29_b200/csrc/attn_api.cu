@@ -162,6 +162,11 @@ int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse,
     p.seqlens_k = Nk > 0 ? seqlens_k : nullptr;
     p.window_left = window_left;
     p.bmask = bmask;
+    // causal row tiles differ in cost (tile t sees about t key tiles): launch
+    // them in decreasing cost across all heads (a sliding window evens the
+    // costs out, and keeps the head-major order for its L2 reuse)
+    p.heavy_first = causal && window_left < 0 && (Nq + 255) / 256 <= 65535 &&
+                    (long long)B * Hq <= 0x7fffffffLL;
     p.lse = lse;
     p.limit_ns = limit_ns;
     p.inject = inject;
@@ -499,6 +504,11 @@ int attn_bwd_blocksparse(const void* q, const void* k, const void* v, const void
     p.seqlens_k = Nk > 0 ? seqlens_k : nullptr;
     p.window_left = window_left;
     p.bmask = BlockMask{block_mask, mask_stride_b, mask_stride_h, mask_stride_row};
+    // decreasing-cost launch order for causal, as in the forward; measured
+    // on one B200 it gains 5-8% at d = 64 and loses 4-6% at d = 128, where
+    // every head's Q, dO, K and V in flight at once exceed the L2
+    p.heavy_first = causal && d == 64 && window_left < 0 && (Nq + 127) / 128 <= 65535 &&
+                    (Nk + 127) / 128 <= 65535 && (long long)B * Hq <= 0x7fffffffLL;
     p.o = o;
     p.dout = dout;
     p.lse = lse;

@@ -199,9 +199,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = &bars->abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int k0 = blockIdx.x * kBlock;
-    const int g = blockIdx.y;
-    const int b = blockIdx.z;
+    // causal: grid (B*Hkv, key tiles), the first key tiles (seen by the most
+    // query tiles) launch first across all heads; otherwise (key tiles, Hkv, B)
+    const int kt = p.heavy_first ? (int)blockIdx.y : (int)blockIdx.x;
+    const int k0 = kt * kBlock;
+    const int g = p.heavy_first ? (int)(blockIdx.x % (unsigned)p.Hkv) : (int)blockIdx.y;
+    const int b = p.heavy_first ? (int)(blockIdx.x / (unsigned)p.Hkv) : (int)blockIdx.z;
     const int Lk = p.seqlens_k ? p.seqlens_k[b] : p.Nk;
     const int off = Lk - p.Nq;  // key j visible to query i iff j <= i + off (causal)
     // query tiles that see at least one key of this tile
@@ -224,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const long long hq = g * p.G + sa / nqs;
             const long long qt = qt_first + sa % nqs;
             return __ldg(p.bmask.m + (long long)b * p.bmask.sb + hq * p.bmask.sh +
-                         qt * p.bmask.srow + blockIdx.x) != 0;
+                         qt * p.bmask.srow + kt) != 0;
         }
         return true;
     };
@@ -599,9 +602,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = &bars->abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int i0 = blockIdx.x * kBlock;
-    const int h = blockIdx.y;
-    const int b = blockIdx.z;
+    // causal: grid (B*Hq, query tiles), the last query tiles (which see the
+    // most keys) launch first across all heads; otherwise (query tiles, Hq, B)
+    const int n_qt = (p.Nq + kBlock - 1) / kBlock;
+    const int qt = p.heavy_first ? (n_qt - 1 - (int)blockIdx.y) : (int)blockIdx.x;
+    const int i0 = qt * kBlock;
+    const int h = p.heavy_first ? (int)(blockIdx.x % (unsigned)p.Hq) : (int)blockIdx.y;
+    const int b = p.heavy_first ? (int)(blockIdx.x / (unsigned)p.Hq) : (int)blockIdx.z;
     const int g = h / p.G;
     const int Lk = p.seqlens_k ? p.seqlens_k[b] : p.Nk;
     const int off = Lk - p.Nq;
@@ -614,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const unsigned char* mrow = nullptr;
     if constexpr (kSparse)
         mrow = p.bmask.m + (long long)b * p.bmask.sb + (long long)h * p.bmask.sh +
-               (long long)blockIdx.x * p.bmask.srow;
+               (long long)qt * p.bmask.srow;
     // the absolute key tile after jj that takes part (jj = j0 - 1: the first)
     auto next_tile = [&](int jj) -> int {
         if constexpr (kSparse) {
@@ -934,12 +941,15 @@ cudaError_t launch_bwd_s(const BwdMaps& m, const BwdParams& p, cudaStream_t stre
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.Nk > 0) {
-        dim3 g1((p.Nk + kBlock - 1) / kBlock, p.Hkv, p.B);
+        const unsigned nkt = (unsigned)((p.Nk + kBlock - 1) / kBlock);
+        const dim3 g1 = p.heavy_first ? dim3((unsigned)p.B * p.Hkv, nkt, 1)
+                                      : dim3(nkt, p.Hkv, p.B);
         k1<<<g1, kThreads, L1::kAlloc, stream>>>(m.q, m.k, m.v, m.dout, p);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    dim3 g2((p.Nq + kBlock - 1) / kBlock, p.Hq, p.B);
+    const unsigned nqt = (unsigned)((p.Nq + kBlock - 1) / kBlock);
+    const dim3 g2 = p.heavy_first ? dim3((unsigned)p.B * p.Hq, nqt, 1) : dim3(nqt, p.Hq, p.B);
     k2<<<g2, kThreads, L2::kAlloc, stream>>>(m.q, m.k, m.v, m.dout, p);
     return cudaGetLastError();
 }

@@ -197,10 +197,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = tid & 31;
 
     // ---- work unit: rows [qbase, qbase + 256) of head h of batch b
+    // causal: the grid is (B*Hq, row tiles) with the costliest (last) row
+    // tile first for every head, so that blocks launch in decreasing cost
+    // across all heads; otherwise (row tiles, Hq, B), consecutive blocks
+    // sharing a head's K/V in L2
     const int n_ctiles = (p.Nq + 2 * kBlockM - 1) / (2 * kBlockM);
-    const int ct = p.causal ? (n_ctiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-    const int h = blockIdx.y;
-    const int b = blockIdx.z;
+    const int ct = p.heavy_first ? (n_ctiles - 1 - (int)blockIdx.y) : (int)blockIdx.x;
+    const int h = p.heavy_first ? (int)(blockIdx.x % (unsigned)p.Hq) : (int)blockIdx.y;
+    const int b = p.heavy_first ? (int)(blockIdx.x / (unsigned)p.Hq) : (int)blockIdx.z;
     const int g = h / p.G;
     const int Lk = p.seqlens_k ? p.seqlens_k[b] : p.Nk;
     const int qbase = ct * 2 * kBlockM;
@@ -766,7 +770,9 @@ cudaError_t launch_fwd_w(const FwdMaps& maps, const FwdParams& p, cudaStream_t s
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc);
     if (e != cudaSuccess) return e;
-    dim3 grid((p.Nq + 2 * kBlockM - 1) / (2 * kBlockM), p.Hq, p.B);
+    const unsigned n_ctiles = (unsigned)((p.Nq + 2 * kBlockM - 1) / (2 * kBlockM));
+    const dim3 grid = p.heavy_first ? dim3((unsigned)p.B * p.Hq, n_ctiles, 1)
+                                    : dim3(n_ctiles, p.Hq, p.B);
     kern<<<grid, kThreads, L::kAlloc, stream>>>(maps.q, maps.k, maps.v, maps.o, p);
     return cudaGetLastError();
 }

@@ -34,6 +34,7 @@ struct FwdParams {
     const int* seqlens_k;  // [B] or nullptr
     int window_left;       // -1, or keys before i + (Lk - Nq) - window_left are masked
     BlockMask bmask;       // block-sparse mask, or m == nullptr
+    int heavy_first;       // grid (B*Hq, tiles): the costliest tile index launches first
     float* lse;            // [B, Hq, Nq]
     unsigned long long limit_ns;
     int inject;       // self-test: the loader skips everything
@@ -57,6 +58,7 @@ struct BwdParams {
     const int* seqlens_k;  // [B] or nullptr
     int window_left;       // -1, or keys before i + (Lk - Nq) - window_left are masked
     BlockMask bmask;       // block-sparse mask, or m == nullptr
+    int heavy_first;       // grids (B*H, tiles): the costliest tile index launches first
     const void* o;         // [B, Nq, Hq, d] forward output
     const void* dout;      // [B, Nq, Hq, d]
     const float* lse;      // [B, Hq, Nq] forward log-sum-exp (natural log)
