@@ -163,10 +163,17 @@ int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse,
     p.window_left = window_left;
     p.bmask = bmask;
     // causal row tiles differ in cost (tile t sees about t key tiles): launch
-    // them in decreasing cost across all heads (a sliding window evens the
-    // costs out, and keeps the head-major order for its L2 reuse)
-    p.heavy_first = causal && window_left < 0 && (Nq + 255) / 256 <= 65535 &&
-                    (long long)B * Hq <= 0x7fffffffLL;
+    // them in decreasing cost, in bands of heads whose K/V fit in L2 together
+    // (a sliding window evens the costs out and keeps the head-major order)
+    p.band = 0;
+    if (causal && window_left < 0 && Nk > 0) {
+        const long long units = (long long)B * Hq * ((Nq + 255) / 256);
+        // K and V bytes of one query head, shared by the G heads of its group
+        const long long per_head = 4LL * Nk * d / (Hq / Hkv);
+        const long long fit = (48LL << 20) / (per_head > 0 ? per_head : 1);
+        if (units <= 0x7fffffffLL)
+            p.band = (int)std::min<long long>((long long)B * Hq, std::max<long long>(8, fit));
+    }
     p.lse = lse;
     p.limit_ns = limit_ns;
     p.inject = inject;
@@ -504,11 +511,22 @@ int attn_bwd_blocksparse(const void* q, const void* k, const void* v, const void
     p.seqlens_k = Nk > 0 ? seqlens_k : nullptr;
     p.window_left = window_left;
     p.bmask = BlockMask{block_mask, mask_stride_b, mask_stride_h, mask_stride_row};
-    // decreasing-cost launch order for causal, as in the forward; measured
-    // on one B200 it gains 5-8% at d = 64 and loses 4-6% at d = 128, where
-    // every head's Q, dO, K and V in flight at once exceed the L2
-    p.heavy_first = causal && d == 64 && window_left < 0 && (Nq + 127) / 128 <= 65535 &&
-                    (Nk + 127) / 128 <= 65535 && (long long)B * Hq <= 0x7fffffffLL;
+    // decreasing-cost launch order for causal, as in the forward, in bands
+    // whose streamed operands fit in L2 together: a dK/dV block streams Q and
+    // dO of the G heads of its kv head, a dQ block K and V of its kv head
+    p.band_kv = p.band_q = 0;
+    if (causal && window_left < 0 && Nk > 0) {
+        const int G = Hq / Hkv;
+        const long long nkt = (Nk + 127) / 128, nqt = (Nq + 127) / 128;
+        const long long per_kv = 4LL * Nq * d * G;        // Q + dO of a group
+        const long long per_q = 4LL * Nk * d / G;         // K + V, shared by G heads
+        const long long fit_kv = (48LL << 20) / (per_kv > 0 ? per_kv : 1);
+        const long long fit_q = (48LL << 20) / (per_q > 0 ? per_q : 1);
+        if ((long long)B * Hkv * nkt <= 0x7fffffffLL)
+            p.band_kv = (int)std::min<long long>((long long)B * Hkv, std::max<long long>(8, fit_kv));
+        if ((long long)B * Hq * nqt <= 0x7fffffffLL)
+            p.band_q = (int)std::min<long long>((long long)B * Hq, std::max<long long>(8, fit_q));
+    }
     p.o = o;
     p.dout = dout;
     p.lse = lse;

@@ -199,12 +199,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = &bars->abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // causal: grid (B*Hkv, key tiles), the first key tiles (seen by the most
-    // query tiles) launch first across all heads; otherwise (key tiles, Hkv, B)
-    const int kt = p.heavy_first ? (int)blockIdx.y : (int)blockIdx.x;
+    // causal: a 1-D grid in bands of (b, kv head) pairs, the first key tiles
+    // (seen by the most query tiles) first; otherwise (key tiles, Hkv, B)
+    int kt, g, b;
+    if (p.band_kv > 0) {
+        int pair, rank;
+        band_unit(blockIdx.x, p.band_kv, p.B * p.Hkv, (p.Nk + kBlock - 1) / kBlock, pair, rank);
+        kt = rank;
+        g = pair % p.Hkv;
+        b = pair / p.Hkv;
+    } else {
+        kt = blockIdx.x;
+        g = blockIdx.y;
+        b = blockIdx.z;
+    }
     const int k0 = kt * kBlock;
-    const int g = p.heavy_first ? (int)(blockIdx.x % (unsigned)p.Hkv) : (int)blockIdx.y;
-    const int b = p.heavy_first ? (int)(blockIdx.x / (unsigned)p.Hkv) : (int)blockIdx.z;
     const int Lk = p.seqlens_k ? p.seqlens_k[b] : p.Nk;
     const int off = Lk - p.Nq;  // key j visible to query i iff j <= i + off (causal)
     // query tiles that see at least one key of this tile
@@ -602,13 +611,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = &bars->abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // causal: grid (B*Hq, query tiles), the last query tiles (which see the
-    // most keys) launch first across all heads; otherwise (query tiles, Hq, B)
+    // causal: a 1-D grid in bands of (b, q head) pairs, the last query tiles
+    // (which see the most keys) first; otherwise (query tiles, Hq, B)
     const int n_qt = (p.Nq + kBlock - 1) / kBlock;
-    const int qt = p.heavy_first ? (n_qt - 1 - (int)blockIdx.y) : (int)blockIdx.x;
+    int qt, h, b;
+    if (p.band_q > 0) {
+        int pair, rank;
+        band_unit(blockIdx.x, p.band_q, p.B * p.Hq, n_qt, pair, rank);
+        qt = n_qt - 1 - rank;
+        h = pair % p.Hq;
+        b = pair / p.Hq;
+    } else {
+        qt = blockIdx.x;
+        h = blockIdx.y;
+        b = blockIdx.z;
+    }
     const int i0 = qt * kBlock;
-    const int h = p.heavy_first ? (int)(blockIdx.x % (unsigned)p.Hq) : (int)blockIdx.y;
-    const int b = p.heavy_first ? (int)(blockIdx.x / (unsigned)p.Hq) : (int)blockIdx.z;
     const int g = h / p.G;
     const int Lk = p.seqlens_k ? p.seqlens_k[b] : p.Nk;
     const int off = Lk - p.Nq;
@@ -942,14 +960,14 @@ cudaError_t launch_bwd_s(const BwdMaps& m, const BwdParams& p, cudaStream_t stre
     if (e != cudaSuccess) return e;
     if (p.Nk > 0) {
         const unsigned nkt = (unsigned)((p.Nk + kBlock - 1) / kBlock);
-        const dim3 g1 = p.heavy_first ? dim3((unsigned)p.B * p.Hkv, nkt, 1)
+        const dim3 g1 = p.band_kv > 0 ? dim3((unsigned)p.B * p.Hkv * nkt, 1, 1)
                                       : dim3(nkt, p.Hkv, p.B);
         k1<<<g1, kThreads, L1::kAlloc, stream>>>(m.q, m.k, m.v, m.dout, p);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     const unsigned nqt = (unsigned)((p.Nq + kBlock - 1) / kBlock);
-    const dim3 g2 = p.heavy_first ? dim3((unsigned)p.B * p.Hq, nqt, 1) : dim3(nqt, p.Hq, p.B);
+    const dim3 g2 = p.band_q > 0 ? dim3((unsigned)p.B * p.Hq * nqt, 1, 1) : dim3(nqt, p.Hq, p.B);
     k2<<<g2, kThreads, L2::kAlloc, stream>>>(m.q, m.k, m.v, m.dout, p);
     return cudaGetLastError();
 }

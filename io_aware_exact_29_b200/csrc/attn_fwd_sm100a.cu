@@ -197,14 +197,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = tid & 31;
 
     // ---- work unit: rows [qbase, qbase + 256) of head h of batch b
-    // causal: the grid is (B*Hq, row tiles) with the costliest (last) row
-    // tile first for every head, so that blocks launch in decreasing cost
-    // across all heads; otherwise (row tiles, Hq, B), consecutive blocks
+    // causal: a 1-D grid in bands of (b, h) pairs, the costliest (last) row
+    // tile of every pair of a band first, so that blocks launch in
+    // decreasing cost; otherwise (row tiles, Hq, B), consecutive blocks
     // sharing a head's K/V in L2
     const int n_ctiles = (p.Nq + 2 * kBlockM - 1) / (2 * kBlockM);
-    const int ct = p.heavy_first ? (n_ctiles - 1 - (int)blockIdx.y) : (int)blockIdx.x;
-    const int h = p.heavy_first ? (int)(blockIdx.x % (unsigned)p.Hq) : (int)blockIdx.y;
-    const int b = p.heavy_first ? (int)(blockIdx.x / (unsigned)p.Hq) : (int)blockIdx.z;
+    int ct, h, b;
+    if (p.band > 0) {
+        int pair, rank;
+        band_unit(blockIdx.x, p.band, p.B * p.Hq, n_ctiles, pair, rank);
+        ct = n_ctiles - 1 - rank;
+        h = pair % p.Hq;
+        b = pair / p.Hq;
+    } else {
+        ct = blockIdx.x;
+        h = blockIdx.y;
+        b = blockIdx.z;
+    }
     const int g = h / p.G;
     const int Lk = p.seqlens_k ? p.seqlens_k[b] : p.Nk;
     const int qbase = ct * 2 * kBlockM;
@@ -771,8 +780,8 @@ cudaError_t launch_fwd_w(const FwdMaps& maps, const FwdParams& p, cudaStream_t s
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc);
     if (e != cudaSuccess) return e;
     const unsigned n_ctiles = (unsigned)((p.Nq + 2 * kBlockM - 1) / (2 * kBlockM));
-    const dim3 grid = p.heavy_first ? dim3((unsigned)p.B * p.Hq, n_ctiles, 1)
-                                    : dim3(n_ctiles, p.Hq, p.B);
+    const dim3 grid = p.band > 0 ? dim3((unsigned)p.B * p.Hq * n_ctiles, 1, 1)
+                                 : dim3(n_ctiles, p.Hq, p.B);
     kern<<<grid, kThreads, L::kAlloc, stream>>>(maps.q, maps.k, maps.v, maps.o, p);
     return cudaGetLastError();
 }

@@ -25,6 +25,21 @@ struct BlockMask {
     int srow;
 };
 
+// Launch order of a grid over (b, head) pairs x tiles whose tiles differ in
+// cost (causal): a 1-D grid in bands of `band` pairs; inside a band the
+// costliest tile rank of every pair comes first, then the next rank.  Block
+// u -> (pair, tile rank 0 = costliest).  Bands bound the K/V (or Q/dO) set
+// in flight, so that it stays in L2.
+__device__ __forceinline__ void band_unit(unsigned u, int band, int n_pairs, int n_tiles,
+                                          int& pair, int& rank) {
+    const unsigned per_band = (unsigned)band * (unsigned)n_tiles;
+    const int bi = (int)(u / per_band);
+    const int r = (int)(u - (unsigned)bi * per_band);
+    const int hb = min(band, n_pairs - bi * band);  // pairs in this band
+    rank = r / hb;
+    pair = bi * band + (r - rank * hb);
+}
+
 struct FwdParams {
     int B, Hq, Hkv, Nq, Nk;
     int G;            // Hq / Hkv
@@ -34,7 +49,7 @@ struct FwdParams {
     const int* seqlens_k;  // [B] or nullptr
     int window_left;       // -1, or keys before i + (Lk - Nq) - window_left are masked
     BlockMask bmask;       // block-sparse mask, or m == nullptr
-    int heavy_first;       // grid (B*Hq, tiles): the costliest tile index launches first
+    int band;              // >0: 1-D grid, bands of `band` (b, h) pairs, costliest tiles first
     float* lse;            // [B, Hq, Nq]
     unsigned long long limit_ns;
     int inject;       // self-test: the loader skips everything
@@ -58,7 +73,8 @@ struct BwdParams {
     const int* seqlens_k;  // [B] or nullptr
     int window_left;       // -1, or keys before i + (Lk - Nq) - window_left are masked
     BlockMask bmask;       // block-sparse mask, or m == nullptr
-    int heavy_first;       // grids (B*H, tiles): the costliest tile index launches first
+    int band_kv;           // >0: dK/dV grid in bands of (b, kv head) pairs, costliest first
+    int band_q;            // >0: dQ grid in bands of (b, q head) pairs, costliest first
     const void* o;         // [B, Nq, Hq, d] forward output
     const void* dout;      // [B, Nq, Hq, d]
     const float* lse;      // [B, Hq, Nq] forward log-sum-exp (natural log)
