@@ -31,7 +31,15 @@
 // Fused masks: the causal rule (adaptation point 2 of the ai6s.net article)
 // and the per-sequence key length (point 3) are index arithmetic on the score
 // row; tiles wholly outside them are never loaded, and V rows behind the real
-// length are zeroed in shared memory so that 0 * NaN cannot reach O.
+// length are zeroed in shared memory so that 0 * NaN cannot reach O.  Two
+// more instances add the mask extensions: a sliding window (a lower edge on
+// each row, tiles before a Q tile's window skipped) and a block mask over
+// 128 x 128 tiles, where the two Q tiles walk their own tile lists in
+// lockstep.
+//
+// Launch order: causal row tiles differ in cost, so the causal grid is 1-D,
+// in bands of (batch, head) pairs whose K/V fit in L2 together, the costliest
+// row tile of every pair of a band first.
 //
 // Lazy rescaling: the reference maximum of a row only moves when a tile's
 // maximum exceeds it by more than 8 (log2 units), so P <= 2^8; numerator and
