@@ -539,7 +539,11 @@ def run_reference(args, rank, world):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16 inputs widened to fp64)",
-        "config": {"workload": "fwd: B=4 H=16 N=4096 d=128 non-causal (sampled query rows)"},
+        "config": {"workload": ("fwd: long-sequence sweep point B=4 H=16 N=4096 d=128 "
+                                "non-causal (the value: the forward TFLOP/s, as in the "
+                                "kernel arm; the oracle takes a sample of query rows per step)"),
+                   "fwd": {"B": fc.B, "H": fc.Hq, "N": fc.Nq, "d": fc.d, "causal": fc.causal},
+                   "parallelism": "rank 0 only, host cores"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
                          "cores": oracle.max_threads(), "kind": "oracle",
                          "sample": f"{len(rows)} query rows per head x 64 heads x 4096 keys"},
