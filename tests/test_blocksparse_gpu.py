@@ -203,3 +203,41 @@ def test_backward_with_key_padding_and_window():
     for w in (-1, 250):
         got, ref = _bwd(inp, c, m, window_left=w, seed=237)
         compare_grads(got, ref, what=f"bwd block-sparse + key padding, window {w}")
+
+
+@pytest.mark.parametrize("nq,nk", [(300, 900), (640, 384)])
+def test_rectangular_causal_bottom_right(nq, nk):
+    # fewer queries than keys (a chunk at the end of a long prefix) and more
+    # queries than keys (rows before the first key see nothing), causal
+    c = FwdCase("bsr", 2, 4, 2, nq, nk, 128, True)
+    inp = fwd_inputs(c, seed=240 + nq)
+    nqb, nkb = _nb(c)
+    m = _mask((c.B, c.Hq, nqb, nkb), 0.6, seed=241 + nk)
+    o, lse, _ = _fwd(inp, c, m)
+    o_ref, l_ref = oracle.attn_fwd(inp["q"], inp["k"], inp["v"], c.scale, True, block_mask=m,
+                                   block_size=BLK)
+    compare(o, lse, o_ref, l_ref, what=f"block-sparse causal {nq}x{nk}")
+
+
+def test_d64_fp16_with_key_padding():
+    c = FwdCase("bs64", 3, 6, 2, 520, 600, 64, False, dtype="fp16")
+    inp = fwd_inputs(c, seed=242)
+    inp["seqlens_k"] = torch.tensor([600, 333, 129], dtype=torch.int32)
+    for b, L in enumerate(inp["seqlens_k"].tolist()):
+        inp["k"][b, L:] = float("nan")
+        inp["v"][b, L:] = float("nan")
+    nqb, nkb = _nb(c)
+    m = _mask((c.B, c.Hq, nqb, nkb), 0.5, seed=243)
+    o, lse, _ = _fwd(inp, c, m)
+    o_ref, l_ref = oracle.attn_fwd(inp["q"], inp["k"], inp["v"], c.scale, False,
+                                   seqlens_k=inp["seqlens_k"], block_mask=m, block_size=BLK)
+    compare(o, lse, o_ref, l_ref, what="block-sparse d64 fp16 key padding")
+
+
+def test_backward_d64_fp16_causal_rectangular():
+    c = FwdCase("bsb64", 2, 4, 1, 300, 520, 64, True, dtype="fp16")
+    inp = fwd_inputs(c, seed=244)
+    nqb, nkb = _nb(c)
+    m = _mask((c.B, c.Hq, nqb, nkb), 0.6, seed=245)
+    got, ref = _bwd(inp, c, m, seed=246)
+    compare_grads(got, ref, what="bwd block-sparse d64 fp16 causal 300x520")
