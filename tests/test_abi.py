@@ -76,6 +76,15 @@ def test_blocksparse_rejects_bad_masks(mask, sb, sh, srow):
     assert rc == -1
 
 
+@pytest.mark.parametrize("sb,sh,srow", [(-1, 0, 8), (0, -16, 8), (0, 0, 7)])
+def test_bwd_blocksparse_rejects_bad_masks(sb, sh, srow):
+    lib = attn.load_library()
+    ws = attn.bwd_workspace_bytes(1, 2, 300)
+    rc = lib.attn_bwd_blocksparse(P, P, P, P, P, P, P, P, P, 1, 2, 1, 300, 1000, 128, 0.09, 0,
+                                  -1, 0, None, P, sb, sh, srow, P, ws, None)
+    assert rc == -1
+
+
 def test_decode_rejects_bad_arguments():
     lib = attn.load_library()
     base = dict(q=P, k=P, v=P, cu=P, sl=P, maxl=100, slots=100, o=P, lse=P, B=2, Hq=8, Hkv=2,
