@@ -37,6 +37,10 @@
  *    runs out records an error word, read with attn_get_device_error().
  *  - Thread safety: calls are independent (tensor maps are built per call
  *    and passed by value to the kernel).
+ *  - One exception to both of the last two points:
+ *    attn_fwd_varlen_kvcache_noalloc uses a scratch array that the library
+ *    itself holds in device memory (one per device, shared by every call), so
+ *    calls of it that overlap on the GPU must be serialised by the caller.
  */
 #ifndef ATTN_B200_H
 #define ATTN_B200_H
@@ -289,13 +293,18 @@ ATTN_API int attn_bwd_blocksparse(const void* q, const void* k, const void* v, c
  *    call returns ATTN_ERR_WORKSPACE before queuing any work.
  *  - Set-up: the first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current) and caches it; make
- *    that first call before any stream capture on the device.
+ *    that first call before any stream capture on the device.  The address
+ *    is looked up again when the current context is not the one it was taken
+ *    in (a device reset destroys the context and may move the array); make
+ *    the first call after a reset before any stream capture too.
  *  - Sharing: every GPU that loads the library holds the array until the
  *    process exits, and all calls on a device share it.  It keeps whatever the
  *    last call left; each call clears the parts that must start at zero (the
  *    split counters) on `stream` before its kernel.  Calls that overlap on the
  *    GPU (other streams, other host threads) race on it: serialise them.
- * Returns the same status codes as attn_fwd_varlen_kvcache.
+ * Returns the same status codes as attn_fwd_varlen_kvcache for the same
+ * arguments (its argument checks run first, in the same order), plus
+ * ATTN_ERR_WORKSPACE for sizes beyond the scratch.
  */
 ATTN_API int attn_fwd_varlen_kvcache_noalloc(const void* q, const void* k_cache,
                                              const void* v_cache, const int* cu_seqlens_k,
@@ -326,8 +335,51 @@ ATTN_API int attn_get_device_error(int* code, void* stream);
 ATTN_API int attn_selftest_watchdog(const void* q, const void* k, const void* v, void* o, float* lse,
                            int limit_ms, void* stream);
 
+/*
+ * Schedule introspection (host only, no device work): the mappings the
+ * kernels use, evaluated by the same code on the host so that a model of the
+ * schedule can be checked against them.
+ *
+ * attn_schedule_band_unit: the launch order of causal grids.  Causal row
+ * tiles differ in cost (ai6s.net article, section "ops-transformer 里的
+ * FlashAttention 做了什么额外的事", point 2: the causal mask is fused into
+ * the blockwise computation and tiles above the diagonal are skipped), so
+ * the 1-D grid runs in bands of `band` (batch, head) pairs and, inside a
+ * band, the costliest tile rank of every pair first.  Block u of a grid of
+ * n_pairs x n_tiles blocks runs *pair, tile rank *rank (0 = costliest).
+ * Requires 0 < band <= n_pairs, n_tiles > 0, u < n_pairs * n_tiles;
+ * returns ATTN_OK or ATTN_ERR_INVALID_ARG.
+ *
+ * attn_schedule_sparse_steps: the lockstep walk of a block-sparse forward
+ * CTA's two 128-row query tiles over their key tiles.  m0, m1: host arrays of
+ * one byte per key tile (nonzero = the tile takes part); Q tile a considers
+ * key tiles [j0a, nta).  Writes 7 ints per step to steps[7 * i ...]:
+ * x0, x1 (key tiles, -1 when absent), pos0, pos1 (their K/V stream
+ * positions), has0, has1, shared (the step's two tiles are one load).
+ * Returns the number of steps (max of the two tile counts), or
+ * ATTN_ERR_INVALID_ARG when it exceeds max_steps or an argument is invalid.
+ */
+ATTN_API int attn_schedule_band_unit(unsigned u, int band, int n_pairs, int n_tiles, int* pair,
+                                     int* rank);
+ATTN_API int attn_schedule_sparse_steps(const unsigned char* m0, const unsigned char* m1, int nt0,
+                                        int nt1, int j00, int j01, int max_steps, int* steps);
+
 /* Library version string. */
 ATTN_API const char* attn_version(void);
+
+/*
+ * Measurement helper, not part of the attention path: reads `bytes` of device
+ * memory at `src` once (16-byte loads that do not allocate in L1) on
+ * `stream` and writes one XOR-folded word per CTA to out[0 .. n_ctas-1].
+ * Timing it gives the read-only device-memory bandwidth, the roofline
+ * denominator of the decode, which reads its KV cache once and writes next to
+ * nothing (ai6s.net article, section "标准注意力的致命伤不在算力，在搬运":
+ * attention is bound by data movement).  src and bytes multiples of 16;
+ * out holds n_ctas words (1 <= n_ctas <= 2^20).  Returns ATTN_OK,
+ * ATTN_ERR_INVALID_ARG or ATTN_ERR_CUDA (launch failure).
+ */
+ATTN_API int attn_hbm_read_probe(const void* src, size_t bytes, unsigned* out, int n_ctas,
+                                 void* stream);
 
 #ifdef __cplusplus
 }

@@ -80,6 +80,13 @@ def load_library():
             lib.attn_selftest_watchdog.argtypes = [vp, vp, vp, vp, vp, i, vp]
             lib.attn_selftest_watchdog.restype = i
             lib.attn_version.restype = ctypes.c_char_p
+            lib.attn_hbm_read_probe.argtypes = [vp, sz, vp, i, vp]
+            lib.attn_hbm_read_probe.restype = i
+            ip = ctypes.POINTER(i)
+            lib.attn_schedule_band_unit.argtypes = [ctypes.c_uint, i, i, i, ip, ip]
+            lib.attn_schedule_band_unit.restype = i
+            lib.attn_schedule_sparse_steps.argtypes = [vp, vp, i, i, i, i, i, ip]
+            lib.attn_schedule_sparse_steps.restype = i
             _lib = lib
     return _lib
 
@@ -346,6 +353,42 @@ def selftest_watchdog(q, k, v, out, lse, limit_ms=200, stream=None):
                                                out.data_ptr(), lse.data_ptr(), int(limit_ms),
                                                _stream_ptr(stream))
     _check("attn_selftest_watchdog", rc)
+
+
+def hbm_read_probe(buf: torch.Tensor, out: torch.Tensor, n_ctas: int, stream=None):
+    """Measurement helper: read `buf` (contiguous CUDA tensor, size a multiple
+    of 16 bytes) once; `out` is an int32/uint32 CUDA tensor of >= n_ctas words."""
+    _dev(buf, "buf")
+    _dev(out, "out")
+    if out.numel() * out.element_size() < 4 * n_ctas:
+        raise ValueError("out holds fewer than n_ctas words")
+    _check("attn_hbm_read_probe",
+           load_library().attn_hbm_read_probe(buf.data_ptr(), buf.numel() * buf.element_size(),
+                                              out.data_ptr(), int(n_ctas), _stream_ptr(stream)))
+
+
+def schedule_band_unit(u: int, band: int, n_pairs: int, n_tiles: int):
+    """(pair, tile rank) that block u of a banded causal grid runs (host only)."""
+    pair, rank = ctypes.c_int(-1), ctypes.c_int(-1)
+    _check("attn_schedule_band_unit",
+           load_library().attn_schedule_band_unit(u, band, n_pairs, n_tiles, ctypes.byref(pair),
+                                                  ctypes.byref(rank)))
+    return pair.value, rank.value
+
+
+def schedule_sparse_steps(m0, m1, nt0, nt1, j00=0, j01=0):
+    """The block-sparse forward's lockstep steps (host only): a list of dicts
+    with x0, x1, pos0, pos1, has0, has1, shared."""
+    n = max(len(m0), len(m1), 1)
+    a = (ctypes.c_ubyte * n)(*[1 if x else 0 for x in m0])
+    b = (ctypes.c_ubyte * n)(*[1 if x else 0 for x in m1])
+    out = (ctypes.c_int * (7 * n))()
+    r = load_library().attn_schedule_sparse_steps(a, b, nt0, nt1, j00, j01, n, out)
+    if r < 0:
+        raise AttnError("attn_schedule_sparse_steps", r)
+    keys = ("x0", "x1", "pos0", "pos1", "has0", "has1", "shared")
+    return [{k: (bool(out[7 * i + c]) if c >= 4 else out[7 * i + c]) for c, k in enumerate(keys)}
+            for i in range(r)]
 
 
 def version() -> str:

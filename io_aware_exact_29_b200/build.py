@@ -20,7 +20,7 @@ INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 BUILD_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libattn.so")
 SOURCES = ["attn_api.cu", "attn_fwd_sm100a.cu", "attn_bwd_sm100a.cu", "attn_decode_sm100a.cu",
-           "attn_decode_tc_sm100a.cu", "attn_decode_noalloc.cu"]
+           "attn_decode_tc_sm100a.cu", "attn_decode_noalloc.cu", "attn_probe.cu"]
 HEADERS = ["ptx.cuh", "attn_internal.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -191,6 +191,29 @@ unsigned* device_error_word() {
     return g_err_addr[dev];
 }
 
+int decode_check_args(const void* q, const void* k_cache, const void* v_cache,
+                      const int* cu_seqlens_k, const int* seqlens_k, int max_seqlen_k,
+                      int cache_slots, const void* o, const float* lse, int B, int Hq, int Hkv,
+                      int Nq, int d, float scale, int dtype, int split_keys) {
+    if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq <= 0 || Nq > 16)
+        return ATTN_ERR_INVALID_ARG;
+    if (B > 65535 || Hkv > 65535 || max_seqlen_k < 0 || cache_slots <= 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (split_keys < 0 || (split_keys % 64) != 0) return ATTN_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    if (!q || !k_cache || !v_cache || !cu_seqlens_k || !seqlens_k || !o || !lse)
+        return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+        !aligned16(lse) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) ||
+        (reinterpret_cast<uintptr_t>(seqlens_k) & 3u))
+        return ATTN_ERR_INVALID_ARG;
+    const DecodeLayout lay = decode_layout(B, Hq, Hkv, Nq, d, max_seqlen_k, split_keys);
+    if (lay.max_splits * lay.n_mgroups > 2147483647 / 2) return ATTN_ERR_INVALID_ARG;
+    return ATTN_OK;
+}
+
 }  // namespace attn
 
 using namespace attn;
@@ -228,6 +251,46 @@ int attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, f
                       stream, 0, kDefaultLimitNs, window_left, bm);
 }
 
+int attn_schedule_band_unit(unsigned u, int band, int n_pairs, int n_tiles, int* pair,
+                            int* rank) {
+    if (!pair || !rank || band <= 0 || n_pairs <= 0 || n_tiles <= 0 || band > n_pairs)
+        return ATTN_ERR_INVALID_ARG;
+    if ((unsigned long long)u >= (unsigned long long)n_pairs * (unsigned long long)n_tiles)
+        return ATTN_ERR_INVALID_ARG;
+    band_unit(u, band, n_pairs, n_tiles, *pair, *rank);
+    return ATTN_OK;
+}
+
+int attn_schedule_sparse_steps(const unsigned char* m0, const unsigned char* m1, int nt0,
+                               int nt1, int j00, int j01, int max_steps, int* steps) {
+    if (!m0 || !m1 || !steps || nt0 < 0 || nt1 < 0 || j00 < 0 || j01 < 0 || max_steps < 0)
+        return ATTN_ERR_INVALID_ARG;
+    const int cnt0 = nt0 - j00 > 0 ? nt0 - j00 : 0, cnt1 = nt1 - j01 > 0 ? nt1 - j01 : 0;
+    auto use = [&](int a, int j) -> bool {
+        const bool in = a == 0 ? (cnt0 > 0 && j >= j00 && j < nt0)
+                               : (cnt1 > 0 && j >= j01 && j < nt1);
+        return in && (a == 0 ? m0[j] : m1[j]) != 0;
+    };
+    int n0 = 0, n1 = 0;
+    for (int j = j00; cnt0 > 0 && j < nt0; ++j) n0 += use(0, j) ? 1 : 0;
+    for (int j = j01; cnt1 > 0 && j < nt1; ++j) n1 += use(1, j) ? 1 : 0;
+    const int nsteps = n0 > n1 ? n0 : n1;
+    if (nsteps > max_steps) return ATTN_ERR_INVALID_ARG;
+    int c0 = j00, c1 = j01, si = 0, pos = 0;
+    for (int i = 0; i < nsteps; ++i) {
+        const PairStep st = sparse_next_step(use, n0, n1, nt0, nt1, c0, c1, si, pos);
+        int* r = steps + 7 * i;
+        r[0] = st.x0;
+        r[1] = st.x1;
+        r[2] = st.pos0;
+        r[3] = st.pos1;
+        r[4] = st.has0;
+        r[5] = st.has1;
+        r[6] = st.shared;
+    }
+    return nsteps;
+}
+
 int attn_selftest_watchdog(const void* q, const void* k, const void* v, void* o, float* lse,
                            int limit_ms, void* stream) {
     if (limit_ms <= 0 || limit_ms > 10000) return ATTN_ERR_INVALID_ARG;
@@ -248,27 +311,16 @@ int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_ca
                             int cache_slots, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
                             int d, float scale, int causal, int dtype, void* workspace,
                             size_t workspace_bytes, int split_keys, void* stream) {
-    if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED;
-    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Nq <= 0 || Nq > 16)
-        return ATTN_ERR_INVALID_ARG;
-    if (B > 65535 || Hkv > 65535 || max_seqlen_k < 0 || cache_slots <= 0)
-        return ATTN_ERR_INVALID_ARG;
-    if (split_keys < 0 || (split_keys % 64) != 0) return ATTN_ERR_INVALID_ARG;
-    if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
-    if (!q || !k_cache || !v_cache || !cu_seqlens_k || !seqlens_k || !o || !lse)
-        return ATTN_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
-        !aligned16(lse) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) ||
-        (reinterpret_cast<uintptr_t>(seqlens_k) & 3u))
-        return ATTN_ERR_INVALID_ARG;
+    const int arg_st = attn::decode_check_args(q, k_cache, v_cache, cu_seqlens_k, seqlens_k,
+                                               max_seqlen_k, cache_slots, o, lse, B, Hq, Hkv,
+                                               Nq, d, scale, dtype, split_keys);
+    if (arg_st != ATTN_OK) return arg_st;
     int dev = 0;
     const int st = check_device(&dev);
     if (st == 0) return ATTN_ERR_CUDA;
     if (st < 0) return ATTN_ERR_UNSUPPORTED;
 
     const DecodeLayout lay = decode_layout(B, Hq, Hkv, Nq, d, max_seqlen_k, split_keys);
-    if (lay.max_splits * lay.n_mgroups > 2147483647 / 2) return ATTN_ERR_INVALID_ARG;
     if (!workspace || workspace_bytes < lay.total ||
         (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return ATTN_ERR_WORKSPACE;

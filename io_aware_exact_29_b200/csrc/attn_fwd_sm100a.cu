@@ -278,30 +278,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = j01; cnt1 > 0 && j < nt1; ++j) n1 += use(1, j) ? 1 : 0;
     }
     const int nsteps = max(n0, n1);
-    struct PairStep {
-        int x0, x1;      // key tiles of Q0 and Q1 (when has0 / has1)
-        int pos0, pos1;  // their positions in the K/V stream
-        bool has0, has1, shared;
-    };
     // c0, c1: next candidate tile of each Q tile; si: step; pos: next position
     auto next_pair = [&](int& c0, int& c1, int& si, int& pos) -> PairStep {
-        PairStep st;
-        st.has0 = si < n0;
-        st.has1 = si < n1;
-        st.x0 = st.x1 = st.pos0 = st.pos1 = -1;
-        if (st.has0) {
-            while (c0 < nt0 - 1 && !use(0, c0)) ++c0;
-            st.x0 = c0++;
-        }
-        if (st.has1) {
-            while (c1 < nt1 - 1 && !use(1, c1)) ++c1;
-            st.x1 = c1++;
-        }
-        st.shared = st.has0 && st.has1 && st.x0 == st.x1;
-        if (st.has0) st.pos0 = pos++;
-        if (st.has1) st.pos1 = st.shared ? st.pos0 : pos++;
-        ++si;
-        return st;
+        return sparse_next_step(use, n0, n1, nt0, nt1, c0, c1, si, pos);
     };
 
     if (tid == 0) {

@@ -30,14 +30,53 @@ struct BlockMask {
 // costliest tile rank of every pair comes first, then the next rank.  Block
 // u -> (pair, tile rank 0 = costliest).  Bands bound the K/V (or Q/dO) set
 // in flight, so that it stays in L2.
-__device__ __forceinline__ void band_unit(unsigned u, int band, int n_pairs, int n_tiles,
-                                          int& pair, int& rank) {
+__host__ __device__ __forceinline__ void band_unit(unsigned u, int band, int n_pairs, int n_tiles,
+                                                   int& pair, int& rank) {
     const unsigned per_band = (unsigned)band * (unsigned)n_tiles;
     const int bi = (int)(u / per_band);
     const int r = (int)(u - (unsigned)bi * per_band);
     const int hb = min(band, n_pairs - bi * band);  // pairs in this band
     rank = r / hb;
     pair = bi * band + (r - rank * hb);
+}
+
+// Block-sparse forward: the two 128-row Q tiles of a CTA walk their own
+// lists of key tiles in lockstep.  Step si pairs the si-th key tile of Q0
+// (x0, when si < n0) with the si-th of Q1 (x1, when si < n1); the K/V stream
+// loads x0, then x1 when it is a different tile, so a step holds one or two
+// stream positions (pos0, pos1; pos1 == pos0 when the tile is shared).  The
+// loader, the MMA issuer and the softmax warps all call this walk, each with
+// its own state (c0, c1: next candidate tile of each Q tile; si: step;
+// pos: next stream position), so they agree on every step.  use(a, j): key
+// tile j takes part for Q tile a; nt0, nt1: one past each Q tile's last
+// candidate tile.
+struct PairStep {
+    int x0, x1;      // key tiles of Q0 and Q1 (when has0 / has1)
+    int pos0, pos1;  // their positions in the K/V stream
+    bool has0, has1, shared;
+};
+
+template <class Use>
+__host__ __device__ __forceinline__ PairStep sparse_next_step(const Use& use, int n0, int n1,
+                                                              int nt0, int nt1, int& c0, int& c1,
+                                                              int& si, int& pos) {
+    PairStep st;
+    st.has0 = si < n0;
+    st.has1 = si < n1;
+    st.x0 = st.x1 = st.pos0 = st.pos1 = -1;
+    if (st.has0) {
+        while (c0 < nt0 - 1 && !use(0, c0)) ++c0;
+        st.x0 = c0++;
+    }
+    if (st.has1) {
+        while (c1 < nt1 - 1 && !use(1, c1)) ++c1;
+        st.x1 = c1++;
+    }
+    st.shared = st.has0 && st.has1 && st.x0 == st.x1;
+    if (st.has0) st.pos0 = pos++;
+    if (st.has1) st.pos1 = st.shared ? st.pos0 : pos++;
+    ++si;
+    return st;
 }
 
 struct FwdParams {
@@ -188,5 +227,13 @@ cudaError_t launch_decode_tc(const CUtensorMap& qmap, const CUtensorMap& kmap,
 
 // Address of the device error word on the current device.
 unsigned* device_error_word();
+
+// The argument checks of attn_fwd_varlen_kvcache that need no device and no
+// workspace (dtype and d first: ATTN_ERR_UNSUPPORTED; then sizes, scale,
+// pointers and alignment: ATTN_ERR_INVALID_ARG); ATTN_OK when they pass.
+int decode_check_args(const void* q, const void* k_cache, const void* v_cache,
+                      const int* cu_seqlens_k, const int* seqlens_k, int max_seqlen_k,
+                      int cache_slots, const void* o, const float* lse, int B, int Hq, int Hkv,
+                      int Nq, int d, float scale, int dtype, int split_keys);
 
 }  // namespace attn

@@ -2,6 +2,8 @@
 on the same stored bits, compare element by element."""
 from __future__ import annotations
 
+import math
+
 import numpy as np
 import torch
 
@@ -22,6 +24,7 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, rows=None, what=""):
         og, o_ref = og[:, rows], o_ref[:, rows]
         lg, lse_ref = lg[:, :, rows], lse_ref[:, :, rows]
     assert np.isfinite(og).all(), f"{what}: non-finite output"
+    assert not np.isnan(lg).any(), f"{what}: NaN in LSE"
     err = np.abs(og - o_ref)
     max_err, mean_err = float(err.max(initial=0.0)), float(err.mean()) if err.size else 0.0
     both_inf = np.isneginf(lg) & np.isneginf(lse_ref)
@@ -37,17 +40,70 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, rows=None, what=""):
     return max_err, mean_err, lse_err
 
 
+def compare_selected(o_gpu, lse_gpu, o_ref, lse_ref, sel, what=""):
+    """As compare, on the query rows selected per (batch, head): sel is a
+    bool array [B, H, Nq] (the reference may hold NaN elsewhere)."""
+    og = o_gpu.float().cpu().numpy().astype(np.float64)
+    lg = lse_gpu.float().cpu().numpy().astype(np.float64)
+    ob, ib, hb = np.nonzero(np.transpose(sel, (0, 2, 1)))  # [B, Nq, H] order
+    return compare(torch.from_numpy(og[ob, ib, hb][None, :, None]),
+                   torch.from_numpy(lg[ob, hb, ib][None, None, :]),
+                   o_ref[ob, ib, hb][None, :, None], lse_ref[ob, hb, ib][None, None, :],
+                   what=what)
+
+
 # Gradients (no tolerance is stated for them): errors normalised by the
 # reference tensor's own magnitude.  Rounding the output to bf16 alone gives
-# about 2^-10 mean and 2^-9 max relative error; P and dS are rounded to bf16
-# for the tensor-core products and D comes from the bf16 forward output, each
-# adding errors of the same order that average out over the sums.
+# about 2^-10 (1e-3) mean and 2^-9 max relative error; P and dS are rounded to
+# bf16 for the tensor-core products and D comes from the bf16 forward output,
+# each adding errors of the same order that partly average out over the sums,
+# so the mean bound is a few times 2^-10 (measured: about 2.3e-3 at every
+# shape, d = 64 and 128, causal or not, bf16 and fp16).
 # The normalisers have a floor of GRAD_FLOOR: where the exact gradient is 0
 # (one key: P = 1, so dS = dP - D = 0) the test is an absolute one, and with
 # N(0, 1) inputs the gradients of every real case are well above it.
 GRAD_MAX_REL = 2e-2   # max |err| / max(max |ref|, floor)
-GRAD_MEAN_REL = 1e-2  # mean |err| / max(mean |ref|, floor)
+GRAD_MEAN_REL = 5e-3  # mean |err| / max(mean |ref|, floor)
 GRAD_FLOOR = 1e-3
+
+
+# ---------------------------------------------------------------- canaries
+# The sanitizer is not available, so outputs and workspaces are placed inside
+# larger device buffers whose margins hold a byte pattern; after the run the
+# margins must be unchanged (no write past either end), and outputs are
+# prefilled with NaN so that an element the kernel never wrote shows up.
+GUARD_BYTES = 4096
+GUARD_BYTE = 0xA5
+
+
+class Guarded:
+    """A device tensor of `shape`/`dtype` at a 256-byte aligned offset inside a
+    buffer with GUARD_BYTES of pattern on each side; `t` is the tensor."""
+
+    def __init__(self, shape, dtype, fill=float("nan"), device="cuda"):
+        elem = torch.empty((), dtype=dtype).element_size()
+        self.nbytes = math.prod(shape) * elem
+        span = -(-self.nbytes // 256) * 256
+        self.raw = torch.full((2 * GUARD_BYTES + span,), GUARD_BYTE, dtype=torch.uint8,
+                              device=device)
+        self.t = self.raw[GUARD_BYTES:GUARD_BYTES + self.nbytes].view(dtype).view(shape)
+        if dtype == torch.uint8:
+            self.t.fill_(0x5A if fill != fill else int(fill))  # NaN -> a junk byte
+        else:
+            self.t.fill_(fill)
+
+    def check(self, what=""):
+        torch.cuda.synchronize()
+        front = self.raw[:GUARD_BYTES]
+        back = self.raw[GUARD_BYTES + self.nbytes:]
+        assert bool((front == GUARD_BYTE).all()), f"{what}: write before the start"
+        assert bool((back == GUARD_BYTE).all()), f"{what}: write past the end"
+
+
+def check_defined(what, *tensors):
+    """No NaN left in outputs that the kernels define everywhere."""
+    for t in tensors:
+        assert not bool(torch.isnan(t.float()).any()), f"{what}: NaN left in an output"
 
 
 def compare_grads(gpu, ref, what="", key_rows=None):
@@ -72,12 +128,21 @@ def compare_grads(gpu, ref, what="", key_rows=None):
 
 
 def run_fwd(inp, causal, scale=None):
+    """The forward on guarded, NaN-prefilled outputs; checks the guards and
+    that every output element was written."""
     q, k, v = inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda()
     sl = inp.get("seqlens_k")
     sl = None if sl is None else sl.cuda()
-    o, lse = attn.attn_fwd(q, k, v, scale=scale, causal=causal, seqlens_k=sl)
+    B, Nq, Hq, _ = q.shape
+    go = Guarded(tuple(q.shape), q.dtype)
+    gl = Guarded((B, Hq, Nq), torch.float32)
+    o, lse = attn.attn_fwd(q, k, v, scale=scale, causal=causal, seqlens_k=sl, out=go.t,
+                           lse=gl.t)
     torch.cuda.synchronize()
     assert attn.get_device_error() == 0
+    go.check("O")
+    gl.check("LSE")
+    check_defined("forward", o, lse)
     return o, lse
 
 

@@ -1,15 +1,19 @@
 """Backward pass (attn_bwd: dQ, dK, dV) against the fp64 oracle's gradients.
 
 The GPU forward provides O and LSE (as in training); the oracle recomputes
-everything from the same stored q, k, v, dO bits."""
+everything from the same stored q, k, v, dO bits.  Gradients and the
+workspace are guarded and NaN/junk-filled (tests/parity.py); the BERT-large
+shape is compared in full and the bench's shape (B=4, H=16, N=4096, d=128)
+on 16 of its 64 (batch, head) pairs, against the matrix-product oracle."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
+from oracle import dense
 from io_aware_exact_29_b200 import attn
 from io_aware_exact_29_b200.workloads import FWD_CASES, FwdCase, fwd_inputs, upstream_grad
-from tests.parity import compare_grads
+from tests.parity import Guarded, check_defined, compare_grads
 
 pytestmark = pytest.mark.gpu
 
@@ -18,10 +22,19 @@ def _run(inp, case, dout):
     dev = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
     o, lse = attn.attn_fwd(dev["q"], dev["k"], dev["v"], scale=case.scale, causal=case.causal,
                            seqlens_k=dev["seqlens_k"])
+    B, Nq, Hq, _ = inp["q"].shape
+    gq = Guarded(tuple(inp["q"].shape), inp["q"].dtype)
+    gk = Guarded(tuple(inp["k"].shape), inp["k"].dtype)
+    gv = Guarded(tuple(inp["v"].shape), inp["v"].dtype)
+    gw = Guarded((attn.bwd_workspace_bytes(B, Hq, Nq),), torch.uint8)
     dq, dk, dv = attn.attn_bwd(dev["q"], dev["k"], dev["v"], o, lse, dout.cuda(),
-                               scale=case.scale, causal=case.causal, seqlens_k=dev["seqlens_k"])
+                               scale=case.scale, causal=case.causal, seqlens_k=dev["seqlens_k"],
+                               workspace=gw.t, dq=gq.t, dk=gk.t, dv=gv.t)
     torch.cuda.synchronize()
     assert attn.get_device_error() == 0
+    for g, n in ((gq, "dq"), (gk, "dk"), (gv, "dv"), (gw, "workspace")):
+        g.check(n)
+    check_defined("backward", dq, dk, dv)
     return dq, dk, dv
 
 
@@ -74,29 +87,36 @@ def test_fp16():
     _check(c, seed=6, what="fp16")
 
 
-def test_bert_shape_sampled_batches():
-    # the BERT-large shape; the oracle checks two of the 16 batch entries
-    c = FWD_CASES["bert_large"]
+@pytest.mark.parametrize("name", ["bert_large", "bert_large_varlen", "gpt2"])
+def test_workload_shapes_in_full(name):
+    # every batch entry and head of the BERT-large (and its key-padded
+    # variant) and GPT-2 shapes against the matrix-product oracle
+    c = FWD_CASES[name]
     inp = fwd_inputs(c, seed=0)
     dout = upstream_grad(inp["q"], seed=0)
     got = _run(inp, c, dout)
-    for b in (0, 11):
-        ref = oracle.attn_bwd(inp["q"][b:b + 1], inp["k"][b:b + 1], inp["v"][b:b + 1],
-                              dout[b:b + 1], c.scale, c.causal)
-        compare_grads(tuple(t[b:b + 1] for t in got), ref, what=f"bert batch {b}")
+    ref = dense.attn_bwd(inp["q"], inp["k"], inp["v"], dout, c.scale, c.causal,
+                         seqlens_k=inp["seqlens_k"])
+    errs = compare_grads(got, ref, what=name)
+    print(name, {k: f"{a:.2e}/{b:.2e}" for k, (a, b) in errs.items()})
 
 
-def test_long_sequence_one_head():
-    # the bench's forward shape (B=4, H=16, N=4096, d=128); heads are
-    # independent (Hq = Hkv), so the oracle checks batch 1, head 5 alone
-    c = FWD_CASES["sweep_d128_n4096"]
+@pytest.mark.parametrize("causal", [False, True])
+def test_long_sequence_sixteen_heads(causal):
+    # the bench's forward shape (B=4, H=16, N=4096, d=128): heads are
+    # independent (Hq = Hkv), so the oracle checks 16 of the 64 (batch, head)
+    # pairs in full -- every batch entry, four heads each
+    c = FWD_CASES["sweep_d128_n4096_causal" if causal else "sweep_d128_n4096"]
     inp = fwd_inputs(c, seed=0)
     dout = upstream_grad(inp["q"], seed=0)
     got = _run(inp, c, dout)
-    sl = (slice(1, 2), slice(None), slice(5, 6))
-    ref = oracle.attn_bwd(inp["q"][sl], inp["k"][sl], inp["v"][sl], dout[sl], c.scale,
-                          c.causal)
-    compare_grads(tuple(t[sl] for t in got), ref, what="N=4096 d=128 b1 h5")
+    heads = (0, 5, 10, 15)
+    ref = dense.attn_bwd(inp["q"], inp["k"], inp["v"], dout, c.scale, c.causal,
+                         heads=[(b, h) for b in range(c.B) for h in heads])
+    sl = (slice(None), slice(None), list(heads))
+    errs = compare_grads(tuple(t[sl] for t in got), tuple(r[sl] for r in ref),
+                         what=f"N=4096 d=128 causal {causal}")
+    print(f"N=4096 causal {causal}", {k: f"{a:.2e}/{b:.2e}" for k, (a, b) in errs.items()})
 
 
 def test_repeatable_bit_for_bit():

@@ -29,7 +29,13 @@ def _worker(rank, world, port, out):
     assert (r, w) == (rank, world)
     bench.barrier(w)
     vals = bench.reduce_max([float(rank + 1), 10.0 - rank, 0.5 * rank], w)
-    out[rank] = torch.tensor(vals)
+    # the bench's aggregation: each rank timed `steps` steps of its own
+    # problems; value = units of all ranks / the slowest rank's time
+    steps, units = 20, 5.0e11
+    fwd_ms = [60.0, 75.0][rank]
+    (max_ms,) = bench.reduce_max([fwd_ms], w)
+    rate = bench.job_rate(units, steps, w, max_ms)
+    out[rank] = torch.tensor(vals + [max_ms, rate])
     bench.barrier(w)
     dist.destroy_process_group()
 
@@ -47,7 +53,11 @@ def test_max_over_ranks_with_gloo():
         p.join(timeout=120)
         assert p.exitcode == 0
     for r in range(world):
-        assert out[r].tolist() == [2.0, 10.0, 0.5]
+        got = out[r].tolist()
+        assert got[:3] == [2.0, 10.0, 0.5]
+        assert got[3] == 75.0
+        # 2 ranks x 20 steps x 5e11 units in 75 ms
+        assert abs(got[4] - 2 * 20 * 5.0e11 / 0.075) <= 1e-6 * got[4]
 
 
 def test_single_rank_needs_no_process_group():
@@ -55,3 +65,25 @@ def test_single_rank_needs_no_process_group():
 
     assert bench.reduce_max([1.0, 2.0], 1) == [1.0, 2.0]
     bench.barrier(1)
+
+
+def test_launch_plan():
+    import bench
+
+    assert bench.launch_plan(1, {}) == "run"
+    assert bench.launch_plan(8, {}) == "spawn"
+    assert bench.launch_plan(4, {"WORLD_SIZE": "4"}) == "run"
+    assert bench.launch_plan(8, {"WORLD_SIZE": "2"}).startswith("error")
+    assert bench.launch_plan(0, {}).startswith("error")
+
+
+def test_mismatched_world_size_is_refused():
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "8"], env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "WORLD_SIZE=2" in r.stderr

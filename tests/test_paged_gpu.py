@@ -1,15 +1,16 @@
 """Decode against a paged KV cache (attn_fwd_paged_kvcache) against the fp64
 oracle: block sizes below, at and above the 128-key tile, shuffled physical
 blocks with NaN in every unused row, and the fused append of the new tokens'
-K/V."""
+K/V.  Outputs and the workspace are guarded and NaN/junk-filled (tests/parity.py)."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
+from oracle import dense
 from io_aware_exact_29_b200 import attn
 from io_aware_exact_29_b200.workloads import DecodeCase, kvcache_inputs, paged_from_packed
-from tests.parity import compare
+from tests.parity import Guarded, check_defined, compare
 
 pytestmark = pytest.mark.gpu
 
@@ -19,12 +20,21 @@ LENS = [0, 1, 16, 127, 128, 129, 1000, 2049, 5000]
 def _run(inp, pg, c, with_new=False, split_keys=0):
     dev = {k: v.cuda() for k, v in pg.items()}
     ml = int(inp["seqlens_k"].max().item())
+    B, Nq, Hq, d = inp["q"].shape
+    go = Guarded((B, Nq, Hq, d), inp["q"].dtype)
+    gl = Guarded((B, Hq, Nq), torch.float32)
+    need = attn.decode_workspace_bytes(B, Hq, c.Hkv, Nq, d, ml, split_keys)
+    gw = Guarded((max(need, 1),), torch.uint8)
     o, lse = attn.attn_fwd_paged_kvcache(
         inp["q"].cuda(), dev["k_cache"], dev["v_cache"], dev["block_table"], dev["seqlens_k"], ml,
         scale=c.scale, causal=c.causal, k_new=dev.get("k_new") if with_new else None,
-        v_new=dev.get("v_new") if with_new else None, split_keys=split_keys)
+        v_new=dev.get("v_new") if with_new else None, split_keys=split_keys, workspace=gw.t,
+        out=go.t, lse=gl.t)
     torch.cuda.synchronize()
     assert attn.get_device_error() == 0
+    for g, n in ((go, "O"), (gl, "LSE"), (gw, "workspace")):
+        g.check(n)
+    check_defined("paged decode", o, lse)
     return o, lse, dev
 
 
@@ -102,23 +112,15 @@ def test_bad_table_entry_is_reported():
     assert attn.get_device_error() == attn.ERR_DECODE_BASE + 8
 
 
-def test_llama70b_shape_paged_bs16_sampled_sequences():
+def test_llama70b_shape_paged_bs16_in_full():
     # the bench's paged decode at full size (B=32, Hq=64, Hkv=8, d=128, lengths
-    # up to 32768, 16-row blocks, shuffled table); sampled sequences against
-    # the oracle, the shortest and longest included
+    # up to 32768, 16-row blocks, shuffled table, NaN in every unused row);
+    # every sequence against the matrix-product oracle on the paged layout
     from io_aware_exact_29_b200.workloads import DECODE_CASES
     c = DECODE_CASES["llama70b_decode"]
     inp = kvcache_inputs(c, seed=0)
     pg = paged_from_packed(inp, 16, seed=0)
     o, lse, _ = _run(inp, pg, c)
-    lens = inp["seqlens_k"].tolist()
-    cu = inp["cu_seqlens_k"].tolist()
-    pick = sorted(set([int(np.argmin(lens)), int(np.argmax(lens)), 3, 11, 30]))
-    for b in pick:
-        sub_k = inp["k_cache"][cu[b]:cu[b + 1]]
-        sub_v = inp["v_cache"][cu[b]:cu[b + 1]]
-        o_ref, lse_ref = oracle.attn_kvcache(inp["q"][b:b + 1], sub_k, sub_v,
-                                             torch.tensor([0, cu[b + 1] - cu[b]]),
-                                             inp["seqlens_k"][b:b + 1], c.scale, c.causal)
-        compare(o[b:b + 1], lse[b:b + 1], o_ref, lse_ref,
-                what=f"paged bs16 seq {b} len {lens[b]}")
+    o_ref, lse_ref = dense.attn_paged(inp["q"], pg["k_cache"], pg["v_cache"], pg["block_table"],
+                                      pg["seqlens_k"], c.scale, c.causal)
+    compare(o, lse, o_ref, lse_ref, what="paged bs16 Llama2-70B shape")

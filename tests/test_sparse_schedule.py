@@ -1,6 +1,8 @@
-"""A model, in Python, of the block-sparse forward's lockstep schedule (the
-loader, MMA-issuer and softmax loops of the kSparse kernel instance walk the
-same steps): over random mask pairs, every K/V stream position is loaded
+"""The block-sparse forward's lockstep schedule.  The steps come from the
+library's own walk (attn_schedule_sparse_steps runs on the host the
+sparse_next_step code that the kernel's loader, MMA issuer and softmax warps
+call) and must equal a Python statement of the walk; a model of the MMA
+issuer's order then checks, over random mask pairs, that every K/V stream position is loaded
 once, in order, each Q tile sees exactly its own tiles in increasing order,
 every stage is released exactly once and after its last reader, the Q tile
 that zeroes a V tile's padded rows is the first to read it, and no load waits
@@ -10,6 +12,8 @@ oracle in test_blocksparse_gpu.py."""
 import random
 
 import pytest
+
+from io_aware_exact_29_b200 import attn
 
 
 def _run(m0, m1, nt0, nt1, j00=0, j01=0, KST=2, VST=3):
@@ -31,6 +35,9 @@ def _run(m0, m1, nt0, nt1, j00=0, j01=0, KST=2, VST=3):
                 else: st['pos1'] = pos; pos += 1
             yield st
     steps = list(gen())
+    lib_steps = attn.schedule_sparse_steps([bool(x) for x in m0], [bool(x) for x in m1],
+                                           nt0, nt1, j00, j01)
+    assert lib_steps == steps, (lib_steps, steps)
     # loader
     loads = []
     for st in steps:

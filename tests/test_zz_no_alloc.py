@@ -55,6 +55,28 @@ def test_rejects_sizes_beyond_the_scratch_before_any_work():
     assert rc == -1
 
 
+def test_same_status_codes_as_the_workspace_entry_point():
+    # the argument checks run before the size check, so a head dim or dtype
+    # the decode does not take is reported as unsupported, as by the
+    # workspace entry point, and oversized batches as invalid
+    fn = _noalloc_fn()
+    lib = attn.load_library()
+    P = 1 << 20
+    cases = [
+        (96, 0, 32),      # d = 96: ATTN_ERR_UNSUPPORTED
+        (128, 7, 32),     # unknown dtype: ATTN_ERR_UNSUPPORTED
+        (128, 0, 70000),  # B > 65535: ATTN_ERR_INVALID_ARG
+    ]
+    for d, dtype, B in cases:
+        a = fn(P, P, P, P, P, 4096, 1 << 20, P, P, B, 64, 8, 1, d, 0.088, 0, dtype, 0, None)
+        b = lib.attn_fwd_varlen_kvcache(P, P, P, P, P, 4096, 1 << 20, P, P, B, 64, 8, 1, d,
+                                        0.088, 0, dtype, P, 1 << 30, 0, None)
+        assert a == b, (d, dtype, B, a, b)
+    assert fn(P, P, P, P, P, 4096, 1 << 20, P, P, 32, 64, 8, 1, 96, 0.088, 0, 0, 0, None) == -2
+    assert fn(P, P, P, P, P, 4096, 1 << 20, P, P, 70000, 64, 8, 1, 128, 0.088, 0, 0, 0,
+              None) == -1
+
+
 def _call_noalloc(fn, dev, case, max_len, split):
     o = torch.empty_like(dev["q"])
     lse = torch.empty((case.B, case.Hq, case.Nq), dtype=torch.float32, device="cuda")
