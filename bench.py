@@ -704,8 +704,11 @@ def run_profile_case(kernel: str, launches: int):
         for _ in range(2 + launches):
             attn.attn_bwd(fin["q"], fin["k"], fin["v"], o, lse, dout, scale=fc.scale,
                           causal=fc.causal)
-    elif kernel == "fwd":
-        fc = FWD_CASE
+    elif kernel.startswith("fwd"):
+        # fwd: the bench's forward; fwd_d64: the N=4096 d=64 sweep point
+        # (134 MB of inputs); fwd_gpt2 / fwd_bert: those workloads
+        fc = {"fwd": FWD_CASE, "fwd_d64": FWD_CASES["sweep_d64_n4096"],
+              "fwd_gpt2": FWD_CASES["gpt2"], "fwd_bert": FWD_CASES["bert_large"]}[kernel]
         fin = fwd_inputs(fc, seed=0, device="cuda")
         for _ in range(2 + launches):
             attn.attn_fwd(fin["q"], fin["k"], fin["v"], scale=fc.scale, causal=fc.causal)
@@ -716,7 +719,15 @@ def run_profile_case(kernel: str, launches: int):
         ml = int(din["seqlens_k"].max().item())
         ws = torch.empty(attn.decode_workspace_bytes(dc.B, dc.Hq, dc.Hkv, dc.Nq, dc.d, ml),
                          dtype=torch.uint8, device=dev)
-        for _ in range(2 + launches):
+        if kernel == "decode_paged":
+            # the same cache in 16-row blocks behind a shuffled table
+            pg = paged_from_packed({k: t.cpu() for k, t in din.items()}, 16, seed=3, fill=0.0)
+            pgd = {k: t.to(dev) for k, t in pg.items()}
+            for _ in range(2 + launches):
+                attn.attn_fwd_paged_kvcache(din["q"], pgd["k_cache"], pgd["v_cache"],
+                                            pgd["block_table"], pgd["seqlens_k"], ml,
+                                            scale=dc.scale, causal=dc.causal, workspace=ws)
+        for _ in range(2 + launches if kernel != "decode_paged" else 0):
             attn.attn_fwd_varlen_kvcache(din["q"], din["k_cache"], din["v_cache"],
                                          din["cu_seqlens_k"], din["seqlens_k"], ml,
                                          scale=dc.scale, causal=dc.causal, workspace=ws)
@@ -842,7 +853,9 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=32)
-    ap.add_argument("--profile", choices=["fwd", "bwd", "decode", "decode_chunk16"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "fwd_d64", "fwd_gpt2", "fwd_bert", "bwd", "decode",
+                                          "decode_chunk16", "decode_paged"],
+                    default=None,
                     help="run a small case of one kernel for an ncu capture and exit")
     ap.add_argument("--profile-launches", type=int, default=3)
     ap.add_argument("--sweep", action="store_true",
