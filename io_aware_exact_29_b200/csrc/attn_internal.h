@@ -81,6 +81,7 @@ __host__ __device__ __forceinline__ PairStep sparse_next_step(const Use& use, in
 
 struct FwdParams {
     int B, Hq, Hkv, Nq, Nk;
+    int n_ctas;       // CTAs launched; each takes every n_ctas-th work unit
     int G;            // Hq / Hkv
     int n_qtiles;     // ceil(Nq / 128)
     int causal;
@@ -89,6 +90,7 @@ struct FwdParams {
     int window_left;       // -1, or keys before i + (Lk - Nq) - window_left are masked
     BlockMask bmask;       // block-sparse mask, or m == nullptr
     int band;              // >0: 1-D grid, bands of `band` (b, h) pairs, costliest tiles first
+    void* o;               // [B, Nq, Hq, d]
     float* lse;            // [B, Hq, Nq]
     unsigned long long limit_ns;
     int inject;       // self-test: the loader skips everything
