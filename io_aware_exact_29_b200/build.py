@@ -19,9 +19,10 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 BUILD_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libattn.so")
-SOURCES = ["attn_api.cu", "attn_fwd_sm100a.cu", "attn_bwd_sm100a.cu", "attn_decode_sm100a.cu",
+SOURCES = ["attn_api.cu", "attn_fwd_sm100a.cu", "attn_fwd_persist_sm100a.cu", "attn_bwd_sm100a.cu",
+           "attn_decode_sm100a.cu",
            "attn_decode_tc_sm100a.cu", "attn_decode_noalloc.cu", "attn_probe.cu"]
-HEADERS = ["ptx.cuh", "attn_internal.h"]
+HEADERS = ["ptx.cuh", "attn_internal.h", "attn_fwd_common.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",

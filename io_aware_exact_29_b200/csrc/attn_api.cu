@@ -174,17 +174,18 @@ int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse,
         if (units <= 0x7fffffffLL)
             p.band = (int)std::min<long long>((long long)B * Hq, std::max<long long>(8, fit));
     }
-    // work units of 256 query rows.  Short units of equal cost (no causal
-    // mask or block mask, at most 4096 keys): one persistent CTA per SM takes
-    // every n_ctas-th unit, overlapping a unit's last tiles and output with
-    // the next unit's loads (+4-8% measured at 512-1024 keys, even at 4096).
-    // Causal and block-sparse units differ in cost, and a static split then
-    // leaves SMs idle at the end (-9 to -15% measured for causal); long units
-    // gain nothing from the overlap (-4% at 16384 keys).  Those grids keep
-    // one CTA per unit and let the hardware hand units to SMs as they free up.
+    // work units of 256 query rows.  Short units of equal cost (no causal,
+    // window or block mask, at most 4096 keys) go to the persistent kernel:
+    // one CTA per SM takes every n_ctas-th unit, overlapping a unit's last
+    // tiles and output with the next unit's loads (measured: BERT-large
+    // +9%, 1024 keys +4-11%, 4096 keys +-1% over one CTA per unit).  Causal
+    // and block-sparse units differ in cost, and a static split leaves SMs
+    // idle at the end (-9 to -15% measured for causal); long units gain
+    // nothing from the overlap (-4% at 16384 keys).  Those grids keep one
+    // CTA per unit and let the hardware hand units to SMs as they free up.
     const long long n_units = (long long)B * Hq * ((Nq + 255) / 256);
     if (n_units > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
-    const bool persist = p.band == 0 && bmask.m == nullptr && Nk <= 4096;
+    const bool persist = !causal && window_left < 0 && bmask.m == nullptr && Nk <= 4096;
     p.n_ctas = persist ? (int)std::min<long long>(n_units, g_sm_count[dev]) : (int)n_units;
     p.o = o;
     p.lse = lse;
@@ -192,7 +193,9 @@ int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse,
     p.inject = inject;
     p.err = g_err_addr[dev];
     // seqlens_k with Nk == 0 means every length is 0: same as no keys.
-    cudaError_t e = launch_fwd(maps, p, d, dtype == ATTN_BF16, static_cast<cudaStream_t>(stream));
+    cudaError_t e =
+        persist ? launch_fwd_persist(maps, p, d, dtype == ATTN_BF16, static_cast<cudaStream_t>(stream))
+                : launch_fwd(maps, p, d, dtype == ATTN_BF16, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -8,28 +8,16 @@
 // only O; the effectstory.com article "FlashAttention：IO 感知的精確注意力演算
 // 法..." states the same single pass: Q, K, V loaded once, O written once).
 //
-// Warp roles (384 threads):
+// Warp roles (320 threads):
 //   warps 0-3   softmax of Q0 (thread t owns query row t = TMEM lane t)
 //   warps 4-7   softmax of Q1
-//   warp 8      TMA loader: Q0, Q1 of each work unit, K_j / V_j into rings
+//   warp 8      TMA loader: Q0, Q1 once, then K_j / V_j into rings
 //   warp 9      tensor-memory owner and single-thread tcgen05.mma issuer
-//   warps 10-11 idle; with warps 8-9 they give registers to the softmax
-//               warpgroups (setmaxnreg), which keep a whole score row in
-//               registers between the two passes
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
 // O1 [256+D, 256+2D).  Each softmax thread reads its score row from S_a,
 // keeps the running max m and sum l (the online softmax of the section above),
 // and writes P (bf16/fp16) back over the first 64 columns of S_a; the P·V MMA
 // reads P straight from tensor memory as its A operand, V from shared memory.
-//
-// Persistent work units: a unit is two 128-row Q tiles of one (batch, head);
-// launched with one CTA per SM, each CTA takes every gridDim.x-th unit and
-// keeps its barriers, tensor memory and K/V ring across units, so that the
-// next unit's Q and K/V loads overlap the current unit's last tiles.  Before
-// the CTA's last unit each thread stores its own output row straight from
-// registers, which leaves the Q buffers free for the next unit's Q as soon as
-// the last S that reads them is complete; the last unit stages O in its Q
-// buffer and writes it with TMA stores.
 //
 // MMA issue order per key tile j:  S0_j, PV1_{j-1}, S1_j, PV0_j.  While the
 // softmax of Q0 works on S0_j the tensor core runs PV1_{j-1} and S1_j, and
@@ -49,6 +37,9 @@
 // 128 x 128 tiles, where the two Q tiles walk their own tile lists in
 // lockstep.
 //
+// Short units of equal cost (no causal, window or block mask, at most 4096
+// keys) run on the persistent variant in attn_fwd_persist_sm100a.cu instead.
+//
 // Launch order: causal row tiles differ in cost, so the causal grid is 1-D,
 // in bands of (batch, head) pairs whose K/V fit in L2 together, the costliest
 // row tile of every pair of a band first.
@@ -56,36 +47,15 @@
 // Lazy rescaling: the reference maximum of a row only moves when a tile's
 // maximum exceeds it by more than 8 (log2 units), so P <= 2^8; numerator and
 // denominator share the reference, so the result is the same exact softmax.
-#include "attn_internal.h"
-#include "ptx.cuh"
+#include "attn_fwd_common.cuh"
 
 namespace attn {
 namespace {
 
-constexpr int kBlockM = 128;  // rows per Q tile
-constexpr int kBlockN = 128;  // keys per K/V tile
-// warps 0-7 softmax (two warpgroups), warp 8 loader, warp 9 MMA issuer,
-// warps 10-11 idle: the producer warpgroup (warps 8-11) gives registers to
-// the softmax warpgroups (setmaxnreg), so that a softmax thread keeps its whole
-// 128-score row in registers between the two passes
-constexpr int kThreads = 384;
-constexpr uint32_t kLaunchRegs = 168;  // 65536 / 384, rounded down to a multiple of 8
-constexpr uint32_t kProducerRegs = 88;
-// the softmax warpgroups' share of the launch's registers: 256 threads x 208
-// + 128 x 88 = 64512 = 384 x 168; per SM sub-partition 2 x 208 + 88 = 504
-// registers of a thread slot (<= 512)
-constexpr uint32_t kSoftmaxRegs = 208;
-static_assert(256 * kSoftmaxRegs + 128 * kProducerRegs <= kThreads * kLaunchRegs,
-              "register split exceeds the launch allocation");
-static_assert(2 * kSoftmaxRegs + kProducerRegs <= 512, "register split exceeds a sub-partition");
-constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;
+using namespace fwd;
+constexpr int kThreads = 320;
 // a window wider than any key range (i + Lk - Nq - kNoWindow stays negative)
 constexpr int kNoWindow = 1 << 30;
-// one exponential pair in FWD_POLY_EVERY(D) is evaluated on the FMA pipe
-#ifndef FWD_POLY_EVERY
-#define FWD_POLY_EVERY(D) 4
-#endif
 
 template <int D, int KST, int VST>
 struct FwdSmem {
@@ -98,24 +68,9 @@ struct FwdSmem {
     static constexpr uint32_t kAlloc = kTotal + 1024;  // manual 1024-B alignment
 };
 
-// One work unit of the forward: rows [qbase, qbase + 256) of head h of batch
-// b, with the key-tile ranges of its two 128-row Q tiles.
-struct FwdUnit {
-    int b, h, g, Lk, qbase, qoff;
-    int nt0, nt1;      // one past the last candidate key tile of Q0, Q1
-    int j00, j01;      // first key tile of Q0, Q1 (sliding window)
-    int cnt0, cnt1;    // candidate tiles of Q0, Q1
-    int jstart, nt;    // the unit's K/V stream covers tiles [jstart, nt)
-    int last0, last1;  // last key tile used by Q0, Q1 (-1: none)
-    int n0, n1, nsteps;  // block-sparse: tiles of Q0, Q1, lockstep steps
-    int stream;        // K/V tiles loaded for the unit
-    const unsigned char* mrow;
-};
-
 template <int KST, int VST>
 struct FwdBars {
     uint64_t q_full[2];
-    uint64_t q_empty[2];  // the last S of a unit that read Q_a is complete
     uint64_t k_full[KST];
     uint64_t k_empty[KST];
     uint64_t v_full[VST];
@@ -124,94 +79,10 @@ struct FwdBars {
     uint64_t p_full[2];
     uint64_t p_half[2];  // first half of P (keys 0..63) is in tensor memory
     uint64_t o_done[2];
-    uint64_t stage_full[2];  // the last unit's output rows are staged for the TMA store
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
 };
-
-__device__ __forceinline__ void record_error(unsigned* err, unsigned code, int* abort_flag) {
-    atomicCAS(err, 0u, code);
-    *reinterpret_cast<volatile int*>(abort_flag) = 1;
-}
-
-// A bounded wait whose outcome is the same for every lane of the warp, so
-// that the warp-collective tcgen05 loads and stores that follow it are
-// reached by all lanes or by none.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
-                                          volatile int* abort_flag) {
-    const bool ok = ptx::mbar_wait(bar, parity, limit_ns, abort_flag);
-    return __all_sync(0xffffffffu, ok);
-}
-
-// Number of key tiles that rows [q_first, q_first + 128) need.
-__device__ __forceinline__ int tiles_for(int q_first, int Nq, int Lk, int causal) {
-    if (q_first >= Nq) return 0;
-    int nt = (Lk + kBlockN - 1) / kBlockN;
-    if (causal) {
-        const int i_last = min(q_first + kBlockM - 1, Nq - 1);
-        const int lim = i_last + Lk - Nq;  // last key visible to the last row
-        nt = lim < 0 ? 0 : min(nt, lim / kBlockN + 1);
-    }
-    return nt;
-}
-
-// Running maxima of 64 score columns (two 32-column TMEM loads) into eight
-// independent chains of three-input maxima.  kMask: the tile reaches past
-// the row's visible keys [row_first, row_lim] (others are masked).
-template <bool kMask, bool kLow>
-__device__ __forceinline__ void half_max(const uint32_t (&r)[2][32], int key_base, int row_first,
-                                         int row_lim, float (&mx8)[8]) {
-#pragma unroll
-    for (int c = 0; c < 64; c += 16) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int c0 = c + u, c1 = c + 8 + u;
-            float v0 = __uint_as_float(r[c0 >> 5][c0 & 31]);
-            float v1 = __uint_as_float(r[c1 >> 5][c1 & 31]);
-            if (kMask) {
-                if (key_base + c0 > row_lim || (kLow && key_base + c0 < row_first)) v0 = -INFINITY;
-                if (key_base + c1 > row_lim || (kLow && key_base + c1 < row_first)) v1 = -INFINITY;
-            }
-            mx8[u] = ptx::max3(mx8[u], v0, v1);
-        }
-    }
-}
-
-// p = 2^(s * scale_log2 - m) for 64 score columns, accumulated into four
-// pair sums and packed two per 32-bit word (bf16 or fp16).  One pair in
-// kPolyEvery goes to the FMA pipe.
-template <bool kMask, bool kLow, bool BF16, int kPolyEvery>
-__device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_base,
-                                         int row_first, int row_lim,
-                                         uint64_t sl2_2, uint64_t nm_2, uint64_t (&acc2)[4],
-                                         uint32_t (&pk)[32]) {
-#pragma unroll
-    for (int c = 0; c < 64; c += 2) {
-        float v0 = __uint_as_float(r[c >> 5][c & 31]);
-        float v1 = __uint_as_float(r[c >> 5][(c & 31) + 1]);
-        if (kMask) {
-            if (key_base + c > row_lim || (kLow && key_base + c < row_first)) v0 = -INFINITY;
-            if (key_base + c + 1 > row_lim || (kLow && key_base + c + 1 < row_first))
-                v1 = -INFINITY;
-        }
-        const uint64_t t2 = ptx::f2_fma(ptx::f2_pack(v0, v1), sl2_2, nm_2);
-        float p0, p1;
-        if (((c >> 1) % kPolyEvery) == kPolyEvery - 1) {
-            // a share of the pairs on the FMA pipe: the exp2 unit and the tensor
-            // pipe carry equal work at d = 128 (a quarter moves), the exp2 unit
-            // twice the tensor pipe's at d = 64
-            ptx::f2_unpack(ptx::exp2_poly2(t2), p0, p1);
-        } else {
-            float t0, t1;
-            ptx::f2_unpack(t2, t0, t1);
-            p0 = ptx::ex2_approx(t0);
-            p1 = ptx::ex2_approx(t1);
-        }
-        acc2[(c >> 1) & 3] = ptx::f2_add(acc2[(c >> 1) & 3], ptx::f2_pack(p0, p1));
-        pk[c >> 1] = ptx::pack2<BF16>(p0, p1);
-    }
-}
 
 template <int D, bool BF16, int KST, int VST, bool kWindow, bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -238,102 +109,92 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = tid >> 5;
     const int lane = tid & 31;
 
-    // ---- work units: rows [qbase, qbase + 256) of head h of batch b.  CTA
-    // c takes units c, c + gridDim.x, c + 2 gridDim.x, ...; launched with
-    // one CTA per SM it keeps its barriers, tensor memory and pipeline across
-    // units, so that a unit's last tiles and output overlap the next unit's
-    // loads.  Unit order: causal, bands of (b, h) pairs with the costliest
-    // (last) row tile of every pair of a band first; otherwise row tile
-    // fastest, then head, then batch, so that consecutive units share a
-    // head's K/V in L2.
+    // ---- work unit: rows [qbase, qbase + 256) of head h of batch b
+    // causal: a 1-D grid in bands of (b, h) pairs, the costliest (last) row
+    // tile of every pair of a band first, so that blocks launch in
+    // decreasing cost; otherwise (row tiles, Hq, B), consecutive blocks
+    // sharing a head's K/V in L2
     const int n_ctiles = (p.Nq + 2 * kBlockM - 1) / (2 * kBlockM);
-    const int n_units = n_ctiles * p.Hq * p.B;
-
-    // key tile j is used by Q tile a when j in [j0a, nta) and (block-sparse)
-    // the mask entry of the pair is set; without a block mask the K/V stream
-    // of a unit is the union of the two, in increasing j
-    auto use = [&](const FwdUnit& U, int a, int j) -> bool {
-        bool u = a == 0 ? (U.cnt0 > 0 && j >= U.j00 && j < U.nt0)
-                        : (U.cnt1 > 0 && j >= U.j01 && j < U.nt1);
+    int ct, h, b;
+    if (p.band > 0) {
+        int pair, rank;
+        band_unit(blockIdx.x, p.band, p.B * p.Hq, n_ctiles, pair, rank);
+        ct = n_ctiles - 1 - rank;
+        h = pair % p.Hq;
+        b = pair / p.Hq;
+    } else {
+        ct = blockIdx.x;
+        h = blockIdx.y;
+        b = blockIdx.z;
+    }
+    const int g = h / p.G;
+    const int Lk = p.seqlens_k ? p.seqlens_k[b] : p.Nk;
+    const int qbase = ct * 2 * kBlockM;
+    const int nt0 = tiles_for(qbase, p.Nq, Lk, p.causal);
+    const int nt1 = tiles_for(qbase + kBlockM, p.Nq, Lk, p.causal);
+    // sliding window: the first key tile each Q tile needs (tiles before it
+    // are never loaded); stages and phases count from the CTA's first tile
+    // jstart and from each Q tile's own first tile
+    const int qoff = Lk - p.Nq;  // query i's own key position is i + qoff
+    int j00 = 0, j01 = 0;
+    if constexpr (kWindow) {  // kWindow: the instance launched for window_left >= 0
+        j00 = max(0, qbase + qoff - p.window_left) / kBlockN;
+        j01 = max(0, qbase + kBlockM + qoff - p.window_left) / kBlockN;
+    }
+    const int cnt0 = max(0, nt0 - j00), cnt1 = max(0, nt1 - j01);
+    const int jstart = cnt0 > 0 ? j00 : j01;
+    const int nt = max(cnt0 > 0 ? nt0 : 0, cnt1 > 0 ? nt1 : 0);
+    // block-sparse instance: the mask rows of the two Q tiles
+    const unsigned char* mrow = nullptr;
+    if constexpr (kSparse)
+        mrow = p.bmask.m + (long long)b * p.bmask.sb + (long long)h * p.bmask.sh +
+               (long long)(qbase / kBlockM) * p.bmask.srow;
+    // key tile j is used by Q0 when j in [j00, nt0), by Q1 when j in
+    // [j01, nt1), and (block-sparse) when the mask entry of the pair is set;
+    // without a block mask the K/V stream is the union of the two, in
+    // increasing j
+    auto use = [&](int a, int j) -> bool {
+        bool u = a == 0 ? (cnt0 > 0 && j >= j00 && j < nt0) : (cnt1 > 0 && j >= j01 && j < nt1);
         if constexpr (kSparse) {
-            if (u) u = __ldg(U.mrow + (a == 0 ? 0 : p.bmask.srow) + j) != 0;
+            if (u) u = __ldg(mrow + (a == 0 ? 0 : p.bmask.srow) + j) != 0;
         }
         return u;
     };
-    auto make_unit = [&](int u) -> FwdUnit {
-        FwdUnit U;
-        int ct;
-        if (p.band > 0) {
-            int pair, rank;
-            band_unit((unsigned)u, p.band, p.B * p.Hq, n_ctiles, pair, rank);
-            ct = n_ctiles - 1 - rank;
-            U.h = pair % p.Hq;
-            U.b = pair / p.Hq;
-        } else {
-            ct = u % n_ctiles;
-            U.h = (u / n_ctiles) % p.Hq;
-            U.b = u / (n_ctiles * p.Hq);
+    // the last key tile each Q tile uses (-1: none, the tile's rows get O = 0)
+    int last0 = -1, last1 = -1;
+    for (int j = nt0 - 1; cnt0 > 0 && j >= j00; --j)
+        if (use(0, j)) {
+            last0 = j;
+            break;
         }
-        U.g = U.h / p.G;
-        U.Lk = p.seqlens_k ? p.seqlens_k[U.b] : p.Nk;
-        U.qbase = ct * 2 * kBlockM;
-        U.qoff = U.Lk - p.Nq;  // query i's own key position is i + qoff
-        U.nt0 = tiles_for(U.qbase, p.Nq, U.Lk, p.causal);
-        U.nt1 = tiles_for(U.qbase + kBlockM, p.Nq, U.Lk, p.causal);
-        // sliding window: the first key tile each Q tile needs (tiles before
-        // it are never loaded); the unit's stream starts at jstart
-        U.j00 = U.j01 = 0;
-        if constexpr (kWindow) {  // kWindow: the instance launched for window_left >= 0
-            U.j00 = max(0, U.qbase + U.qoff - p.window_left) / kBlockN;
-            U.j01 = max(0, U.qbase + kBlockM + U.qoff - p.window_left) / kBlockN;
+    for (int j = nt1 - 1; cnt1 > 0 && j >= j01; --j)
+        if (use(1, j)) {
+            last1 = j;
+            break;
         }
-        U.cnt0 = max(0, U.nt0 - U.j00);
-        U.cnt1 = max(0, U.nt1 - U.j01);
-        U.jstart = U.cnt0 > 0 ? U.j00 : U.j01;
-        U.nt = max(U.cnt0 > 0 ? U.nt0 : 0, U.cnt1 > 0 ? U.nt1 : 0);
-        U.mrow = nullptr;
-        if constexpr (kSparse)
-            U.mrow = p.bmask.m + (long long)U.b * p.bmask.sb + (long long)U.h * p.bmask.sh +
-                     (long long)(U.qbase / kBlockM) * p.bmask.srow;
-        // the last key tile each Q tile uses (-1: none, the tile's rows get O = 0)
-        U.last0 = U.last1 = -1;
-        for (int j = U.nt0 - 1; U.cnt0 > 0 && j >= U.j00; --j)
-            if (use(U, 0, j)) {
-                U.last0 = j;
-                break;
-            }
-        for (int j = U.nt1 - 1; U.cnt1 > 0 && j >= U.j01; --j)
-            if (use(U, 1, j)) {
-                U.last1 = j;
-                break;
-            }
-        // block-sparse: the number of key tiles of each Q tile (the lockstep
-        // walk takes max(n0, n1) steps) and the unit's K/V stream length
-        U.n0 = U.n1 = 0;
-        if constexpr (kSparse) {
-            for (int j = U.j00; U.cnt0 > 0 && j < U.nt0; ++j) U.n0 += use(U, 0, j) ? 1 : 0;
-            for (int j = U.j01; U.cnt1 > 0 && j < U.nt1; ++j) U.n1 += use(U, 1, j) ? 1 : 0;
-            int c0 = U.j00, c1 = U.j01, si = 0, pos = 0;
-            auto use_u = [&](int a, int j) { return use(U, a, j); };
-            for (int i = 0; i < max(U.n0, U.n1); ++i)
-                sparse_next_step(use_u, U.n0, U.n1, U.nt0, U.nt1, c0, c1, si, pos);
-            U.stream = pos;
-        } else {
-            U.stream = max(0, U.nt - U.jstart);
-        }
-        U.nsteps = max(U.n0, U.n1);
-        return U;
+    // Block-sparse schedule: the two Q tiles walk their own tile lists in
+    // lockstep.  Step i pairs the i-th key tile of Q0 with the i-th of Q1, and
+    // the K/V stream loads Q0's tile, then Q1's when it is a different one, so
+    // that masks that differ between the two cost max(n0, n1) steps, not the
+    // size of the union.
+    int n0 = 0, n1 = 0;  // key tiles of each Q tile
+    if constexpr (kSparse) {
+        for (int j = j00; cnt0 > 0 && j < nt0; ++j) n0 += use(0, j) ? 1 : 0;
+        for (int j = j01; cnt1 > 0 && j < nt1; ++j) n1 += use(1, j) ? 1 : 0;
+    }
+    const int nsteps = max(n0, n1);
+    // c0, c1: next candidate tile of each Q tile; si: step; pos: next position
+    auto next_pair = [&](int& c0, int& c1, int& si, int& pos) -> PairStep {
+        return sparse_next_step(use, n0, n1, nt0, nt1, c0, c1, si, pos);
     };
 
     if (tid == 0) {
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(&bars->q_full[a], 1);
-            ptx::mbar_init(&bars->q_empty[a], 1);
             ptx::mbar_init(&bars->s_full[a], 1);
             ptx::mbar_init(&bars->p_full[a], 128);
             ptx::mbar_init(&bars->p_half[a], 128);
             ptx::mbar_init(&bars->o_done[a], 1);
-            ptx::mbar_init(&bars->stage_full[a], 128);
         }
         for (int s = 0; s < KST; ++s) {
             ptx::mbar_init(&bars->k_full[s], 1);
@@ -362,85 +223,64 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    if (warp >= 8) {
-      // the producer warpgroup hands registers to the softmax warpgroups
-      ptx::setmaxnreg_dec<kProducerRegs>();
-      if (warp == 8) {
+    if (warp == 8) {
         // ================================================= TMA loader
-        if (lane == 0 && !p.inject) {
-            int issued_k = 0, issued_v = 0;  // over all units
-            int nq[2] = {0, 0};              // Q_a loads so far
-            int t = -1;                      // stream position, over all units
-            bool fail = false;
-            for (int u = blockIdx.x; !fail && u < n_units; u += gridDim.x) {
-                const FwdUnit U = make_unit(u);
-                if (U.nt <= 0) continue;
-                for (int a = 0; a < 2; ++a) {
-                    // only a Q tile that takes part is loaded; a buffer is
-                    // reused once the last S of the previous unit that read
-                    // it is complete
-                    if ((a == 0 ? U.last0 : U.last1) < 0) continue;
-                    if (nq[a] > 0 && !ptx::mbar_wait(&bars->q_empty[a], (nq[a] - 1) & 1,
-                                                     p.limit_ns, abort_flag)) {
-                        record_error(p.err, kErrFwdBase + 12, &bars->abort);
-                        fail = true;
-                        break;
-                    }
-                    ptx::mbar_arrive_expect_tx(&bars->q_full[a], kTileBytes);
-                    for (int c = 0; c < kDBlocks; ++c)
-                        ptx::tma_load_4d(smem + L::kQ + a * kTileBytes + c * kBlockBytes, &tm_q,
-                                         &bars->q_full[a], c * 64, U.h, U.qbase + a * kBlockM,
-                                         U.b);
-                    ++nq[a];
-                }
-                if (fail) break;
-                int c0 = U.j00, c1 = U.j01, si = 0, spos = 0;  // block-sparse schedule
-                auto use_u = [&](int a, int j) { return use(U, a, j); };
-                PairStep st{};
-                int e = 1;  // block-sparse: which tile of step st comes next
-                const int n_iter = kSparse ? 2 * U.nsteps : U.nt - U.jstart;
-                for (int it = 0; it < n_iter; ++it) {
-                    int j;
-                    if constexpr (kSparse) {
-                        if (e == 1) {
-                            st = sparse_next_step(use_u, U.n0, U.n1, U.nt0, U.nt1, c0, c1, si,
-                                                  spos);
-                            e = 0;
-                        } else {
-                            e = 1;
-                        }
-                        const bool has = e == 0 ? st.has0 : (st.has1 && !st.shared);
-                        if (!has) continue;
-                        j = e == 0 ? st.x0 : st.x1;
+        if (lane == 0 && nt > 0 && !p.inject) {
+            int issued_k = 0, issued_v = 0;
+            bool issued_q[2] = {false, false};
+            for (int a = 0; a < 2; ++a) {
+                // only a Q tile that takes part: the epilogue of the others
+                // stages O in the Q buffer without waiting for anything
+                if ((a == 0 ? last0 : last1) < 0) continue;
+                ptx::mbar_arrive_expect_tx(&bars->q_full[a], kTileBytes);
+                for (int c = 0; c < kDBlocks; ++c)
+                    ptx::tma_load_4d(smem + L::kQ + a * kTileBytes + c * kBlockBytes, &tm_q,
+                                     &bars->q_full[a], c * 64, h, qbase + a * kBlockM, b);
+                issued_q[a] = true;
+            }
+            int t = -1;  // position of tile j in the stream
+            int c0 = j00, c1 = j01, si = 0, spos = 0;  // block-sparse schedule
+            PairStep st{};
+            int e = 1;   // block-sparse: which tile of step st comes next
+            const int n_iter = kSparse ? 2 * nsteps : nt - jstart;
+            for (int it = 0; it < n_iter; ++it) {
+                int j;
+                if constexpr (kSparse) {
+                    if (e == 1) {
+                        st = next_pair(c0, c1, si, spos);
+                        e = 0;
                     } else {
-                        j = U.jstart + it;
+                        e = 1;
                     }
-                    ++t;
-                    const int sk = t % KST;
-                    if (!ptx::mbar_wait(&bars->k_empty[sk], ((t / KST) & 1) ^ 1, p.limit_ns,
-                                        abort_flag)) {
-                        record_error(p.err, kErrFwdBase + 1, &bars->abort);
-                        fail = true;
-                        break;
-                    }
-                    ptx::mbar_arrive_expect_tx(&bars->k_full[sk], kTileBytes);
-                    for (int c = 0; c < kDBlocks; ++c)
-                        ptx::tma_load_4d(smem + L::kK + sk * kTileBytes + c * kBlockBytes, &tm_k,
-                                         &bars->k_full[sk], c * 64, U.g, j * kBlockN, U.b);
-                    ++issued_k;
-                    const int sv = t % VST;
-                    if (!ptx::mbar_wait(&bars->v_empty[sv], ((t / VST) & 1) ^ 1, p.limit_ns,
-                                        abort_flag)) {
-                        record_error(p.err, kErrFwdBase + 2, &bars->abort);
-                        fail = true;
-                        break;
-                    }
-                    ptx::mbar_arrive_expect_tx(&bars->v_full[sv], kTileBytes);
-                    for (int c = 0; c < kDBlocks; ++c)
-                        ptx::tma_load_4d(smem + L::kV + sv * kTileBytes + c * kBlockBytes, &tm_v,
-                                         &bars->v_full[sv], c * 64, U.g, j * kBlockN, U.b);
-                    ++issued_v;
+                    const bool has = e == 0 ? st.has0 : (st.has1 && !st.shared);
+                    if (!has) continue;
+                    j = e == 0 ? st.x0 : st.x1;
+                } else {
+                    j = jstart + it;
                 }
+                ++t;
+                const int sk = t % KST;
+                if (!ptx::mbar_wait(&bars->k_empty[sk], ((t / KST) & 1) ^ 1, p.limit_ns,
+                                    abort_flag)) {
+                    record_error(p.err, kErrFwdBase + 1, &bars->abort);
+                    break;
+                }
+                ptx::mbar_arrive_expect_tx(&bars->k_full[sk], kTileBytes);
+                for (int c = 0; c < kDBlocks; ++c)
+                    ptx::tma_load_4d(smem + L::kK + sk * kTileBytes + c * kBlockBytes, &tm_k,
+                                     &bars->k_full[sk], c * 64, g, j * kBlockN, b);
+                ++issued_k;
+                const int sv = t % VST;
+                if (!ptx::mbar_wait(&bars->v_empty[sv], ((t / VST) & 1) ^ 1, p.limit_ns,
+                                    abort_flag)) {
+                    record_error(p.err, kErrFwdBase + 2, &bars->abort);
+                    break;
+                }
+                ptx::mbar_arrive_expect_tx(&bars->v_full[sv], kTileBytes);
+                for (int c = 0; c < kDBlocks; ++c)
+                    ptx::tma_load_4d(smem + L::kV + sv * kTileBytes + c * kBlockBytes, &tm_v,
+                                     &bars->v_full[sv], c * 64, g, j * kBlockN, b);
+                ++issued_v;
             }
             // Never leave the CTA with a copy in flight: wait (bounded, and
             // regardless of the abort flag) for the last phase of each
@@ -448,8 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int zero = 0;
             volatile int* no_abort = &zero;
             for (int a = 0; a < 2; ++a)
-                if (nq[a] > 0)
-                    ptx::mbar_wait(&bars->q_full[a], (nq[a] - 1) & 1, p.limit_ns, no_abort);
+                if (issued_q[a]) ptx::mbar_wait(&bars->q_full[a], 0, p.limit_ns, no_abort);
             for (int j = max(0, issued_k - KST); j < issued_k; ++j)
                 ptx::mbar_wait(&bars->k_full[j % KST], (j / KST) & 1, p.limit_ns, no_abort);
             for (int j = max(0, issued_v - VST); j < issued_v; ++j)
@@ -457,11 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 9) {
         // ================================================= MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && nt > 0) {
             bool ok = true;
-            int t_base = 0;                       // stream position of the unit's first tile
-            int nq[2] = {0, 0};                   // Q_a loads consumed
-            int npv[2] = {0, 0};                  // P_a V products issued
+            bool q_ready[2] = {false, false};
             const uint32_t col_s[2] = {0u, 128u};
             const uint32_t col_o[2] = {256u, 256u + D};
             const uint32_t q_addr[2] = {sbase + L::kQ, sbase + L::kQ + kTileBytes};
@@ -472,141 +309,126 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 return ok;
             };
-            for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-                const FwdUnit U = make_unit(u);
-                if (U.nt <= 0) continue;
-                bool q_ready[2] = {false, false};
-                // S_a of the tile at stream position t; last: the unit's last
-                // S_a, after which its Q buffer may be reloaded
-                auto issue_s = [&](int a, int t, bool last) {
-                    if (!q_ready[a]) {
-                        if (!wait_or_fail(&bars->q_full[a], nq[a] & 1, 3)) return;
-                        ++nq[a];
-                        ptx::tc_fence_after();
-                        q_ready[a] = true;
-                    }
-                    const uint32_t k_addr = sbase + L::kK + (t % KST) * kTileBytes;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
-                        ptx::umma_ss(tmem + col_s[a],
-                                     ptx::sdesc_sw128(q_addr[a] + off, 16, 1024),
-                                     ptx::sdesc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0);
-                    }
-                    ptx::umma_commit(&bars->s_full[a]);
-                    if (last) ptx::umma_commit(&bars->q_empty[a]);
-                };
-                // P_a·V of the tile at stream position t, the Q tile's ia-th
-                // tile of the unit; last: the Q tile's O is complete after it
-                auto issue_pv = [&](int a, int t, int ia, bool last) {
-                    if (!wait_or_fail(&bars->p_half[a], npv[a] & 1, 5)) return;
-                    if (!wait_or_fail(&bars->v_full[t % VST], (t / VST) & 1, 6)) return;
+            // S_a of the tile at stream position t
+            auto issue_s = [&](int a, int t) {
+                if (!q_ready[a]) {
+                    if (!wait_or_fail(&bars->q_full[a], 0, 3)) return;
                     ptx::tc_fence_after();
-                    const uint32_t v_addr = sbase + L::kV + (t % VST) * kTileBytes;
+                    q_ready[a] = true;
+                }
+                const uint32_t k_addr = sbase + L::kK + (t % KST) * kTileBytes;
 #pragma unroll
-                    for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                        if (kk == kBlockN / 32) {
-                            if (!wait_or_fail(&bars->p_full[a], npv[a] & 1, 5)) return;
-                            ptx::tc_fence_after();
-                        }
-                        ptx::umma_ts(tmem + col_o[a], tmem + col_s[a] + kk * 8,
-                                     ptx::sdesc_sw128(v_addr + kk * 16 * 128, kBlockBytes, 1024),
-                                     kIdescO, (ia > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
+                    ptx::umma_ss(tmem + col_s[a], ptx::sdesc_sw128(q_addr[a] + off, 16, 1024),
+                                 ptx::sdesc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0);
+                }
+                ptx::umma_commit(&bars->s_full[a]);
+            };
+            // P_a·V of the tile at stream position t, the Q tile's ia-th tile;
+            // last: the Q tile's O is complete after it
+            auto issue_pv = [&](int a, int t, int ia, bool last) {
+                if (!wait_or_fail(&bars->p_half[a], ia & 1, 5)) return;
+                if (!wait_or_fail(&bars->v_full[t % VST], (t / VST) & 1, 6)) return;
+                ptx::tc_fence_after();
+                const uint32_t v_addr = sbase + L::kV + (t % VST) * kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                    if (kk == kBlockN / 32) {
+                        if (!wait_or_fail(&bars->p_full[a], ia & 1, 5)) return;
+                        ptx::tc_fence_after();
                     }
-                    ++npv[a];
-                    if (last) ptx::umma_commit(&bars->o_done[a]);
-                };
-                if constexpr (kSparse) {
-                    // lockstep steps: S0_i, PV1_{i-1}, S1_i, PV0_i, a stage is
-                    // released after its last user's product
-                    auto use_u = [&](int a, int j) { return use(U, a, j); };
-                    int c0 = U.j00, c1 = U.j01, si = 0, spos = 0;
-                    PairStep prev{};
-                    bool have_prev = false;
-                    for (int i = 0; ok && i <= U.nsteps; ++i) {
-                        PairStep st{};
-                        if (i < U.nsteps) {
-                            st = sparse_next_step(use_u, U.n0, U.n1, U.nt0, U.nt1, c0, c1, si,
-                                                  spos);
-                            if (st.has0) {
-                                const int t0 = t_base + st.pos0;
-                                if (!wait_or_fail(&bars->k_full[t0 % KST], (t0 / KST) & 1, 4))
+                    ptx::umma_ts(tmem + col_o[a], tmem + col_s[a] + kk * 8,
+                                 ptx::sdesc_sw128(v_addr + kk * 16 * 128, kBlockBytes, 1024),
+                                 kIdescO, (ia > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (last) ptx::umma_commit(&bars->o_done[a]);
+            };
+            if constexpr (kSparse) {
+                // lockstep steps: S0_i, PV1_{i-1}, S1_i, PV0_i, a stage is
+                // released after its last user's product
+                int c0 = j00, c1 = j01, si = 0, spos = 0;
+                PairStep prev{};
+                bool have_prev = false;
+                for (int i = 0; ok && i <= nsteps; ++i) {
+                    PairStep st{};
+                    if (i < nsteps) {
+                        st = next_pair(c0, c1, si, spos);
+                        if (st.has0) {
+                            if (!wait_or_fail(&bars->k_full[st.pos0 % KST], (st.pos0 / KST) & 1,
+                                              4))
+                                break;
+                            ptx::tc_fence_after();
+                            issue_s(0, st.pos0);
+                            if (!ok) break;
+                            if (!st.shared) ptx::umma_commit(&bars->k_empty[st.pos0 % KST]);
+                        }
+                    }
+                    if (have_prev && prev.has1) {
+                        issue_pv(1, prev.pos1, i - 1, i - 1 == n1 - 1);
+                        if (!ok) break;
+                        ptx::umma_commit(&bars->v_empty[prev.pos1 % VST]);
+                    }
+                    if (i < nsteps) {
+                        if (st.has1) {
+                            if (!st.shared) {
+                                if (!wait_or_fail(&bars->k_full[st.pos1 % KST],
+                                                  (st.pos1 / KST) & 1, 4))
                                     break;
                                 ptx::tc_fence_after();
-                                issue_s(0, t0, i == U.n0 - 1);
-                                if (!ok) break;
-                                if (!st.shared) ptx::umma_commit(&bars->k_empty[t0 % KST]);
                             }
-                        }
-                        if (have_prev && prev.has1) {
-                            const int t1 = t_base + prev.pos1;
-                            issue_pv(1, t1, i - 1, i - 1 == U.n1 - 1);
+                            issue_s(1, st.pos1);
                             if (!ok) break;
-                            ptx::umma_commit(&bars->v_empty[t1 % VST]);
+                            ptx::umma_commit(&bars->k_empty[st.pos1 % KST]);
                         }
-                        if (i < U.nsteps) {
-                            if (st.has1) {
-                                const int t1 = t_base + st.pos1;
-                                if (!st.shared) {
-                                    if (!wait_or_fail(&bars->k_full[t1 % KST], (t1 / KST) & 1, 4))
-                                        break;
-                                    ptx::tc_fence_after();
-                                }
-                                issue_s(1, t1, i == U.n1 - 1);
-                                if (!ok) break;
-                                ptx::umma_commit(&bars->k_empty[t1 % KST]);
-                            }
-                            if (st.has0) {
-                                const int t0 = t_base + st.pos0;
-                                issue_pv(0, t0, i, i == U.n0 - 1);
-                                if (!ok) break;
-                                if (!st.shared) ptx::umma_commit(&bars->v_empty[t0 % VST]);
-                            }
+                        if (st.has0) {
+                            issue_pv(0, st.pos0, i, i == n0 - 1);
+                            if (!ok) break;
+                            if (!st.shared) ptx::umma_commit(&bars->v_empty[st.pos0 % VST]);
                         }
-                        prev = st;
-                        have_prev = i < U.nsteps;
                     }
-                } else {
-                    // a stage is released after its last user's product
-                    int t = t_base, i0 = 0, i1 = 0;           // stream position, per-tile counts
-                    int prev_t = 0, prev_i1 = 0, prev_j = -1;  // the previous tile of the stream
-                    bool prev_u1 = false;
-                    for (int j = U.jstart; ok && j <= U.nt; ++j) {
-                        bool u0 = false, u1 = false;
-                        if (j < U.nt) {
-                            u0 = use(U, 0, j);
-                            u1 = use(U, 1, j);
-                            if (!wait_or_fail(&bars->k_full[t % KST], (t / KST) & 1, 4)) break;
-                            ptx::tc_fence_after();
-                            if (u0) issue_s(0, t, j == U.last0);
-                            if (!ok) break;
-                        }
-                        if (prev_u1) {
-                            issue_pv(1, prev_t, prev_i1, prev_j == U.last1);
-                            if (!ok) break;
-                            ptx::umma_commit(&bars->v_empty[prev_t % VST]);
-                        }
-                        if (j < U.nt) {
-                            if (u1) issue_s(1, t, j == U.last1);
-                            if (!ok) break;
-                            ptx::umma_commit(&bars->k_empty[t % KST]);
-                            if (u0) {
-                                issue_pv(0, t, i0, j == U.last0);
-                                if (!ok) break;
-                            }
-                            if (!u1) ptx::umma_commit(&bars->v_empty[t % VST]);
-                        }
-                        prev_u1 = u1;
-                        prev_t = t;
-                        prev_i1 = i1;
-                        prev_j = j;
-                        i0 += u0 ? 1 : 0;
-                        i1 += u1 ? 1 : 0;
-                        ++t;
-                    }
+                    prev = st;
+                    have_prev = i < nsteps;
                 }
-                t_base += U.stream;
+            } else {
+            // a stage is released after its last user's product
+            int t = 0, i0 = 0, i1 = 0;                      // stream position, per-tile counts
+            int prev_t = 0, prev_i1 = 0, prev_j = -1;       // the previous tile of the stream
+            bool prev_u1 = false;
+            for (int j = jstart; ok && j <= nt; ++j) {
+                bool u0 = false, u1 = false;
+                if (j < nt) {
+                    u0 = use(0, j);
+                    u1 = use(1, j);
+                    if (!wait_or_fail(&bars->k_full[t % KST], (t / KST) & 1, 4)) break;
+                    ptx::tc_fence_after();
+                    if (u0) issue_s(0, t);
+                    if (!ok) break;
+                }
+                if (prev_u1) {
+                    issue_pv(1, prev_t, prev_i1, prev_j == last1);
+                    if (!ok) break;
+                    ptx::umma_commit(&bars->v_empty[prev_t % VST]);
+                }
+                if (j < nt) {
+                    if (u1) issue_s(1, t);
+                    if (!ok) break;
+                    ptx::umma_commit(&bars->k_empty[t % KST]);
+                    if (u0) {
+                        issue_pv(0, t, i0, j == last0);
+                        if (!ok) break;
+                    }
+                    if (!u1) ptx::umma_commit(&bars->v_empty[t % VST]);
+                }
+                prev_u1 = u1;
+                prev_t = t;
+                prev_i1 = i1;
+                prev_j = j;
+                i0 += u0 ? 1 : 0;
+                i1 += u1 ? 1 : 0;
+                ++t;
             }
+            }  // dense / window stream
             if (!ok) {
                 // make sure no MMA is still running before TMEM is freed
                 int zero = 0;
@@ -615,251 +437,220 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::mbar_wait(&bars->drain, 0, p.limit_ns, no_abort);
             }
         }
-      }
     } else {
-        ptx::setmaxnreg_inc<kSoftmaxRegs>();
         // ================================================= softmax warpgroups
         const int a = warp >> 2;  // which Q tile
+        const int nta = a == 0 ? (cnt0 > 0 ? nt0 : 0) : (cnt1 > 0 ? nt1 : 0);
+        const int ja = a == 0 ? j00 : j01;  // its first key tile
         const uint32_t quarter = (uint32_t)(warp & 3);
         const uint32_t row = quarter * 32u + (uint32_t)lane;
         const uint32_t lane_addr = (quarter * 32u) << 16;
+        const int qa = qbase + a * kBlockM;
+        const int i = qa + (int)row;
+        int row_lim = Lk - 1;  // last visible key of this row
+        if (p.causal) row_lim = min(row_lim, i + Lk - p.Nq);
+        // first visible key of this row (the sliding window's lower edge)
+        const int row_first = kWindow ? i + qoff - p.window_left : 0;
         const float sl2 = p.scale_log2;
-        const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
+        float m_ref = -INFINITY;  // running reference max, scale*log2 units
+        float l_sum = 0.f;        // running sum of exp2(s*sl2 - m_ref)
+        bool ok = true;
         const uint32_t t_s = tmem + lane_addr + (a == 0 ? 0u : 128u);
         const uint32_t t_o = tmem + lane_addr + (a == 0 ? 256u : 256u + D);
-        bool ok = true;
-        int t_base = 0;      // stream position of the unit's first tile
-        int tiles_done = 0;  // S_a products consumed (parity of s_full)
-        int units_done = 0;  // units in which this Q tile had work (parity of o_done)
-        for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-            const FwdUnit U = make_unit(u);
-            const int nta = a == 0 ? (U.cnt0 > 0 ? U.nt0 : 0) : (U.cnt1 > 0 ? U.nt1 : 0);
-            const int ja = a == 0 ? U.j00 : U.j01;  // its first key tile
-            const int qa = U.qbase + a * kBlockM;
-            const int i = qa + (int)row;
-            int row_lim = U.Lk - 1;  // last visible key of this row
-            if (p.causal) row_lim = min(row_lim, i + U.Lk - p.Nq);
-            // first visible key of this row (the sliding window's lower edge)
-            const int row_first = kWindow ? i + U.qoff - p.window_left : 0;
-            float m_ref = -INFINITY;  // running reference max, scale*log2 units
-            float l_sum = 0.f;        // running sum of exp2(s*sl2 - m_ref)
-            auto use_u = [&](int aa, int j) { return use(U, aa, j); };
 
-            int ia = 0;  // key tiles of this Q tile done so far in the unit
-            int c0 = U.j00, c1 = U.j01, si = 0, spos = 0;  // block-sparse schedule
-            const int n_iter = U.nt <= 0 ? 0 : kSparse ? (a == 0 ? U.n0 : U.n1) : max(0, nta - ja);
-            for (int it = 0; it < n_iter; ++it) {
-                int j, t;         // key tile, its stream position
-                bool first_user;  // this Q tile's P·V is the first to read V_j
-                if constexpr (kSparse) {
-                    const PairStep st = sparse_next_step(use_u, U.n0, U.n1, U.nt0, U.nt1, c0, c1,
-                                                         si, spos);
-                    j = a == 0 ? st.x0 : st.x1;
-                    t = t_base + (a == 0 ? st.pos0 : st.pos1);
-                    first_user = a == 0 || !st.shared;
-                } else {
-                    j = ja + it;
-                    t = t_base + (j - U.jstart);
-                    first_user = a == 0 || !use(U, 0, j);
-                }
-                if (!warp_wait(&bars->s_full[a], tiles_done & 1, p.limit_ns, abort_flag)) {
-                    record_error(p.err, kErrFwdBase + 7, &bars->abort);
-                    ok = false;
-                    break;
-                }
-                ++tiles_done;
-                ptx::tc_fence_after();
-                const int key0 = j * kBlockN;
-                const bool masked = key0 + kBlockN - 1 > row_lim || (kWindow && key0 < row_first);
-                // pass 1: row maximum, two halves of 64 columns, eight independent
-                // chains of three-input maxima
-                float mx8[8];
+        int ia = 0;  // key tiles of this Q tile done so far
+        int c0 = j00, c1 = j01, si = 0, spos = 0;  // block-sparse schedule
+        const int n_iter = kSparse ? (a == 0 ? n0 : n1) : max(0, nta - ja);
+        for (int it = 0; it < n_iter; ++it) {
+            int j, t;         // key tile, its stream position
+            bool first_user;  // this Q tile's P·V is the first to read V_j
+            if constexpr (kSparse) {
+                const PairStep st = next_pair(c0, c1, si, spos);
+                j = a == 0 ? st.x0 : st.x1;
+                t = a == 0 ? st.pos0 : st.pos1;
+                first_user = a == 0 || !st.shared;
+            } else {
+                j = ja + it;
+                t = j - jstart;
+                first_user = a == 0 || !use(0, j);
+            }
+            if (!warp_wait(&bars->s_full[a], ia & 1, p.limit_ns, abort_flag)) {
+                record_error(p.err, kErrFwdBase + 7, &bars->abort);
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            const int key0 = j * kBlockN;
+            const bool masked = key0 + kBlockN - 1 > row_lim || (kWindow && key0 < row_first);
+            // pass 1: row maximum, two halves of 64 columns, eight independent
+            // chains of three-input maxima
+            float mx8[8];
 #pragma unroll
-                for (int uu = 0; uu < 8; ++uu) mx8[uu] = -INFINITY;
-                // the whole row stays in registers for pass 2 (one load of S per tile)
-                uint32_t rs[2][2][32];
-                {
-                    auto& r = rs;
-#pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        ptx::tmem_ld32(t_s + hf * 64, r[hf][0]);
-                        ptx::tmem_ld32(t_s + hf * 64 + 32, r[hf][1]);
-                    }
-#pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        ptx::tmem_wait_ld_dep(r[hf][0]);
-                        ptx::tmem_wait_ld_dep(r[hf][1]);
-                        if (masked)
-                            half_max<true, kWindow>(r[hf], key0 + hf * 64, row_first, row_lim, mx8);
-                        else
-                            half_max<false, kWindow>(r[hf], key0 + hf * 64, row_first, row_lim,
-                                                     mx8);
-                    }
-                }
-                const float mx = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]),
-                                           ptx::max3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-                const float m_tile = mx * sl2;  // -inf stays -inf (sl2 > 0)
-                float alpha = 1.f;
-                bool rescale = false;
-                if (m_tile > m_ref + kRescaleThreshold) {
-                    alpha = ptx::ex2_approx(m_ref - m_tile);  // 0 when m_ref = -inf
-                    rescale = (ia > 0) && (m_ref != -INFINITY);
-                    m_ref = m_tile;
-                }
-                const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-                const uint64_t nm_2 = ptx::f2_pack(-m_use, -m_use);
-                if (__any_sync(0xffffffffu, rescale)) {
-                    // the previous P_a V has completed (it precedes S_a_j); done
-                    // before the exponentials, since the first half of P_a V may
-                    // start while the second half of P_a is still being formed
-                    const float sc = rescale ? alpha : 1.f;
-#pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t r[32];
-                        ptx::tmem_ld32(t_o + c * 32, r);
-                        ptx::tmem_wait_ld_dep(r);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            r[e] = __float_as_uint(__uint_as_float(r[e]) * sc);
-                        ptx::tmem_st32(t_o + c * 32, r);
-                    }
-                    ptx::tmem_wait_st();
-                }
-                ptx::tmem_wait_st();
-                // the Q tile whose P·V reads V_j first zeroes its rows behind the
-                // real length (Q0 if it uses the tile, else Q1)
-                const bool zero_v = p.seqlens_k != nullptr && key0 + kBlockN > U.Lk && first_user;
-                if (zero_v) {
-                    // keys behind the real length: zero their V rows so that a
-                    // non-finite value stored there cannot reach O through 0 * NaN
-                    const int sv = t % VST;
-                    if (!warp_wait(&bars->v_full[sv], (t / VST) & 1, p.limit_ns, abort_flag)) {
-                        record_error(p.err, kErrFwdBase + 8, &bars->abort);
-                        ok = false;
-                        break;
-                    }
-                    if (key0 + (int)row >= U.Lk) {
-                        uint8_t* vt = smem + L::kV + sv * kTileBytes;
-#pragma unroll
-                        for (int c = 0; c < kDBlocks; ++c)
-#pragma unroll
-                            for (int ch = 0; ch < 8; ++ch)
-                                *reinterpret_cast<uint4*>(vt + c * kBlockBytes + row * 128 + ch * 16) =
-                                    make_uint4(0, 0, 0, 0);
-                    }
-                    ptx::fence_proxy_async_smem();
-                }
-                uint64_t acc2[4] = {0, 0, 0, 0};  // four pair accumulators of the row sum
-                // pass 2: exponentials per half; P of half hf goes to columns
-                // [32 hf, 32 hf + 32) of S_a, which pass 2 has already consumed,
-                // and is published on its own barrier (p_half, then p_full) so
-                // that the MMA of keys 0..63 overlaps the exponentials of 64..127
+            for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
+            // d = 128 keeps the first half of the row in registers for pass 2
+            // (one tensor-memory round trip less per tile; at d = 64 the
+            // extra registers cost more than the load)
+            uint32_t rs[2][2][32];
+            {
+                auto& r = rs;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    auto& r = rs[hf];
-                    uint32_t pk[32];
-                    if (masked)
-                        half_exp<true, kWindow, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
-                                                                  row_lim, sl2_2, nm_2, acc2, pk);
-                    else
-                        half_exp<false, kWindow, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
-                                                                   row_lim, sl2_2, nm_2, acc2, pk);
-                    ptx::tmem_st32(t_s + hf * 32, pk);
-                    ptx::tmem_wait_st();
-                    ptx::tc_fence_before();
-                    ptx::mbar_arrive(hf == 0 ? &bars->p_half[a] : &bars->p_full[a]);
+                    ptx::tmem_ld32(t_s + hf * 64, r[hf][0]);
+                    ptx::tmem_ld32(t_s + hf * 64 + 32, r[hf][1]);
                 }
-                float s0, s1, s2, s3, s4, s5, s6, s7;
-                ptx::f2_unpack(acc2[0], s0, s1);
-                ptx::f2_unpack(acc2[1], s2, s3);
-                ptx::f2_unpack(acc2[2], s4, s5);
-                ptx::f2_unpack(acc2[3], s6, s7);
-                const float rowsum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
-                l_sum = l_sum * alpha + rowsum;
-                ++ia;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    ptx::tmem_wait_ld_dep(r[hf][0]);
+                    ptx::tmem_wait_ld_dep(r[hf][1]);
+                    if (masked)
+                        half_max<true, kWindow>(r[hf], key0 + hf * 64, row_first, row_lim, mx8);
+                    else
+                        half_max<false, kWindow>(r[hf], key0 + hf * 64, row_first, row_lim, mx8);
+                }
             }
-            if (!ok) break;
-
-            // ---- epilogue of the unit: O / l -> bf16/fp16 and LSE.  The CTA's
-            // last unit stages O in its Q buffer (free: no Q follows) and
-            // writes it with TMA stores; earlier units store each thread's
-            // row straight from registers, since their Q buffer already holds
-            // the next unit's Q.
-            const bool last_unit = u + (int)gridDim.x >= n_units;
-            if (ia > 0) {
-                if (!warp_wait(&bars->o_done[a], units_done & 1, p.limit_ns, abort_flag)) {
-                    record_error(p.err, kErrFwdBase + 9, &bars->abort);
+            const float mx = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]),
+                                       ptx::max3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+            const float m_tile = mx * sl2;  // -inf stays -inf (sl2 > 0)
+            float alpha = 1.f;
+            bool rescale = false;
+            if (m_tile > m_ref + kRescaleThreshold) {
+                alpha = ptx::ex2_approx(m_ref - m_tile);  // 0 when m_ref = -inf
+                rescale = (ia > 0) && (m_ref != -INFINITY);
+                m_ref = m_tile;
+            }
+            const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+            const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
+            const uint64_t nm_2 = ptx::f2_pack(-m_use, -m_use);
+            if (__any_sync(0xffffffffu, rescale)) {
+                // the previous P_a V has completed (it precedes S_a_j); done
+                // before the exponentials, since the first half of P_a V may
+                // start while the second half of P_a is still being formed
+                const float s = rescale ? alpha : 1.f;
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    ptx::tmem_ld32(t_o + c * 32, r);
+                    ptx::tmem_wait_ld_dep(r);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * s);
+                    ptx::tmem_st32(t_o + c * 32, r);
+                }
+                ptx::tmem_wait_st();
+            }
+            ptx::tmem_wait_st();
+            // the Q tile whose P·V reads V_j first zeroes its rows behind the
+            // real length (Q0 if it uses the tile, else Q1)
+            const bool zero_v = p.seqlens_k != nullptr && key0 + kBlockN > Lk && first_user;
+            if (zero_v) {
+                // keys behind the real length: zero their V rows so that a
+                // non-finite value stored there cannot reach O through 0 * NaN
+                const int sv = t % VST;
+                if (!warp_wait(&bars->v_full[sv], (t / VST) & 1, p.limit_ns, abort_flag)) {
+                    record_error(p.err, kErrFwdBase + 8, &bars->abort);
                     ok = false;
                     break;
                 }
-                ++units_done;
-                ptx::tc_fence_after();
-            }
-            const bool have = ia > 0 && l_sum > 0.f;
-            const float inv_l = have ? 1.f / l_sum : 0.f;
-            if (qa < p.Nq) {
-                uint8_t* orow = static_cast<uint8_t*>(p.o) +
-                                (((size_t)U.b * p.Nq + (size_t)i) * p.Hq + U.h) * (size_t)(D * 2);
-                uint8_t* stage = smem + L::kQ + a * kTileBytes;
+                if (key0 + (int)row >= Lk) {
+                    uint8_t* vt = smem + L::kV + sv * kTileBytes;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t r[32];
-                    if (ia > 0) {
-                        ptx::tmem_ld32(t_o + c * 32, r);
-                        ptx::tmem_wait_ld_dep(r);
-                    } else {
+                    for (int c = 0; c < kDBlocks; ++c)
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) r[e] = 0u;
-                    }
-                    uint32_t o2[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        o2[e] = ptx::pack2<BF16>(__uint_as_float(r[2 * e]) * inv_l,
-                                                 __uint_as_float(r[2 * e + 1]) * inv_l);
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const uint4 w = make_uint4(o2[q4 * 4], o2[q4 * 4 + 1], o2[q4 * 4 + 2],
-                                                   o2[q4 * 4 + 3]);
-                        if (last_unit) {
-                            // 32 columns = 4 chunks of 16 bytes in block c/2, chunks
-                            // (c%2)*4 .. +3 of the 128-byte swizzled row
-                            const uint32_t ch = (uint32_t)((c & 1) * 4 + q4);
-                            *reinterpret_cast<uint4*>(stage + (c >> 1) * kBlockBytes + row * 128u +
-                                                      ((ch ^ (row & 7u)) << 4)) = w;
-                        } else if (i < p.Nq) {
-                            *reinterpret_cast<uint4*>(orow + c * 64 + q4 * 16) = w;
-                        }
-                    }
+                        for (int ch = 0; ch < 8; ++ch)
+                            *reinterpret_cast<uint4*>(vt + c * kBlockBytes + row * 128 + ch * 16) =
+                                make_uint4(0, 0, 0, 0);
                 }
-                if (last_unit) {
-                    // the staged tile goes out by TMA once all 128 rows are in;
-                    // a bounded wait, so that a warp that left on an error
-                    // cannot hold the others
-                    ptx::fence_proxy_async_smem();
-                    ptx::mbar_arrive(&bars->stage_full[a]);
-                    if (quarter == 0 && lane == 0) {
-                        if (ptx::mbar_wait(&bars->stage_full[a], 0, p.limit_ns, abort_flag)) {
-                            for (int c = 0; c < kDBlocks; ++c)
-                                ptx::tma_store_4d(&tm_o, stage + c * kBlockBytes, c * 64, U.h,
-                                                  qa, U.b);
-                            ptx::bulk_commit_group();
-                            ptx::bulk_wait_group_read0();
-                        } else {
-                            record_error(p.err, kErrFwdBase + 13, &bars->abort);
-                        }
-                    }
+                ptx::fence_proxy_async_smem();
+            }
+            uint64_t acc2[4] = {0, 0, 0, 0};  // four pair accumulators of the row sum
+            // pass 2: exponentials per half; P of half hf goes to columns
+            // [32 hf, 32 hf + 32) of S_a, which pass 2 has already consumed,
+            // and is published on its own barrier (p_half, then p_full) so
+            // that the MMA of keys 0..63 overlaps the exponentials of 64..127
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                constexpr int kKept = D == 128 ? 1 : 0;  // halves kept from pass 1
+                uint32_t rl[2][32];
+                if (hf >= kKept) {
+                    ptx::tmem_ld32(t_s + hf * 64, rl[0]);
+                    ptx::tmem_ld32(t_s + hf * 64 + 32, rl[1]);
+                    ptx::tmem_wait_ld_dep(rl[0]);
+                    ptx::tmem_wait_ld_dep(rl[1]);
+                }
+                auto& r = hf >= kKept ? rl : rs[hf];
+                uint32_t pk[32];
+                if (masked)
+                    half_exp<true, kWindow, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
+                                                              row_lim, sl2_2,
+                                                     nm_2, acc2, pk);
+                else
+                    half_exp<false, kWindow, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
+                                                               row_lim, sl2_2,
+                                                      nm_2, acc2, pk);
+                ptx::tmem_st32(t_s + hf * 32, pk);
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(hf == 0 ? &bars->p_half[a] : &bars->p_full[a]);
+            }
+            float s0, s1, s2, s3, s4, s5, s6, s7;
+            ptx::f2_unpack(acc2[0], s0, s1);
+            ptx::f2_unpack(acc2[1], s2, s3);
+            ptx::f2_unpack(acc2[2], s4, s5);
+            ptx::f2_unpack(acc2[3], s6, s7);
+            const float rowsum = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+            l_sum = l_sum * alpha + rowsum;
+            ++ia;
+        }
+
+        // ---- epilogue: O / l -> bf16/fp16 -> swizzled staging (the Q_a
+        // buffer, free once the last S_a MMA is done) -> TMA store
+        if (ok && ia > 0) {
+            if (!warp_wait(&bars->o_done[a], 0, p.limit_ns, abort_flag)) {
+                record_error(p.err, kErrFwdBase + 9, &bars->abort);
+                ok = false;
+            }
+            ptx::tc_fence_after();
+        }
+        const bool have = ok && ia > 0 && l_sum > 0.f;
+        const float inv_l = have ? 1.f / l_sum : 0.f;
+        uint8_t* stage = smem + L::kQ + a * kTileBytes;
+        if (qa < p.Nq) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                if (ok && ia > 0) {
+                    ptx::tmem_ld32(t_o + c * 32, r);
+                    ptx::tmem_wait_ld_dep(r);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) r[e] = 0u;
+                }
+                uint32_t o2[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    o2[e] = ptx::pack2<BF16>(__uint_as_float(r[2 * e]) * inv_l,
+                                             __uint_as_float(r[2 * e + 1]) * inv_l);
+                // 32 columns = 4 chunks of 16 bytes in block c/2, chunks (c%2)*4..+3
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const uint32_t ch = (uint32_t)((c & 1) * 4 + q4);
+                    *reinterpret_cast<uint4*>(stage + (c >> 1) * kBlockBytes +
+                                              sw128_offset(row, ch)) =
+                        make_uint4(o2[q4 * 4], o2[q4 * 4 + 1], o2[q4 * 4 + 2], o2[q4 * 4 + 3]);
                 }
             }
-            if (i < p.Nq) {
-                const float lse = have ? (m_ref + ptx::lg2_approx(l_sum)) * 0.69314718055994531f
-                                       : -INFINITY;
-                p.lse[((size_t)U.b * p.Hq + U.h) * p.Nq + i] = lse;
-            }
-            // the tensor-memory reads of O complete before this warpgroup
-            // publishes the next unit's first P, after which the first P·V
-            // of that unit overwrites O
-            ptx::tc_fence_before();
-            t_base += U.stream;
+            ptx::fence_proxy_async_smem();
+        }
+        ptx::named_barrier_sync(1 + a, 128);
+        if (quarter == 0 && lane == 0 && qa < p.Nq) {
+            for (int c = 0; c < kDBlocks; ++c)
+                ptx::tma_store_4d(&tm_o, stage + c * kBlockBytes, c * 64, h, qa, b);
+            ptx::bulk_commit_group();
+            ptx::bulk_wait_group_read0();
+        }
+        if (i < p.Nq) {
+            const float lse = have ? (m_ref + ptx::lg2_approx(l_sum)) * 0.69314718055994531f
+                                   : -INFINITY;
+            p.lse[((size_t)b * p.Hq + h) * p.Nq + i] = lse;
         }
     }
 
@@ -880,7 +671,10 @@ cudaError_t launch_fwd_w(const FwdMaps& maps, const FwdParams& p, cudaStream_t s
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::kAlloc);
     if (e != cudaSuccess) return e;
-    kern<<<dim3((unsigned)p.n_ctas), kThreads, L::kAlloc, stream>>>(maps.q, maps.k, maps.v, maps.o, p);
+    const unsigned n_ctiles = (unsigned)((p.Nq + 2 * kBlockM - 1) / (2 * kBlockM));
+    const dim3 grid = p.band > 0 ? dim3((unsigned)p.B * p.Hq * n_ctiles, 1, 1)
+                                 : dim3(n_ctiles, p.Hq, p.B);
+    kern<<<grid, kThreads, L::kAlloc, stream>>>(maps.q, maps.k, maps.v, maps.o, p);
     return cudaGetLastError();
 }
 

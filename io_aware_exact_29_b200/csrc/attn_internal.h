@@ -81,7 +81,7 @@ __host__ __device__ __forceinline__ PairStep sparse_next_step(const Use& use, in
 
 struct FwdParams {
     int B, Hq, Hkv, Nq, Nk;
-    int n_ctas;       // CTAs launched; each takes every n_ctas-th work unit
+    int n_ctas;       // persistent forward: CTAs launched, each taking every n_ctas-th unit
     int G;            // Hq / Hkv
     int n_qtiles;     // ceil(Nq / 128)
     int causal;
@@ -90,7 +90,7 @@ struct FwdParams {
     int window_left;       // -1, or keys before i + (Lk - Nq) - window_left are masked
     BlockMask bmask;       // block-sparse mask, or m == nullptr
     int band;              // >0: 1-D grid, bands of `band` (b, h) pairs, costliest tiles first
-    void* o;               // [B, Nq, Hq, d]
+    void* o;               // [B, Nq, Hq, d] (persistent forward: rows stored from registers)
     float* lse;            // [B, Hq, Nq]
     unsigned long long limit_ns;
     int inject;       // self-test: the loader skips everything
@@ -101,9 +101,16 @@ struct FwdMaps {
     CUtensorMap q, k, v, o;
 };
 
-// Launch the forward kernel for head dim d (64/128) and element type.
+// Launch the forward kernel for head dim d (64/128) and element type: one
+// CTA per work unit of 256 query rows, every mask (attn_fwd_sm100a.cu).
 cudaError_t launch_fwd(const FwdMaps& maps, const FwdParams& p, int d, bool bf16,
                        cudaStream_t stream);
+
+// The persistent forward (attn_fwd_persist_sm100a.cu): p.n_ctas CTAs, each
+// taking every n_ctas-th work unit; for units of equal cost only (no causal,
+// window or block mask).
+cudaError_t launch_fwd_persist(const FwdMaps& maps, const FwdParams& p, int d, bool bf16,
+                               cudaStream_t stream);
 
 struct BwdParams {
     int B, Hq, Hkv, Nq, Nk;
@@ -138,7 +145,7 @@ cudaError_t launch_bwd(const BwdMaps& maps, const BwdParams& p, int d, bool bf16
 
 struct DecodeParams {
     const void* q;         // [B, Nq, Hq, d]
-    void* o;               // [B, Nq, Hq, d]
+    void* o;               // [B, Nq, Hq, d] (persistent forward: rows stored from registers)
     float* lse;            // [B, Hq, Nq]
     const int* cu_seqlens_k;
     const int* seqlens_k;

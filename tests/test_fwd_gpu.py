@@ -83,6 +83,17 @@ def test_long_sequence_sweep_sampled_rows(name):
     compare_selected(o, lse, o_ref, lse_ref, sel, what=name)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("kpad", [False, True])
+def test_persistent_units_more_than_sms_ragged(d, kpad):
+    # the persistent forward (non-causal, at most 4096 keys): 300 units of
+    # 256 query rows for 148 CTAs, the last row tile of every head only
+    # partly filled (Nq = 300), grouped heads, optionally key lengths
+    c = FwdCase("pu", 3, 50, 10, 300, 700, d, False, kpad_range=(1, 700) if kpad else None)
+    check_fwd(fwd_inputs(c, seed=d + kpad), False, c.scale,
+              what=f"persistent units d{d} kpad {kpad}")
+
+
 def test_fp16_head128_causal_gqa():
     c = FwdCase("h", 2, 8, 2, 384, 384, 128, True, dtype="fp16")
     check_fwd(fwd_inputs(c, seed=3), True, c.scale, what="fp16 d128 gqa causal")
