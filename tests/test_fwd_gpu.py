@@ -94,6 +94,29 @@ def test_persistent_units_more_than_sms_ragged(d, kpad):
               what=f"persistent units d{d} kpad {kpad}")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_d64_units_key_lengths_at_tile_edges(dtype):
+    # the d = 64 forward without masks (persistent units of 256 query rows):
+    # Nq = 600 leaves a unit with one partly filled Q tile; 9 x 20 heads give
+    # 540 units for 148 CTAs; the key lengths sit at and around the half-tile
+    # (64) and tile (128) edges, including none at all, and the keys behind
+    # each length hold NaN
+    c = FwdCase("u64", 9, 20, 4, 600, 333, 64, False, dtype=dtype)
+    inp = fwd_inputs(c, seed=21)
+    inp["seqlens_k"] = torch.tensor([0, 1, 63, 64, 65, 127, 128, 129, 333], dtype=torch.int32)
+    o_ref, lse_ref = dense.attn_fwd(inp["q"], inp["k"], inp["v"], c.scale, False,
+                                    seqlens_k=inp["seqlens_k"])
+    o, lse = run_fwd(inp, False, c.scale)
+    clean = compare(o, lse, o_ref, lse_ref, what=f"d64 units {dtype}")
+    assert torch.all(o[0] == 0) and torch.all(torch.isneginf(lse[0]))  # no keys
+    for b, L in enumerate(inp["seqlens_k"].tolist()):
+        inp["k"][b, L:] = float("nan")
+        inp["v"][b, L:] = float("nan")
+    o2, lse2 = run_fwd(inp, False, c.scale)
+    assert torch.equal(o2, o) and torch.equal(lse2, lse)
+    assert clean == compare(o2, lse2, o_ref, lse_ref, what=f"d64 units {dtype} NaN padding")
+
+
 def test_fp16_head128_causal_gqa():
     c = FwdCase("h", 2, 8, 2, 384, 384, 128, True, dtype="fp16")
     check_fwd(fwd_inputs(c, seed=3), True, c.scale, what="fp16 d128 gqa causal")
