@@ -76,6 +76,23 @@ def test_unfilled_slots_hold_nan():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("nq", [1, 16])
+def test_largest_batch_decode(nq):
+    # B = 65535 sequences, the largest batch the C ABI takes, 8 query heads
+    # on one kv head (the tensor-core path: its plan covers every sequence),
+    # short lengths; compared on 64 seeded sequences including the first and
+    # the last
+    c = DecodeCase("maxb", 65535, 8, 1, nq, 128, (nq, 40), nq > 1, slack=2)
+    inp = kvcache_inputs(c, seed=8)
+    o, lse = _run(inp, c)
+    g = torch.Generator().manual_seed(7)
+    sel = sorted(set([0, 1, c.B - 1] + torch.randperm(c.B, generator=g)[:61].tolist()))
+    cu, lens = inp["cu_seqlens_k"], inp["seqlens_k"]
+    o_ref, lse_ref = dense.attn_kvcache(inp["q"][sel], inp["k_cache"], inp["v_cache"], cu[sel],
+                                        lens[sel], c.scale, c.causal)
+    compare(o[sel], lse[sel], o_ref, lse_ref, what=f"B=65535 Nq={nq}")
+
+
 @pytest.mark.parametrize("d,dtype", [(64, "bf16"), (128, "fp16"), (64, "fp16")])
 def test_head_dims_and_fp16(d, dtype):
     c = DecodeCase("h", 5, 12, 3, 1, d, (1, 2500), False, dtype=dtype)

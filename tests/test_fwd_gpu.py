@@ -117,6 +117,38 @@ def test_d64_units_key_lengths_at_tile_edges(dtype):
     assert clean == compare(o2, lse2, o_ref, lse_ref, what=f"d64 units {dtype} NaN padding")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_largest_batch(d, causal):
+    # B = 65535, the largest batch the C ABI takes: one work unit per
+    # sequence (the persistent kernel strides each CTA over about 443 of
+    # them, the causal grid has 65535 CTAs); compared on 64 seeded sequences
+    # including the first and the last
+    c = FwdCase("maxb", 65535, 1, 1, 3, 5, d, causal)
+    inp = fwd_inputs(c, seed=31)
+    o, lse = run_fwd(inp, causal, c.scale)
+    g = torch.Generator().manual_seed(5)
+    sel = sorted(set([0, 1, c.B - 1] + torch.randperm(c.B, generator=g)[:61].tolist()))
+    o_ref, lse_ref = dense.attn_fwd(inp["q"][sel], inp["k"][sel], inp["v"][sel], c.scale, causal)
+    compare(o[sel], lse[sel], o_ref, lse_ref, what=f"B=65535 d{d} causal {causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_largest_head_count(causal):
+    # Hq = 65535 query heads on 5 kv heads (13107 per group), the largest
+    # head count the C ABI takes; compared on 64 seeded heads, each against
+    # its own kv head
+    c = FwdCase("maxh", 1, 65535, 5, 2, 3, 64, causal)
+    inp = fwd_inputs(c, seed=32)
+    o, lse = run_fwd(inp, causal, c.scale)
+    g = torch.Generator().manual_seed(6)
+    sel = sorted(set([0, 13106, 13107, c.Hq - 1] + torch.randperm(c.Hq, generator=g)[:60].tolist()))
+    kv = [h // (c.Hq // c.Hkv) for h in sel]
+    o_ref, lse_ref = dense.attn_fwd(inp["q"][:, :, sel], inp["k"][:, :, kv], inp["v"][:, :, kv],
+                                    c.scale, causal)
+    compare(o[:, :, sel], lse[:, sel], o_ref, lse_ref, what=f"Hq=65535 causal {causal}")
+
+
 def test_fp16_head128_causal_gqa():
     c = FwdCase("h", 2, 8, 2, 384, 384, 128, True, dtype="fp16")
     check_fwd(fwd_inputs(c, seed=3), True, c.scale, what="fp16 d128 gqa causal")
