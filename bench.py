@@ -743,7 +743,7 @@ def run_profile_case(kernel: str, launches: int):
 def run_sweep(reps: int = 20):
     """One JSON line per configured workload (forward TFLOP/s, decode GB/s),
     each timed with CUDA events over `reps` back-to-back launches after 3
-    warm-ups; inputs seeded on the device.  Not the default line."""
+    warm-ups; inputs seeded on the device.  Separate from the one JSON line of the default run."""
     from io_aware_exact_29_b200 import attn
 
     peaks, _ = load_peaks()
