@@ -210,6 +210,80 @@ def attn_fwd(q, k, v, scale=None, causal=False, seqlens_k=None, out=None, lse=No
     return out, lse
 
 
+class PinnedForward:
+    """attn_fwd on pinned host tensors, pipelined over pieces of the batch.
+
+    Every call copies all of q, k, v host -> device and all of o, lse
+    device -> host.  The batch is cut into `pieces` contiguous pieces so that
+    the copy of piece i + 1 in, the forward of piece i (one attn_fwd launch on
+    the sub-batch) and the copy of piece i - 1 out run at the same time on
+    three CUDA streams; the copies in and out also overlap across calls.  The
+    device buffers, streams and events live as long as the object: a piece's
+    input buffers are refilled only after the previous call's forward of that
+    piece has read them, and its output buffers rewritten only after the
+    previous call's copy out has read them.  Call `join(stream)` before
+    reading the host outputs or timing on `stream`.
+    """
+
+    def __init__(self, B, Nq, Hq, Nk, Hkv, d, dtype=torch.bfloat16, pieces=4, device=None):
+        dev = torch.device("cuda") if device is None else torch.device(device)
+        self.pieces = max(1, min(int(pieces), B))
+        bounds = [B * i // self.pieces for i in range(self.pieces + 1)]
+        self.ranges = [(a, b) for a, b in zip(bounds[:-1], bounds[1:]) if b > a]
+        self.q = torch.empty((B, Nq, Hq, d), dtype=dtype, device=dev)
+        self.k = torch.empty((B, Nk, Hkv, d), dtype=dtype, device=dev)
+        self.v = torch.empty((B, Nk, Hkv, d), dtype=dtype, device=dev)
+        self.o = torch.empty((B, Nq, Hq, d), dtype=dtype, device=dev)
+        self.lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
+        self.s_in = torch.cuda.Stream(dev)
+        self.s_run = torch.cuda.Stream(dev)
+        self.s_out = torch.cuda.Stream(dev)
+        n = len(self.ranges)
+        self.ev_in = [torch.cuda.Event() for _ in range(n)]
+        self.ev_run = [torch.cuda.Event() for _ in range(n)]
+        self.ev_out = [torch.cuda.Event() for _ in range(n)]
+        self.used = False  # events recorded by an earlier call
+
+    def __call__(self, q_h, k_h, v_h, o_h, lse_h, scale=None, causal=False):
+        for t, n in ((q_h, "q"), (k_h, "k"), (v_h, "v"), (o_h, "o"), (lse_h, "lse")):
+            if t.is_cuda or not t.is_pinned() or not t.is_contiguous():
+                raise ValueError(f"{n} must be a contiguous pinned host tensor")
+        if q_h.shape != self.q.shape or k_h.shape != self.k.shape or v_h.shape != self.v.shape:
+            raise ValueError("input shapes differ from the ones this object was built for")
+        if o_h.shape != self.o.shape or lse_h.shape != self.lse.shape:
+            raise ValueError("output shapes differ from the ones this object was built for")
+        if q_h.dtype != self.q.dtype or o_h.dtype != self.o.dtype or lse_h.dtype != torch.float32:
+            raise TypeError("dtype differs from the one this object was built for")
+        # work queued on the caller's stream before this call comes first
+        self.s_in.wait_stream(torch.cuda.current_stream())
+        for i, (a, b) in enumerate(self.ranges):
+            with torch.cuda.stream(self.s_in):
+                if self.used:
+                    self.s_in.wait_event(self.ev_run[i])  # the last forward read them
+                self.q[a:b].copy_(q_h[a:b], non_blocking=True)
+                self.k[a:b].copy_(k_h[a:b], non_blocking=True)
+                self.v[a:b].copy_(v_h[a:b], non_blocking=True)
+                self.ev_in[i].record(self.s_in)
+            self.s_run.wait_event(self.ev_in[i])
+            if self.used:
+                self.s_run.wait_event(self.ev_out[i])  # the last copy out read them
+            attn_fwd(self.q[a:b], self.k[a:b], self.v[a:b], scale=scale, causal=causal,
+                     out=self.o[a:b], lse=self.lse[a:b], stream=self.s_run)
+            self.ev_run[i].record(self.s_run)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(self.ev_run[i])
+                o_h[a:b].copy_(self.o[a:b], non_blocking=True)
+                lse_h[a:b].copy_(self.lse[a:b], non_blocking=True)
+                self.ev_out[i].record(self.s_out)
+        self.used = True
+        return o_h, lse_h
+
+    def join(self, stream=None):
+        """Make `stream` (default: the current one) wait for every copy out."""
+        s = stream if stream is not None else torch.cuda.current_stream()
+        s.wait_stream(self.s_out)
+
+
 def bwd_workspace_bytes(B, Hq, Nq) -> int:
     return int(load_library().attn_bwd_workspace_bytes(B, Hq, Nq))
 
