@@ -1,0 +1,125 @@
+"""Seeded random shapes against the matrix-product fp64 oracle.
+
+Each case draws its sizes from a generator seeded by the case number: batch,
+heads and their grouping, query and key lengths (ragged against the 128-row
+tiles, more queries than keys or fewer), head dim, causal or not, bf16 or
+fp16, and per-sequence key lengths with NaN behind them.  The decode cases
+add token counts 1..16, empty sequences, unfilled slots holding NaN and split
+sizes (both the tensor-core and the mma.sync instance), the paged ones block
+sizes 16..256 with NaN in every unused row, and the backward cases the
+gradients of all three inputs.  Every output element is compared, through
+guarded, NaN-prefilled buffers.
+"""
+import pytest
+import torch
+
+from oracle import dense
+from io_aware_exact_29_b200 import attn
+from io_aware_exact_29_b200.workloads import (DecodeCase, FwdCase, fwd_inputs, kvcache_inputs,
+                                              paged_from_packed, upstream_grad)
+from tests.parity import compare, compare_grads, run_fwd
+from tests.test_bwd_gpu import _run as run_bwd
+from tests.test_decode_gpu import _run as run_decode
+from tests.test_paged_gpu import _run as run_paged
+
+pytestmark = pytest.mark.gpu
+
+NAN = float("nan")
+
+
+class _Draw:
+    """Integers and choices from one seeded generator."""
+
+    def __init__(self, seed):
+        self.g = torch.Generator().manual_seed(7919 * (seed + 1))
+
+    def int(self, lo, hi):
+        return int(torch.randint(lo, hi + 1, (1,), generator=self.g).item())
+
+    def pick(self, options):
+        return options[self.int(0, len(options) - 1)]
+
+
+def _nan_behind(inp, lens):
+    for b, L in enumerate(lens):
+        inp["k"][b, L:] = NAN
+        inp["v"][b, L:] = NAN
+
+
+@pytest.mark.parametrize("seed", range(48))
+def test_forward_random_shapes(seed):
+    r = _Draw(seed)
+    B, Hkv, G = r.int(1, 4), r.pick([1, 2, 4]), r.pick([1, 2, 4, 8])
+    Nq, Nk, d = r.int(1, 700), r.int(1, 900), r.pick([64, 128])
+    causal, dtype, kpad = bool(r.int(0, 1)), r.pick(["bf16", "fp16"]), r.int(0, 2) == 0
+    c = FwdCase("fz", B, Hkv * G, Hkv, Nq, Nk, d, causal, dtype=dtype)
+    inp = fwd_inputs(c, seed=seed)
+    what = f"B{B} Hq{Hkv * G} Hkv{Hkv} Nq{Nq} Nk{Nk} d{d} causal {causal} {dtype} kpad {kpad}"
+    if kpad:
+        lens = [r.int(0, Nk) for _ in range(B)]
+        inp["seqlens_k"] = torch.tensor(lens, dtype=torch.int32)
+        _nan_behind(inp, lens)
+    o, lse = run_fwd(inp, causal, c.scale)
+    o_ref, lse_ref = dense.attn_fwd(inp["q"], inp["k"], inp["v"], c.scale, causal,
+                                    seqlens_k=inp.get("seqlens_k"))
+    compare(o, lse, o_ref, lse_ref, what=what)
+
+
+@pytest.mark.parametrize("seed", range(32))
+def test_decode_random_shapes(seed):
+    r = _Draw(100 + seed)
+    B, Hkv, G = r.int(1, 40), r.pick([1, 2, 8]), r.pick([1, 2, 4, 8, 16])
+    Nq = r.pick([1, r.int(2, 16)])
+    d, dtype = r.pick([64, 128]), r.pick(["bf16", "fp16"])
+    causal = Nq > 1 and bool(r.int(0, 1))
+    split = r.pick([0, 0, 64, 128, 1024])
+    lo = Nq if causal else 0
+    lens = [r.pick([lo, r.int(lo, 3000), r.int(lo, 3000)]) for _ in range(B)]
+    c = DecodeCase("fzd", B, Hkv * G, Hkv, Nq, d, (lo, 3000), causal, dtype=dtype,
+                   slack=r.int(0, 9))
+    inp = kvcache_inputs(c, seed=seed, seqlens=lens, slack_fill=NAN)
+    o, lse = run_decode(inp, c, split_keys=split)
+    o_ref, lse_ref = dense.attn_kvcache(inp["q"], inp["k_cache"], inp["v_cache"],
+                                        inp["cu_seqlens_k"], inp["seqlens_k"], c.scale, causal)
+    compare(o, lse, o_ref, lse_ref,
+            what=f"decode B{B} G{G} Hkv{Hkv} Nq{Nq} d{d} {dtype} causal {causal} split {split}")
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_paged_random_shapes(seed):
+    r = _Draw(200 + seed)
+    block = r.pick([16, 32, 64, 128, 256])
+    B, Hkv, G = r.int(1, 24), r.pick([1, 2, 8]), r.pick([1, 2, 4, 8, 16])
+    Nq = r.int(1, min(16, 128 // G))
+    d, dtype = r.pick([64, 128]), r.pick(["bf16", "fp16"])
+    causal = Nq > 1 and bool(r.int(0, 1))
+    lo = Nq if causal else 0
+    lens = [r.int(lo, 3000) for _ in range(B)]
+    c = DecodeCase("fzp", B, Hkv * G, Hkv, Nq, d, (lo, 3000), causal, dtype=dtype)
+    inp = kvcache_inputs(c, seed=seed, seqlens=lens)
+    pg = paged_from_packed(inp, block, seed=seed)
+    o, lse, _ = run_paged(inp, pg, c)
+    o_ref, lse_ref = dense.attn_kvcache(inp["q"], inp["k_cache"], inp["v_cache"],
+                                        inp["cu_seqlens_k"], inp["seqlens_k"], c.scale, causal)
+    compare(o, lse, o_ref, lse_ref,
+            what=f"paged bs{block} B{B} G{G} Hkv{Hkv} Nq{Nq} d{d} {dtype} causal {causal}")
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_backward_random_shapes(seed):
+    r = _Draw(300 + seed)
+    B, Hkv, G = r.int(1, 3), r.pick([1, 2]), r.pick([1, 2, 4])
+    Nq, Nk, d = r.int(1, 400), r.int(1, 500), r.pick([64, 128])
+    causal, dtype, kpad = bool(r.int(0, 1)), r.pick(["bf16", "fp16"]), r.int(0, 2) == 0
+    c = FwdCase("fzb", B, Hkv * G, Hkv, Nq, Nk, d, causal, dtype=dtype)
+    inp = fwd_inputs(c, seed=seed)
+    if kpad:
+        lens = [r.int(1, Nk) for _ in range(B)]
+        inp["seqlens_k"] = torch.tensor(lens, dtype=torch.int32)
+        _nan_behind(inp, lens)
+    dout = upstream_grad(inp["q"], seed=seed)
+    got = run_bwd(inp, c, dout)
+    ref = dense.attn_bwd(inp["q"], inp["k"], inp["v"], dout, c.scale, causal,
+                         seqlens_k=inp.get("seqlens_k"))
+    compare_grads(got, ref, what=f"bwd B{B} Hq{Hkv * G} Hkv{Hkv} Nq{Nq} Nk{Nk} d{d} "
+                                 f"causal {causal} {dtype} kpad {kpad}")
