@@ -62,8 +62,15 @@ def compare_selected(o_gpu, lse_gpu, o_ref, lse_ref, sel, what=""):
 # The normalisers have a floor of GRAD_FLOOR: where the exact gradient is 0
 # (one key: P = 1, so dS = dP - D = 0) the test is an absolute one, and with
 # N(0, 1) inputs the gradients of every real case are well above it.
+# With fewer than 64 visible keys per row nothing shrinks |O| by averaging,
+# so the error D inherits from the bf16 output (about sqrt(d) 2^-9 |dO| |O|)
+# is no longer small against dP - D: for a two-key row dS_0 = -dS_1 =
+# P_0 P_1 (dP_0 - dP_1) and the relative error of dq grows as 1 / P_1, up to
+# about 1% for a peaked row.  Such shapes get the looser mean bound.
 GRAD_MAX_REL = 2e-2   # max |err| / max(max |ref|, floor)
 GRAD_MEAN_REL = 5e-3  # mean |err| / max(mean |ref|, floor)
+GRAD_MEAN_REL_FEW_KEYS = 1e-2  # the same, rows with fewer than 64 visible keys
+GRAD_FEW_KEYS = 64
 GRAD_FLOOR = 1e-3
 
 
@@ -106,9 +113,10 @@ def check_defined(what, *tensors):
         assert not bool(torch.isnan(t.float()).any()), f"{what}: NaN left in an output"
 
 
-def compare_grads(gpu, ref, what="", key_rows=None):
+def compare_grads(gpu, ref, what="", key_rows=None, mean_rel=GRAD_MEAN_REL):
     """gpu: (dq, dk, dv) tensors; ref: the oracle's float64 arrays.
-    key_rows: optional slice of key rows that dk/dv are compared on."""
+    key_rows: optional slice of key rows that dk/dv are compared on;
+    mean_rel: the mean bound (GRAD_MEAN_REL_FEW_KEYS for few-key shapes)."""
     out = {}
     for name, g, r in zip(("dq", "dk", "dv"), gpu, ref):
         a = g.float().cpu().numpy().astype(np.float64)
@@ -123,7 +131,7 @@ def compare_grads(gpu, ref, what="", key_rows=None):
         out[name] = (emax, emean)
         msg = f"{what} {name}: max rel {emax:.3e} mean rel {emean:.3e}"
         assert emax <= GRAD_MAX_REL, msg
-        assert emean <= GRAD_MEAN_REL, msg
+        assert emean <= mean_rel, msg
     return out
 
 

@@ -7,9 +7,13 @@ fp16, and per-sequence key lengths with NaN behind them.  The decode cases
 add token counts 1..16, empty sequences, unfilled slots holding NaN and split
 sizes (both the tensor-core and the mma.sync instance), the paged ones block
 sizes 16..256 with NaN in every unused row, and the backward cases the
-gradients of all three inputs.  Every output element is compared, through
+gradients of all three inputs.  The softmax scale is 1/sqrt(d) in most cases
+and otherwise small (nearly uniform rows) or large (nearly one-hot rows, many
+moves of the running maximum).  Every output element is compared, through
 guarded, NaN-prefilled buffers.
 """
+from types import SimpleNamespace
+
 import pytest
 import torch
 
@@ -17,7 +21,8 @@ from oracle import dense
 from io_aware_exact_29_b200 import attn
 from io_aware_exact_29_b200.workloads import (DecodeCase, FwdCase, fwd_inputs, kvcache_inputs,
                                               paged_from_packed, upstream_grad)
-from tests.parity import compare, compare_grads, run_fwd
+from tests.parity import (GRAD_FEW_KEYS, GRAD_MEAN_REL, GRAD_MEAN_REL_FEW_KEYS, compare,
+                          compare_grads, run_fwd)
 from tests.test_bwd_gpu import _run as run_bwd
 from tests.test_decode_gpu import _run as run_decode
 from tests.test_paged_gpu import _run as run_paged
@@ -53,14 +58,16 @@ def test_forward_random_shapes(seed):
     Nq, Nk, d = r.int(1, 700), r.int(1, 900), r.pick([64, 128])
     causal, dtype, kpad = bool(r.int(0, 1)), r.pick(["bf16", "fp16"]), r.int(0, 2) == 0
     c = FwdCase("fz", B, Hkv * G, Hkv, Nq, Nk, d, causal, dtype=dtype)
+    scale = r.pick([c.scale, c.scale, c.scale, 0.02, 0.3, 1.0])
     inp = fwd_inputs(c, seed=seed)
-    what = f"B{B} Hq{Hkv * G} Hkv{Hkv} Nq{Nq} Nk{Nk} d{d} causal {causal} {dtype} kpad {kpad}"
+    what = (f"B{B} Hq{Hkv * G} Hkv{Hkv} Nq{Nq} Nk{Nk} d{d} causal {causal} {dtype} "
+            f"kpad {kpad} scale {scale}")
     if kpad:
         lens = [r.int(0, Nk) for _ in range(B)]
         inp["seqlens_k"] = torch.tensor(lens, dtype=torch.int32)
         _nan_behind(inp, lens)
-    o, lse = run_fwd(inp, causal, c.scale)
-    o_ref, lse_ref = dense.attn_fwd(inp["q"], inp["k"], inp["v"], c.scale, causal,
+    o, lse = run_fwd(inp, causal, scale)
+    o_ref, lse_ref = dense.attn_fwd(inp["q"], inp["k"], inp["v"], scale, causal,
                                     seqlens_k=inp.get("seqlens_k"))
     compare(o, lse, o_ref, lse_ref, what=what)
 
@@ -77,12 +84,14 @@ def test_decode_random_shapes(seed):
     lens = [r.pick([lo, r.int(lo, 3000), r.int(lo, 3000)]) for _ in range(B)]
     c = DecodeCase("fzd", B, Hkv * G, Hkv, Nq, d, (lo, 3000), causal, dtype=dtype,
                    slack=r.int(0, 9))
+    scale = r.pick([c.scale, c.scale, c.scale, 0.02, 0.3, 1.0])
     inp = kvcache_inputs(c, seed=seed, seqlens=lens, slack_fill=NAN)
-    o, lse = run_decode(inp, c, split_keys=split)
+    o, lse = run_decode(inp, SimpleNamespace(scale=scale, causal=causal, Hkv=Hkv),
+                        split_keys=split)
     o_ref, lse_ref = dense.attn_kvcache(inp["q"], inp["k_cache"], inp["v_cache"],
-                                        inp["cu_seqlens_k"], inp["seqlens_k"], c.scale, causal)
-    compare(o, lse, o_ref, lse_ref,
-            what=f"decode B{B} G{G} Hkv{Hkv} Nq{Nq} d{d} {dtype} causal {causal} split {split}")
+                                        inp["cu_seqlens_k"], inp["seqlens_k"], scale, causal)
+    compare(o, lse, o_ref, lse_ref, what=f"decode B{B} G{G} Hkv{Hkv} Nq{Nq} d{d} {dtype} "
+                                         f"causal {causal} split {split} scale {scale}")
 
 
 @pytest.mark.parametrize("seed", range(16))
@@ -98,11 +107,12 @@ def test_paged_random_shapes(seed):
     c = DecodeCase("fzp", B, Hkv * G, Hkv, Nq, d, (lo, 3000), causal, dtype=dtype)
     inp = kvcache_inputs(c, seed=seed, seqlens=lens)
     pg = paged_from_packed(inp, block, seed=seed)
-    o, lse, _ = run_paged(inp, pg, c)
+    scale = r.pick([c.scale, c.scale, 0.3, 1.0])
+    o, lse, _ = run_paged(inp, pg, SimpleNamespace(scale=scale, causal=causal, Hkv=Hkv))
     o_ref, lse_ref = dense.attn_kvcache(inp["q"], inp["k_cache"], inp["v_cache"],
-                                        inp["cu_seqlens_k"], inp["seqlens_k"], c.scale, causal)
-    compare(o, lse, o_ref, lse_ref,
-            what=f"paged bs{block} B{B} G{G} Hkv{Hkv} Nq{Nq} d{d} {dtype} causal {causal}")
+                                        inp["cu_seqlens_k"], inp["seqlens_k"], scale, causal)
+    compare(o, lse, o_ref, lse_ref, what=f"paged bs{block} B{B} G{G} Hkv{Hkv} Nq{Nq} d{d} "
+                                         f"{dtype} causal {causal} scale {scale}")
 
 
 @pytest.mark.parametrize("seed", range(16))
@@ -117,9 +127,20 @@ def test_backward_random_shapes(seed):
         lens = [r.int(1, Nk) for _ in range(B)]
         inp["seqlens_k"] = torch.tensor(lens, dtype=torch.int32)
         _nan_behind(inp, lens)
+    scale = r.pick([c.scale, c.scale, 0.02, 0.3])
     dout = upstream_grad(inp["q"], seed=seed)
-    got = run_bwd(inp, c, dout)
-    ref = dense.attn_bwd(inp["q"], inp["k"], inp["v"], dout, c.scale, causal,
+    got = run_bwd(inp, SimpleNamespace(scale=scale, causal=causal), dout)
+    ref = dense.attn_bwd(inp["q"], inp["k"], inp["v"], dout, scale, causal,
                          seqlens_k=inp.get("seqlens_k"))
+    # keys each row sees (bottom-right causal), averaged over rows that see any
+    seen = []
+    for b in range(B):
+        L = lens[b] if kpad else Nk
+        for i in range(Nq):
+            n = max(0, min(L, i + L - Nq + 1)) if causal else L
+            if n > 0:
+                seen.append(n)
+    few = not seen or sum(seen) / len(seen) < GRAD_FEW_KEYS
     compare_grads(got, ref, what=f"bwd B{B} Hq{Hkv * G} Hkv{Hkv} Nq{Nq} Nk{Nk} d{d} "
-                                 f"causal {causal} {dtype} kpad {kpad}")
+                                 f"causal {causal} {dtype} kpad {kpad} scale {scale}",
+                  mean_rel=GRAD_MEAN_REL_FEW_KEYS if few else GRAD_MEAN_REL)
