@@ -6,8 +6,10 @@ tiles, more queries than keys or fewer), head dim, causal or not, bf16 or
 fp16, and per-sequence key lengths with NaN behind them.  The decode cases
 add token counts 1..16, empty sequences, unfilled slots holding NaN and split
 sizes (both the tensor-core and the mma.sync instance), the paged ones block
-sizes 16..256 with NaN in every unused row, and the backward cases the
-gradients of all three inputs.  The softmax scale is 1/sqrt(d) in most cases
+sizes 16..256 with NaN in every unused row (and the fused append of the new
+tokens' K/V), the backward cases the gradients of all three inputs, and the
+masked cases sliding windows and block masks in the forward and backward
+(against the C oracle, which takes both).  The softmax scale is 1/sqrt(d) in most cases
 and otherwise small (nearly uniform rows) or large (nearly one-hot rows, many
 moves of the running maximum).  Every output element is compared, through
 guarded, NaN-prefilled buffers.
@@ -144,3 +146,89 @@ def test_backward_random_shapes(seed):
     compare_grads(got, ref, what=f"bwd B{B} Hq{Hkv * G} Hkv{Hkv} Nq{Nq} Nk{Nk} d{d} "
                                  f"causal {causal} {dtype} kpad {kpad} scale {scale}",
                   mean_rel=GRAD_MEAN_REL_FEW_KEYS if few else GRAD_MEAN_REL)
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_masked_forward_and_backward_random_shapes(seed):
+    # sliding windows and block masks (against the C oracle, which takes both)
+    import numpy as np
+
+    import oracle
+
+    r = _Draw(400 + seed)
+    B, Hkv, G = r.int(1, 2), r.pick([1, 2]), r.pick([1, 2, 4])
+    Nq, Nk, d = r.int(1, 400), r.int(1, 500), r.pick([64, 128])
+    causal, dtype = bool(r.int(0, 1)), r.pick(["bf16", "fp16"])
+    window = r.pick([-1, r.int(0, 300)])
+    sparse = r.int(0, 1) == 1 or window < 0
+    c = FwdCase("fzm", B, Hkv * G, Hkv, Nq, Nk, d, causal, dtype=dtype)
+    inp = fwd_inputs(c, seed=seed)
+    what = f"masked B{B} Hq{Hkv * G} Nq{Nq} Nk{Nk} d{d} causal {causal} window {window}"
+    mask = None
+    if sparse:
+        blk = attn.MASK_BLOCK
+        rng = np.random.default_rng(seed)
+        shape = (r.pick([1, B]), r.pick([1, Hkv * G]), -(-Nq // blk), -(-Nk // blk))
+        mask = (rng.random(shape) < r.pick([0.3, 0.6, 0.9])).astype(np.uint8)
+        what += f" block mask {shape}"
+    dev = {n: inp[n].cuda() for n in ("q", "k", "v")}
+    m = None if mask is None else torch.from_numpy(mask).cuda()
+    o, lse = attn.attn_fwd(dev["q"], dev["k"], dev["v"], scale=c.scale, causal=causal,
+                           window_left=window, block_mask=m)
+    dout = upstream_grad(inp["q"], seed=seed)
+    dq, dk, dv = attn.attn_bwd(dev["q"], dev["k"], dev["v"], o, lse, dout.cuda(),
+                               scale=c.scale, causal=causal, window_left=window, block_mask=m)
+    torch.cuda.synchronize()
+    assert attn.get_device_error() == 0
+    kw = dict(window_left=window)
+    if mask is not None:
+        kw.update(block_mask=mask, block_size=attn.MASK_BLOCK)
+    o_ref, lse_ref = oracle.attn_fwd(inp["q"], inp["k"], inp["v"], c.scale, causal, **kw)
+    compare(o, lse, o_ref, lse_ref, what=what)
+    ref = oracle.attn_bwd(inp["q"], inp["k"], inp["v"], dout, c.scale, causal, **kw)
+    # keys each (batch, head, row) sees under causal, window and block mask,
+    # averaged over the rows that see any (the mean bound depends on it)
+    i = np.arange(Nq)[:, None]
+    j = np.arange(Nk)[None, :]
+    vis = np.ones((Nq, Nk), dtype=bool)
+    if causal:
+        vis &= j <= i + Nk - Nq
+    if window >= 0:
+        vis &= j >= i + Nk - Nq - window
+    seen = []
+    for b in range(B):
+        for h in range(Hkv * G):
+            v_bh = vis
+            if mask is not None:
+                mb = mask[min(b, mask.shape[0] - 1), min(h, mask.shape[1] - 1)]
+                v_bh = vis & mb[i // attn.MASK_BLOCK, j // attn.MASK_BLOCK].astype(bool)
+            n = v_bh.sum(axis=1)
+            seen.extend(n[n > 0].tolist())
+    few = not seen or sum(seen) / len(seen) < GRAD_FEW_KEYS
+    compare_grads((dq, dk, dv), ref, what=what,
+                  mean_rel=GRAD_MEAN_REL_FEW_KEYS if few else GRAD_MEAN_REL)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_paged_append_random_shapes(seed):
+    # the fused append writes the new tokens' K/V into the paged cache, then
+    # the decode reads them with the rest of each sequence
+    import oracle
+
+    r = _Draw(500 + seed)
+    block = r.pick([16, 32, 64, 256])
+    B, Hkv, G = r.int(1, 12), r.pick([1, 2, 8]), r.pick([1, 2, 4, 8])
+    Nq = r.int(1, min(16, 128 // G))
+    d, dtype = r.pick([64, 128]), r.pick(["bf16", "fp16"])
+    causal = Nq > 1 and bool(r.int(0, 1))
+    lens = [r.int(Nq, 3000) for _ in range(B)]
+    c = DecodeCase("fza", B, Hkv * G, Hkv, Nq, d, (Nq, 3000), causal, dtype=dtype)
+    inp = kvcache_inputs(c, seed=seed, seqlens=lens)
+    full = paged_from_packed(inp, block, seed=seed)
+    holes = paged_from_packed(inp, block, seed=seed, new_tokens=Nq)
+    o, lse, dev = run_paged(inp, holes, c, with_new=True)
+    o_ref, lse_ref = oracle.attn_kvcache(inp["q"], inp["k_cache"], inp["v_cache"],
+                                         inp["cu_seqlens_k"], inp["seqlens_k"], c.scale, causal)
+    compare(o, lse, o_ref, lse_ref, what=f"append bs{block} B{B} G{G} Nq{Nq} d{d} {dtype}")
+    for name in ("k_cache", "v_cache"):
+        assert torch.equal(dev[name].cpu().view(torch.int16), full[name].view(torch.int16))
