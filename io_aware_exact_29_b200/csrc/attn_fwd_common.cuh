@@ -16,7 +16,8 @@ constexpr uint32_t kTmemCols = 512;
 // maximum exceeds it by more than this (log2 units), so P <= 2^8; numerator
 // and denominator share the reference, so the result is the same exact softmax.
 constexpr float kRescaleThreshold = 8.0f;
-// one exponential pair in FWD_POLY_EVERY(D) is evaluated on the FMA pipe
+// one exponential pair in FWD_POLY_EVERY(D) is evaluated on the FMA pipe (the
+// one-CTA-per-unit kernel; the persistent kernel sets its own share)
 #ifndef FWD_POLY_EVERY
 #define FWD_POLY_EVERY(D) 4
 #endif

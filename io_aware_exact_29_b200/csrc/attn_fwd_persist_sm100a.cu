@@ -116,7 +116,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kBlockBytes = kBlockM * 128;
     constexpr uint32_t kIdescS = ptx::idesc_f16(kBlockM, kBlockN, BF16, false);
     constexpr uint32_t kIdescO = ptx::idesc_f16(kBlockM, D, BF16, true);
-    constexpr int kPolyEvery = FWD_POLY_EVERY(D);
+    // one exponential pair in kPolyEvery on the FMA pipe: fewer than in the
+    // one-CTA-per-unit kernel, whose long causal grids prefer a quarter
+    // (measured on this kernel: 1/6 at d = 128 +1.4% at 4096 keys against
+    // 1/4, 1/12 at d = 64 +4%; more or fewer lost)
+    constexpr int kPolyEvery = D == 64 ? 12 : 6;
     // d = 64 leaves 128 tensor-memory columns free: P_a gets its own 64
     // columns (P0 [384, 448), P1 [448, 512)), so S_a of the next tile can be
     // computed as soon as the softmax has loaded S_a, while it still forms P_a
