@@ -97,9 +97,9 @@ __device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_bas
         const uint64_t t2 = ptx::f2_fma(ptx::f2_pack(v0, v1), sl2_2, nm_2);
         float p0, p1;
         if (((c >> 1) % kPolyEvery) == kPolyEvery - 1) {
-            // a share of the pairs on the FMA pipe: the exp2 unit and the tensor
-            // pipe carry equal work at d = 128 (a quarter moves), the exp2 unit
-            // twice the tensor pipe's at d = 64
+            // a share of the pairs on the FMA pipe, taking load off the exp2
+            // unit (each kernel sets its share: it trades exp2-unit cycles
+            // for FMA-pipe and issue cycles of the same warps)
             ptx::f2_unpack(ptx::exp2_poly2(t2), p0, p1);
         } else {
             float t0, t1;
