@@ -112,5 +112,93 @@ __device__ __forceinline__ void half_exp(const uint32_t (&r)[2][32], int key_bas
     }
 }
 
+// Masked tiles, 32 columns at a time: for a chunk of keys
+// [key_base, key_base + 32) the warp takes one of three paths, the same for
+// all its lanes -- every key visible for every row (kVisible: the unmasked
+// arithmetic), every key masked for every row (kHidden: nothing to compute,
+// P = 0), or a mix (kMixed: the per-element mask).  On a causal diagonal tile
+// most warps have chunks of the first two kinds.  The results are those of
+// the per-element mask, bit for bit: a visible key's value is untouched by
+// it, and a hidden key's exponential is exactly 0.
+enum ChunkMode : int { kVisible = 0, kMixed = 1, kHidden = 2 };
+
+template <bool kLow>
+__device__ __forceinline__ int chunk_mode(int key_base, int row_first, int row_lim) {
+    const bool vis = key_base + 31 <= row_lim && (!kLow || key_base >= row_first);
+    const bool hid = key_base > row_lim || (kLow && key_base + 31 < row_first);
+    if (__all_sync(0xffffffffu, vis)) return kVisible;
+    if (__all_sync(0xffffffffu, hid)) return kHidden;
+    return kMixed;
+}
+
+// half_max over a masked tile's 64 columns, chunk by chunk.
+template <bool kLow>
+__device__ __forceinline__ void half_max_chunks(const uint32_t (&r)[2][32], int key_base,
+                                                int row_first, int row_lim, float (&mx8)[8]) {
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+        const int mode = chunk_mode<kLow>(key_base + 32 * ch, row_first, row_lim);
+        if (mode == kHidden) continue;
+        const bool mask = mode == kMixed;
+#pragma unroll
+        for (int c = 32 * ch; c < 32 * ch + 32; c += 16) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int c0 = c + u, c1 = c + 8 + u;
+                float v0 = __uint_as_float(r[c0 >> 5][c0 & 31]);
+                float v1 = __uint_as_float(r[c1 >> 5][c1 & 31]);
+                if (mask) {
+                    if (key_base + c0 > row_lim || (kLow && key_base + c0 < row_first))
+                        v0 = -INFINITY;
+                    if (key_base + c1 > row_lim || (kLow && key_base + c1 < row_first))
+                        v1 = -INFINITY;
+                }
+                mx8[u] = ptx::max3(mx8[u], v0, v1);
+            }
+        }
+    }
+}
+
+// half_exp over a masked tile's 64 columns, chunk by chunk (hidden chunks
+// give P = 0 and add nothing to the row sum).
+template <bool kLow, bool BF16, int kPolyEvery>
+__device__ __forceinline__ void half_exp_chunks(const uint32_t (&r)[2][32], int key_base,
+                                                int row_first, int row_lim, uint64_t sl2_2,
+                                                uint64_t nm_2, uint64_t (&acc2)[4],
+                                                uint32_t (&pk)[32]) {
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+        const int mode = chunk_mode<kLow>(key_base + 32 * ch, row_first, row_lim);
+        if (mode == kHidden) {
+#pragma unroll
+            for (int c = 32 * ch; c < 32 * ch + 32; c += 2) pk[c >> 1] = 0u;
+            continue;
+        }
+        const bool mask = mode == kMixed;
+#pragma unroll
+        for (int c = 32 * ch; c < 32 * ch + 32; c += 2) {
+            float v0 = __uint_as_float(r[c >> 5][c & 31]);
+            float v1 = __uint_as_float(r[c >> 5][(c & 31) + 1]);
+            if (mask) {
+                if (key_base + c > row_lim || (kLow && key_base + c < row_first)) v0 = -INFINITY;
+                if (key_base + c + 1 > row_lim || (kLow && key_base + c + 1 < row_first))
+                    v1 = -INFINITY;
+            }
+            const uint64_t t2 = ptx::f2_fma(ptx::f2_pack(v0, v1), sl2_2, nm_2);
+            float p0, p1;
+            if (((c >> 1) % kPolyEvery) == kPolyEvery - 1) {
+                ptx::f2_unpack(ptx::exp2_poly2(t2), p0, p1);
+            } else {
+                float t0, t1;
+                ptx::f2_unpack(t2, t0, t1);
+                p0 = ptx::ex2_approx(t0);
+                p1 = ptx::ex2_approx(t1);
+            }
+            acc2[(c >> 1) & 3] = ptx::f2_add(acc2[(c >> 1) & 3], ptx::f2_pack(p0, p1));
+            pk[c >> 1] = ptx::pack2<BF16>(p0, p1);
+        }
+    }
+}
+
 }  // namespace fwd
 }  // namespace attn

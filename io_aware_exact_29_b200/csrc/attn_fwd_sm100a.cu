@@ -482,6 +482,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_after();
             const int key0 = j * kBlockN;
             const bool masked = key0 + kBlockN - 1 > row_lim || (kWindow && key0 < row_first);
+            // the chunk-wise path holds warp-collective votes: taken by the
+            // whole warp when any of its rows needs the mask (a row that does
+            // not finds all its chunks visible, with the same results)
+            const bool masked_w = __any_sync(0xffffffffu, masked);
             // pass 1: row maximum, two halves of 64 columns, eight independent
             // chains of three-input maxima
             float mx8[8];
@@ -502,8 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int hf = 0; hf < 2; ++hf) {
                     ptx::tmem_wait_ld_dep(r[hf][0]);
                     ptx::tmem_wait_ld_dep(r[hf][1]);
-                    if (masked)
+                    if (masked && kWindow)
                         half_max<true, kWindow>(r[hf], key0 + hf * 64, row_first, row_lim, mx8);
+                    else if (!kWindow && masked_w)
+                        half_max_chunks<false>(r[hf], key0 + hf * 64, row_first, row_lim, mx8);
                     else
                         half_max<false, kWindow>(r[hf], key0 + hf * 64, row_first, row_lim, mx8);
                 }
@@ -578,10 +584,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 auto& r = hf >= kKept ? rl : rs[hf];
                 uint32_t pk[32];
-                if (masked)
+                if (masked && kWindow)
                     half_exp<true, kWindow, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
-                                                              row_lim, sl2_2,
-                                                     nm_2, acc2, pk);
+                                                              row_lim, sl2_2, nm_2, acc2, pk);
+                else if (!kWindow && masked_w)
+                    half_exp_chunks<false, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
+                                                             row_lim, sl2_2, nm_2, acc2, pk);
                 else
                     half_exp<false, kWindow, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
                                                                row_lim, sl2_2,
