@@ -490,6 +490,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tc_fence_after();
                 const int key0 = j * kBlockN;
                 const bool masked = key0 + kBlockN - 1 > row_lim;
+                // d = 64: masked tiles are taken 32 columns at a time, by the
+                // whole warp (the chunk votes are warp-collective; a row
+                // without masked keys finds its chunks visible, with the same
+                // results).  At d = 128 the chunk code cost the unmasked tiles
+                // 1.3% (measured), so that instance keeps the per-element mask.
+                constexpr bool kChunkMask = D == 64;
+                const bool masked_w = kChunkMask && __any_sync(0xffffffffu, masked);
                 // pass 1: row maximum, two halves of 64 columns, eight independent
                 // chains of three-input maxima
                 float mx8[8];
@@ -508,7 +515,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int hf = 0; hf < 2; ++hf) {
                         ptx::tmem_wait_ld_dep(r[hf][0]);
                         ptx::tmem_wait_ld_dep(r[hf][1]);
-                        if (masked)
+                        if (masked_w)
+                            half_max_chunks<false>(r[hf], key0 + hf * 64, row_first, row_lim, mx8);
+                        else if (!kChunkMask && masked)
                             half_max<true, false>(r[hf], key0 + hf * 64, row_first, row_lim, mx8);
                         else
                             half_max<false, false>(r[hf], key0 + hf * 64, row_first, row_lim,
@@ -592,7 +601,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int hf = 0; hf < 2; ++hf) {
                     auto& r = rs[hf];
                     uint32_t pk[32];
-                    if (masked)
+                    if (masked_w)
+                        half_exp_chunks<false, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
+                                                                  row_lim, sl2_2, nm_2, acc2, pk);
+                    else if (!kChunkMask && masked)
                         half_exp<true, false, BF16, kPolyEvery>(r, key0 + hf * 64, row_first,
                                                                   row_lim, sl2_2, nm_2, acc2, pk);
                     else
