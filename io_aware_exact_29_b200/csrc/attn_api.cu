@@ -113,6 +113,19 @@ bool map_bnhd(CUtensorMap* m, int dtype, const void* base, int B, int N, int H, 
     return encode_map(m, dtype, base, 4, dims, strides, box);
 }
 
+// V of a KV cache [slots, Hkv, d] for the tensor-core decode, seen as
+// {64 columns, slot, 64-column block, head} (the third dimension's stride,
+// 128 bytes, is smaller than the second's: the map walks the same memory in
+// another order).  One box of `rows` slots lands as [64-column block][row]
+// [128 B]: a run of cache rows with all d columns.
+bool map_v_runs(CUtensorMap* m, int dtype, const void* base, uint64_t slots, int Hkv, int d,
+                int rows) {
+    const uint64_t dims[4] = {64, slots, (uint64_t)d / 64, (uint64_t)Hkv};
+    const uint64_t strides[3] = {(uint64_t)Hkv * d * 2, 128, (uint64_t)d * 2};
+    const uint32_t box[4] = {64, (uint32_t)rows, (uint32_t)d / 64, 1};
+    return encode_map(m, dtype, base, 4, dims, strides, box);
+}
+
 constexpr BlockMask kNoBlockMask{nullptr, 0, 0, 0};
 
 int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
@@ -347,7 +360,8 @@ int attn_fwd_varlen_kvcache(const void* q, const void* k_cache, const void* v_ca
     const uint64_t strides[2] = {(uint64_t)d * 2, (uint64_t)Hkv * d * 2};
     const uint32_t box[3] = {64, 1, lay.tc ? 128u : 64u};
     if (!encode_map(&kmap, dtype, k_cache, 3, dims, strides, box) ||
-        !encode_map(&vmap, dtype, v_cache, 3, dims, strides, box))
+        !(lay.tc ? map_v_runs(&vmap, dtype, v_cache, (uint64_t)cache_slots, Hkv, d, 128)
+                 : encode_map(&vmap, dtype, v_cache, 3, dims, strides, box)))
         return ATTN_ERR_INVALID_ARG;
     if (lay.tc) {
         // Q and O [B, Nq, Hq, d] seen as {d, G, Hkv, Nq, B}: one box gathers
@@ -448,7 +462,7 @@ int attn_fwd_paged_kvcache(const void* q, void* k_cache, void* v_cache, const in
     const uint64_t strides[2] = {(uint64_t)d * 2, (uint64_t)Hkv * d * 2};
     const uint32_t box[3] = {64, 1, (uint32_t)std::min(128, block_size)};
     if (!encode_map(&kmap, dtype, k_cache, 3, dims, strides, box) ||
-        !encode_map(&vmap, dtype, v_cache, 3, dims, strides, box))
+        !map_v_runs(&vmap, dtype, v_cache, slots, Hkv, d, std::min(128, block_size)))
         return ATTN_ERR_INVALID_ARG;
     const uint64_t qdims[5] = {(uint64_t)d, (uint64_t)G, (uint64_t)Hkv, (uint64_t)Nq, (uint64_t)B};
     const uint64_t qstrides[4] = {(uint64_t)d * 2, (uint64_t)G * d * 2, (uint64_t)Hq * d * 2,

@@ -27,7 +27,7 @@
 // gathers the 128 rows (tokens past Nq read as zeros).
 // Warp roles (576 threads):
 //   warps 0-15  softmax: rows 32*(w%4) .. +31, score columns 32*(w/4) .. +31
-//   warp 16     loader: work list, Q, 128-key K / V tiles of the packed cache
+//   warp 16     loader: work list, Q, 128-key K / V tiles
 //   warp 17     tensor-memory owner and tcgen05.mma issuer (elected lane)
 // Tensor memory: S[0] [0,128), S[1] [128,256) double-buffered scores,
 // O [256, 256+D), Q [384, 384+D/2).  The softmax warps copy each item's Q
@@ -370,6 +370,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kPartD = D / 4;
     constexpr int kLoaderWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
     static_assert(sizeof(TcBars<KST, VST>) <= 1024, "barrier block");
+    // A tile's keys arrive in runs of 2^sub_shift rows: a paged cache's block
+    // (or a 128-row piece of a larger one), or the whole tile of a packed
+    // cache.  K is laid out [64-column block][row][128 B]; V is laid out
+    // [run][64-column block][run row][128 B], so that one TMA box brings a
+    // run's rows with all their columns (a 16-row block then costs one V
+    // box instead of D / 64; the number of boxes, not of bytes, bounds a
+    // 16-row paged decode).  For the whole tile the two layouts coincide.
+    const int sub_shift = p.block_table ? min(7, p.block_shift) : 7;
+    const uint32_t run_bytes = (uint32_t)D * 2u << sub_shift;
+    auto v_row = [&](int key) -> uint32_t {  // byte offset of tile row `key`, block 0
+        return (uint32_t)(key >> sub_shift) * run_bytes +
+               (uint32_t)(key & ((1 << sub_shift) - 1)) * 128u;
+    };
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = ptx::smem_u32(smem_raw);
@@ -482,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         // a paged cache is read in runs of sub_rows rows (one block, or one
         // 128-row tile of a larger block)
-        const int sub_rows = p.block_table ? min(kBlockN, 1 << p.block_shift) : kBlockN;
+        const int sub_rows = 1 << sub_shift;
         const int n_sub = kBlockN / sub_rows;
         int n = 0;        // items pushed
         int it = 0;       // items with keys (Q loads)
@@ -545,14 +558,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                             row0 = (blk << p.block_shift) + (pos & ((1 << p.block_shift) - 1));
                         }
                     }
-                    // issue the tile's copies: n_sub runs of sub_rows rows per
-                    // 64-column block, each at its own place in the tile; lane u
-                    // issues run u (the lanes' copies go out together)
-                    auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar) {
+                    // issue the tile's copies, lane u run u (the lanes' copies
+                    // go out together): for K one box per 64-column block, each
+                    // at its own place in the tile; for V one box per run
+                    auto load_k = [&](uint8_t* dst, uint64_t* bar) {
                         if (lane < n_sub)
                             for (int c = 0; c < kDBlocks; ++c)
-                                ptx::tma_load_3d(dst + c * kBlockBytes + lane * sub_rows * 128, map,
-                                                 bar, c * 64, item.g, row0);
+                                ptx::tma_load_3d(dst + c * kBlockBytes + lane * sub_rows * 128,
+                                                 &tm_k, bar, c * 64, item.g, row0);
+                    };
+                    auto load_v = [&](uint8_t* dst, uint64_t* bar) {
+                        if (lane < n_sub)
+                            ptx::tma_load_4d(dst + lane * run_bytes, &tm_v, bar, 0, row0, 0,
+                                             item.g);
                     };
                     const int sk = tg % KST;
                     if (!warp_wait(&bars->k_empty[sk], ((tg / KST) & 1) ^ 1, p.limit_ns,
@@ -563,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (lane == 0) ptx::mbar_arrive_expect_tx(&bars->k_full[sk], kTileBytes);
                     __syncwarp();
-                    load_tile(smem + L::kK + sk * kTileBytes, &tm_k, &bars->k_full[sk]);
+                    load_k(smem + L::kK + sk * kTileBytes, &bars->k_full[sk]);
                     __syncwarp();
                     const int sv = tg % VST;
                     if (!warp_wait(&bars->v_empty[sv], ((tg / VST) & 1) ^ 1, p.limit_ns,
@@ -575,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (lane == 0) ptx::mbar_arrive_expect_tx(&bars->v_full[sv], kTileBytes);
                     __syncwarp();
-                    load_tile(smem + L::kV + sv * kTileBytes, &tm_v, &bars->v_full[sv]);
+                    load_v(smem + L::kV + sv * kTileBytes, &bars->v_full[sv]);
                     __syncwarp();
                     if (j == 0) {
                         // look the next piece up while this one's tiles stream in
@@ -609,7 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             return ok;
         };
         const uint64_t k_desc0 = ptx::sdesc_sw128(sbase + L::kK, 16, 1024);
-        const uint64_t v_desc0 = ptx::sdesc_sw128(sbase + L::kV, kBlockBytes, 1024);
+        // V: 64-column blocks of a run 2^sub_shift rows apart, 8-row groups 1024 B
+        const uint64_t v_desc0 = ptx::sdesc_sw128(sbase + L::kV, 128u << sub_shift, 1024);
         constexpr uint64_t kTileUnits = kTileBytes >> 4;
         auto issue_s = [&](int t) {
             if (!wait_or_fail(&bars->k_full[t % KST], (t / KST) & 1, 6)) return;
@@ -657,7 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < kBlockN / 16; ++kk)
                     ptx::umma_ts_elect(tmem + kColO, a_p + kk * 8,
-                                       vd + (uint64_t)((kk * 16 * 128) >> 4), kIdescO,
+                                       vd + (uint64_t)(v_row(kk * 16) >> 4), kIdescO,
                                        kk > 0 ? 1u : acc0);
                 ptx::umma_commit_elect(&bars->o_done);
                 if (j == nt - 1) ptx::umma_commit_elect(&bars->o_final);
@@ -856,12 +875,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     if (key_begin + j * kBlockN + (int)row >= key_end) {
-                        uint8_t* vt = smem + L::kV + sv * kTileBytes;
+                        uint8_t* vt = smem + L::kV + sv * kTileBytes + v_row((int)row);
 #pragma unroll
                         for (int c = 0; c < kDBlocks; ++c)
 #pragma unroll
                             for (int ch = 0; ch < 8; ++ch)
-                                *reinterpret_cast<uint4*>(vt + c * kBlockBytes + row * 128 +
+                                *reinterpret_cast<uint4*>(vt + (c * 128u << sub_shift) +
                                                           ch * 16) = make_uint4(0, 0, 0, 0);
                     }
                     ptx::fence_proxy_async_smem();
