@@ -1,6 +1,5 @@
 """The C-ABI library loads without a GPU and exports what include/attn.h
 declares; host-side validation rejects bad arguments before any CUDA call."""
-import ctypes
 import os
 import subprocess
 

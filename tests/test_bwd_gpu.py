@@ -5,7 +5,6 @@ everything from the same stored q, k, v, dO bits.  Gradients and the
 workspace are guarded and NaN/junk-filled (tests/parity.py); the BERT-large
 shape is compared in full and the bench's shape (B=4, H=16, N=4096, d=128)
 on 16 of its 64 (batch, head) pairs, against the matrix-product oracle."""
-import numpy as np
 import pytest
 import torch
 

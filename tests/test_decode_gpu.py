@@ -1,6 +1,5 @@
 """KV-cache decode kernel (split-K over a packed variable-length cache)
 against the fp64 oracle."""
-import numpy as np
 import pytest
 import torch
 

@@ -8,13 +8,11 @@ random rows per head plus rows 0, 1, 127, 128 and N - 1, in the launch
 configuration the bench times.  Outputs are written into guarded, NaN-filled
 buffers (tests/parity.py: run_fwd).
 """
-import math
 
 import numpy as np
 import pytest
 import torch
 
-import oracle
 from oracle import dense
 from io_aware_exact_29_b200 import attn
 from io_aware_exact_29_b200.workloads import FWD_CASES, FwdCase, default_scale, fwd_inputs

@@ -2,7 +2,6 @@
 oracle: block sizes below, at and above the 128-key tile, shuffled physical
 blocks with NaN in every unused row, and the fused append of the new tokens'
 K/V.  Outputs and the workspace are guarded and NaN/junk-filled (tests/parity.py)."""
-import numpy as np
 import pytest
 import torch
 

@@ -2,7 +2,6 @@
 oracle with the same window: windows inside one key tile, across tile edges
 and wider than the keys, causal and not, ragged sizes, key padding, GQA and
 both head sizes."""
-import numpy as np
 import pytest
 import torch
 
